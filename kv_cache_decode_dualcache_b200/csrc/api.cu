@@ -1,0 +1,1143 @@
+// Host side of the decoder: context, weight layout, the forward pass over a
+// contiguous range of rows, the block-wise decode loop and the C ABI.
+//
+// One forward covers rows [r0, r0 + M) of the sequence and attends over keys
+// [0, L) taken from the paged KV cache (its own rows are written there first,
+// by the QKV epilogue):
+//   block-start refresh / cache-off step   r0 = 0, M = L
+//   DualCache block step                   r0 = s, M = block
+//   prefix-cache step                      r0 = s, M = L - s
+// The LM head then runs on `n_lm` rows starting at row `lm0` of the forward
+// and a single-CTA kernel merges its partials and applies the unmask rule.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/fdllm.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace fd;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+const int kNtChoices[3] = {64, 128, 256};   // token-tile rows (two-term: rows/2 tokens)
+constexpr size_t kWorkspaceBytes = 64ull << 20;
+constexpr int kMaxLmRows = 256;
+constexpr int kMaxAttnSplit = 16;
+constexpr int kAttnSplitMaxM = 64;
+
+thread_local std::string g_create_error = "no error";
+
+struct LayerW {
+  void* wqkv = nullptr;
+  void* wo = nullptr;
+  void* wgu = nullptr;
+  void* wd = nullptr;
+  float* attn_norm = nullptr;
+  float* ffn_norm = nullptr;
+  CUtensorMap m_qkv, m_o, m_gu, m_d;
+};
+
+int nt_index(int nt) {
+  for (int i = 0; i < 3; ++i)
+    if (kNtChoices[i] == nt) return i;
+  return -1;
+}
+
+// Rows of a two-term activation matrix holding `tokens` tokens.
+size_t pair_rows(size_t tokens) { return 2 * ((tokens + 31) / 32) * 32; }
+
+}  // namespace
+
+struct fdllm_ctx {
+  fdllm_config cfg{};
+  int device = 0;
+  cudaStream_t stream = nullptr;
+  bool own_stream = false;
+  fdllm_allocator alloc{};
+  bool custom_alloc = false;
+  std::string err = "no error";
+  std::vector<void*> allocations;
+  bool weights_loaded = false;
+  int num_sms = 0;
+  bool tc = false;          // bf16 model on tensor cores
+  int f32 = 0;              // fp32 model
+  size_t esz = 2;           // bytes per weight / activation element
+  EncodeTiledFn encode = nullptr;
+
+  void* weights = nullptr;
+  void* embed = nullptr;
+  void* lm_head = nullptr;
+  float* final_norm = nullptr;
+  std::vector<LayerW> layers;
+  CUtensorMap m_head;
+
+  void* kv_pool = nullptr;
+  int kv_planes = 2;        // fp32: K, V; bf16: K hi, K lo, V hi, V lo
+  int n_pages = 0;
+  size_t q_plane = 0;       // elements per q plane (bf16 two-term q)
+  int* page_table = nullptr;
+  float2* rope = nullptr;
+  int* x = nullptr;
+  float* h = nullptr;
+  void* a = nullptr;
+  void* q = nullptr;
+  void* o = nullptr;
+  void* f = nullptr;
+  float* ws = nullptr;
+  int* counters = nullptr;
+  int n_counters = 0;
+  float* attn_po = nullptr;
+  float* attn_ml = nullptr;
+  float* lm_part = nullptr;
+  size_t lm_part_cap = 0;   // SoftmaxState entries
+  float* conf = nullptr;
+  int* tok = nullptr;
+  uint8_t* unmask = nullptr;
+  float* dbg = nullptr;
+  size_t dbg_cap = 0;
+  DecodeState* state = nullptr;
+  DecodeState* state_host = nullptr;
+  int* err_dev = nullptr;
+  int* err_host = nullptr;
+  int* check = nullptr;        // self-check record (FDLLM_CHECKS builds)
+  size_t cap_h = 0, cap_q = 0, cap_kv = 0, cap_f = 0;
+  CUtensorMap m_a[3], m_o[3], m_f[3];
+  std::map<std::tuple<int, int, int, int>, GemmShape> plans;
+  int64_t launches = 0;
+  // per-kernel-class timing (fdllm_profile_enable)
+  struct ProfPending {
+    cudaEvent_t a, b;
+    int cls;
+    double bytes, flops;
+  };
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<ProfPending> prof_pending;
+  std::vector<fdllm_kernel_stat> prof_stats;
+};
+
+namespace {
+
+int fail(fdllm_ctx* c, int code, const std::string& msg) {
+  if (c) c->err = msg; else g_create_error = msg;
+  return code;
+}
+
+int prof_class(fdllm_ctx* ctx, const std::string& name) {
+  for (size_t i = 0; i < ctx->prof_stats.size(); ++i)
+    if (name == ctx->prof_stats[i].name) return (int)i;
+  fdllm_kernel_stat st{};
+  std::snprintf(st.name, sizeof(st.name), "%s", name.c_str());
+  ctx->prof_stats.push_back(st);
+  return (int)ctx->prof_stats.size() - 1;
+}
+
+cudaEvent_t prof_event(fdllm_ctx* ctx) {
+  if (!ctx->ev_pool.empty()) {
+    cudaEvent_t e = ctx->ev_pool.back();
+    ctx->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) e = nullptr;
+  return e;
+}
+
+// Bracket one launch with events when profiling is on.
+struct ProfScope {
+  fdllm_ctx* ctx;
+  cudaEvent_t a = nullptr;
+  int cls = -1;
+  double bytes, flops;
+  ProfScope(fdllm_ctx* c, const std::string& name, double by, double fl)
+      : ctx(c), bytes(by), flops(fl) {
+    if (!ctx->prof) return;
+    a = prof_event(ctx);
+    if (!a) return;
+    cls = prof_class(ctx, name);
+    cudaEventRecord(a, ctx->stream);
+  }
+  ~ProfScope() {
+    if (!ctx->prof || !a) return;
+    cudaEvent_t b = prof_event(ctx);
+    if (!b) { ctx->ev_pool.push_back(a); return; }
+    cudaEventRecord(b, ctx->stream);
+    ctx->prof_pending.push_back({a, b, cls, bytes, flops});
+  }
+};
+
+// Called after the stream has been synchronised.
+void prof_harvest(fdllm_ctx* ctx) {
+  for (auto& p : ctx->prof_pending) {
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+      fdllm_kernel_stat& st = ctx->prof_stats[p.cls];
+      st.launches += 1;
+      st.total_ms += ms;
+      st.bytes += p.bytes;
+      st.flops += p.flops;
+    }
+    ctx->ev_pool.push_back(p.a);
+    ctx->ev_pool.push_back(p.b);
+  }
+  ctx->prof_pending.clear();
+}
+
+#define CK(call)                                                                       \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(ctx, FDLLM_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+#define KL(call)                                                                       \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    ++ctx->launches;                                                                   \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(ctx, FDLLM_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+void* dalloc(fdllm_ctx* ctx, size_t bytes) {
+  if (bytes == 0) bytes = 256;
+  bytes = (bytes + 255) & ~(size_t)255;
+  void* p = nullptr;
+  if (ctx->custom_alloc) {
+    p = ctx->alloc.alloc(bytes, ctx->alloc.user);
+  } else if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    p = nullptr;
+  }
+  if (p) ctx->allocations.push_back(p);
+  return p;
+}
+
+void dfree_all(fdllm_ctx* ctx) {
+  for (void* p : ctx->allocations) {
+    if (ctx->custom_alloc) ctx->alloc.free(p, ctx->alloc.user);
+    else cudaFree(p);
+  }
+  ctx->allocations.clear();
+}
+
+bool make_map(fdllm_ctx* ctx, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int check_config(const fdllm_config* c, std::string* why) {
+  auto bad = [&](const char* m) { *why = m; return FDLLM_ERR_ARG; };
+  if (!c) return bad("config is NULL");
+  if (c->n_layers < 1) return bad("n_layers must be >= 1");
+  if (c->d_model < 64 || c->d_model % 64) return bad("d_model must be a positive multiple of 64");
+  if (c->ffn_dim < 64 || c->ffn_dim % 64) return bad("ffn_dim must be a positive multiple of 64");
+  if (!(c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 128))
+    return bad("head_dim must be 32, 64 or 128");
+  if (c->n_heads < 1 || c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads)
+    return bad("n_heads must be a positive multiple of n_kv_heads");
+  if ((c->n_heads * c->head_dim) % 64) return bad("n_heads * head_dim must be a multiple of 64");
+  if (c->vocab < 2) return bad("vocab must be >= 2");
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) return bad("mask_id must be in [0, vocab)");
+  if (!(c->dtype == FDLLM_DTYPE_F32 || c->dtype == FDLLM_DTYPE_BF16)) return bad("unknown dtype");
+  if (c->dtype == FDLLM_DTYPE_BF16 && c->head_dim == 32)
+    return bad("the bf16 attention kernel needs head_dim 64 or 128");
+  if (c->max_batch != 1) return bad("max_batch must be 1");
+  if (c->max_seq < 1 || c->max_seq > (1 << 20)) return bad("max_seq out of range");
+  if (!(c->rms_eps >= 0.0f) || !std::isfinite(c->rope_theta) || !(c->rope_theta > 0.0f) ||
+      !std::isfinite(c->logit_scale))
+    return bad("rope_theta, rms_eps and logit_scale must be finite (theta > 0, eps >= 0)");
+  return FDLLM_OK;
+}
+
+// --------------------------------------------------------------- GEMM plan
+// fp32 model: CUDA-core tiles of 128 features x 32 tokens.  bf16 model:
+// token tile of nt rows (nt/2 tokens, two-term), the K split chosen to
+// balance the per-CTA K blocks over the persistent grid (deterministic
+// reduction of the splits).  Plans are memoised per shape.
+GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split) {
+  GemmShape g{};
+  g.N = N;
+  g.M = M;
+  g.K = K;
+  g.n_tiles = (N + 127) / 128;
+  g.kb_total = (K + 63) / 64;
+  if (!ctx->tc) {
+    g.nt = 32;
+    g.splits = 1;
+    g.n_tt = (M + 31) / 32;
+    g.units = g.n_tiles * g.n_tt;
+    g.grid = g.units;
+    return g;
+  }
+  int nt = 64;
+  while (nt / 2 < M && nt < 256) nt *= 2;
+  g.nt = nt;
+  g.n_tt = (M + nt / 2 - 1) / (nt / 2);
+  const int base_units = g.n_tiles * g.n_tt;
+  const int max_split = allow_split ? std::min(16, std::max(1, g.kb_total / 4)) : 1;
+  double best = 1e300;
+  int best_s = 1;
+  for (int s = 1; s <= max_split; ++s) {
+    const long long units = (long long)base_units * s;
+    if (s > 1 && (size_t)units * (nt / 2) * 128 * sizeof(float) > kWorkspaceBytes) break;
+    const int grid = (int)std::min<long long>(units, ctx->num_sms);
+    // per-CTA cost in K blocks of its units, +2 per unit (pipeline fill and
+    // epilogue), +1 per unit when split (partial tile write and reduction)
+    std::vector<double> load(grid, 0.0);
+    for (long long u = 0; u < units; ++u) {
+      const int sp = (int)(u % s);
+      const int kb = (int)((long long)(sp + 1) * g.kb_total / s - (long long)sp * g.kb_total / s);
+      load[u % grid] += kb + 2.0 + (s > 1 ? 1.0 : 0.0);
+    }
+    double mx = 0.0;
+    for (double v : load) mx = std::max(mx, v);
+    if (mx < best * 0.995) {
+      best = mx;
+      best_s = s;
+    }
+  }
+  g.splits = best_s;
+  g.units = base_units * best_s;
+  g.grid = std::min(g.units, ctx->num_sms);
+  return g;
+}
+
+GemmShape plan_gemm(fdllm_ctx* ctx, int N, int M, int K, bool allow_split) {
+  const auto key = std::make_tuple(N, M, K, allow_split ? 1 : 0);
+  auto it = ctx->plans.find(key);
+  if (it != ctx->plans.end()) return it->second;
+  GemmShape g = make_plan(ctx, N, M, K, allow_split);
+  ctx->plans[key] = g;
+  return g;
+}
+
+const CUtensorMap* act_map(CUtensorMap* maps, int nt) { return &maps[nt_index(nt)]; }
+
+int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* wmap,
+             const void* act, CUtensorMap* amaps, int act_row0, int N, int M, int K,
+             const EpiParams& ep_in, int* n_part_out = nullptr) {
+  const bool lm = ep_in.kind == EPI_LMHEAD;
+  GemmShape gs = plan_gemm(ctx, N, M, K, !lm);
+  EpiParams ep = ep_in;
+  ep.N = N;
+  ep.M = M;
+  ep.act_f32 = ctx->f32;
+  if (lm && (size_t)gs.grid * M > ctx->lm_part_cap)
+    return fail(ctx, FDLLM_ERR_CUDA, "LM-head partial buffer too small");
+  if (gs.n_tiles * gs.n_tt > ctx->n_counters)
+    return fail(ctx, FDLLM_ERR_CUDA, "split-K counter buffer too small");
+  const double es = (double)ctx->esz;
+  double out_bytes = 0.0;
+  switch (ep.kind) {
+    case EPI_QKV: out_bytes = (double)M * N * es; break;
+    case EPI_RESID: out_bytes = 2.0 * M * N * 4.0; break;
+    case EPI_SWIGLU: out_bytes = (double)M * (N / 2) * es; break;
+    case EPI_STORE: out_bytes = (double)M * N * 4.0; break;
+    default: break;
+  }
+  ProfScope ps(ctx, std::string("gemm.") + tag + (M <= 64 ? ".step" : ".full"),
+               (double)N * K * es + (double)M * K * es + out_bytes, 2.0 * M * N * K);
+  if (ctx->tc) {
+    GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
+                   ctx->n_counters};
+    KL(launch_gemm_tc(wmap, act_map(amaps, gs.nt), gs, ep, sc, ctx->stream));
+  } else {
+    KL(launch_gemm_simt((const float*)w, (const float*)act, act_row0, K, gs, ep, ctx->stream));
+  }
+  if (n_part_out) *n_part_out = gs.grid;
+  return FDLLM_OK;
+}
+
+EpiParams epi_base(fdllm_ctx* ctx, int kind) {
+  EpiParams ep{};
+  ep.kind = kind;
+  ep.check = ctx->check;
+  ep.cap_h = ctx->cap_h;
+  ep.cap_q = ctx->cap_q;
+  ep.cap_kv = ctx->cap_kv;
+  ep.cap_f = ctx->cap_f;
+  ep.cap_dbg = ctx->dbg_cap;
+  ep.cap_lm = ctx->lm_part_cap;
+  ep.kv_pool = ctx->kv_pool;
+  ep.kv_planes = ctx->kv_planes;
+  ep.q_plane = ctx->q_plane;
+  ep.page_table = ctx->page_table;
+  ep.n_pages = ctx->n_pages;
+  ep.rope = ctx->rope;
+  ep.n_heads = ctx->cfg.n_heads;
+  ep.n_kv_heads = ctx->cfg.n_kv_heads;
+  ep.head_dim = ctx->cfg.head_dim;
+  ep.logit_scale = ctx->cfg.logit_scale;
+  ep.mask_id = ctx->cfg.mask_id;
+  return ep;
+}
+
+int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullptr,
+                  void* o = nullptr) {
+  const fdllm_config& c = ctx->cfg;
+  AttnParams ap{};
+  ap.q = q ? q : ctx->q;
+  ap.q_plane = q ? (size_t)M * c.n_heads * c.head_dim : ctx->q_plane;
+  ap.o = o ? o : ctx->o;
+  ap.kv_pool = ctx->kv_pool;
+  ap.kv_planes = ctx->kv_planes;
+  ap.page_table = ctx->page_table;
+  ap.n_pages = ctx->n_pages;
+  ap.layer = layer;
+  ap.M = M;
+  ap.L = L;
+  ap.n_heads = c.n_heads;
+  ap.n_kv_heads = c.n_kv_heads;
+  ap.head_dim = c.head_dim;
+  ap.part_o = ctx->attn_po;
+  ap.part_ml = ctx->attn_ml;
+  ap.n_split = 1;
+  ap.keys_per_split = ((L + 63) / 64) * 64;
+  const double es = (double)ctx->esz;
+  const double kv_bytes = (double)ctx->kv_planes * L * c.n_kv_heads * c.head_dim * es;
+  const double qo_bytes = (ctx->f32 ? 2.0 : 4.0) * M * c.n_heads * c.head_dim * es;
+  const double att_flops = 4.0 * M * c.n_heads * (double)L * c.head_dim;
+  const std::string att_tag = M <= 64 ? "attn.step" : "attn.full";
+  if (!ctx->tc) {
+    ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
+    KL(launch_attn_simt(ap, ctx->stream));
+    return FDLLM_OK;
+  }
+  const int rep = c.n_heads / c.n_kv_heads;
+  const int ctas = ((M * rep + 63) / 64) * c.n_kv_heads;
+  const int key_tiles = (L + 63) / 64;
+  if (M <= kAttnSplitMaxM) {
+    int want = std::max(1, (2 * ctx->num_sms) / std::max(1, ctas));
+    want = std::min(want, std::min(kMaxAttnSplit, key_tiles));
+    const int tiles_per = (key_tiles + want - 1) / want;
+    ap.keys_per_split = tiles_per * 64;
+    ap.n_split = (key_tiles + tiles_per - 1) / tiles_per;
+  }
+  {
+    const double part = ap.n_split > 1 ? (double)ap.n_split * M * c.n_heads * c.head_dim * 4.0 : 0;
+    ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes + part, att_flops);
+    KL(launch_attn_mma(ap, ctx->stream));
+  }
+  if (ap.n_split > 1) {
+    ProfScope ps(ctx, "attn.combine", (double)ap.n_split * M * c.n_heads * c.head_dim * 4.0 +
+                                          qo_bytes / 2, 0.0);
+    KL(launch_attn_combine(ap, ctx->f32, ctx->stream));
+  }
+  return FDLLM_OK;
+}
+
+// Forward over rows [r0, r0+M) with keys [0, L); LM head on rows
+// [lm0, lm0+n_lm) of the forward.  Returns the number of LM partials.
+int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg, int* n_part) {
+  const fdllm_config& c = ctx->cfg;
+  const int d = c.d_model, hq = c.n_heads * c.head_dim, hkv = c.n_kv_heads * c.head_dim;
+  const int nqkv = hq + 2 * hkv;
+  const double es = (double)ctx->esz;
+  {
+    ProfScope ps(ctx, "embed_rmsnorm", (double)M * d * (2.0 * es + 4.0), 0.0);
+    KL(launch_embed_rmsnorm(ctx->x, r0, M, ctx->embed, d, c.vocab, ctx->layers[0].attn_norm,
+                            c.rms_eps, ctx->h, ctx->a, ctx->f32, ctx->err_dev, ctx->stream));
+  }
+  int rc;
+  for (int l = 0; l < c.n_layers; ++l) {
+    LayerW& lw = ctx->layers[l];
+    EpiParams ep = epi_base(ctx, EPI_QKV);
+    ep.q_out = ctx->q;
+    ep.layer = l;
+    ep.pos0 = r0;
+    if ((rc = run_gemm(ctx, "qkv", lw.wqkv, &lw.m_qkv, ctx->a, ctx->m_a, 0, nqkv, M, d, ep))) return rc;
+    if ((rc = run_attention(ctx, l, M, L))) return rc;
+    ep = epi_base(ctx, EPI_RESID);
+    ep.h = ctx->h;
+    if ((rc = run_gemm(ctx, "o", lw.wo, &lw.m_o, ctx->o, ctx->m_o, 0, d, M, hq, ep))) return rc;
+    {
+      ProfScope ps(ctx, "rmsnorm", (double)M * d * (es + 4.0), 0.0);
+      KL(launch_rmsnorm(ctx->h, 0, M, d, lw.ffn_norm, c.rms_eps, ctx->a, ctx->f32, ctx->stream));
+    }
+    ep = epi_base(ctx, EPI_SWIGLU);
+    ep.f_out = ctx->f;
+    if ((rc = run_gemm(ctx, "ffn_up", lw.wgu, &lw.m_gu, ctx->a, ctx->m_a, 0, 2 * c.ffn_dim, M, d, ep)))
+      return rc;
+    ep = epi_base(ctx, EPI_RESID);
+    ep.h = ctx->h;
+    if ((rc = run_gemm(ctx, "ffn_down", lw.wd, &lw.m_d, ctx->f, ctx->m_f, 0, d, M, c.ffn_dim, ep))) return rc;
+    // next layer's attention norm over all rows, or the final norm over the
+    // LM-head rows only (written to rows [0, n_lm) of the activation buffer)
+    const bool last = l + 1 == c.n_layers;
+    const int nr = last ? n_lm : M;
+    {
+      ProfScope ps(ctx, "rmsnorm", (double)nr * d * (es + 4.0), 0.0);
+      KL(launch_rmsnorm(ctx->h, last ? lm0 : 0, nr, d,
+                        last ? ctx->final_norm : ctx->layers[l + 1].attn_norm, c.rms_eps, ctx->a,
+                        ctx->f32, ctx->stream));
+    }
+  }
+  EpiParams ep = epi_base(ctx, EPI_LMHEAD);
+  ep.lm_part = ctx->lm_part;
+  ep.dbg_logits = dbg;
+  return run_gemm(ctx, "lm_head", ctx->lm_head, &ctx->m_head, ctx->a, ctx->m_a, 0, c.vocab, n_lm,
+                  d, ep, n_part);
+}
+
+int sync_state(fdllm_ctx* ctx) {
+  CK(cudaMemcpyAsync(ctx->state_host, ctx->state, sizeof(DecodeState), cudaMemcpyDeviceToHost,
+                     ctx->stream));
+  CK(cudaMemcpyAsync(ctx->err_host, ctx->err_dev, sizeof(int), cudaMemcpyDeviceToHost,
+                     ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  if (!ctx->prof_pending.empty()) prof_harvest(ctx);
+#ifdef FDLLM_CHECKS
+  {
+    int chk[4] = {0, 0, 0, 0};
+    CK(cudaMemcpy(chk, ctx->check, sizeof(chk), cudaMemcpyDeviceToHost));
+    if (chk[0]) {
+      const int zero4[4] = {0, 0, 0, 0};
+      cudaMemcpy(ctx->check, zero4, sizeof(zero4), cudaMemcpyHostToDevice);
+      return fail(ctx, FDLLM_ERR_CUDA,
+                  "device self-check failed: " + std::to_string(chk[0]) + " violations, first code " +
+                      std::to_string(chk[1]) + " index " + std::to_string(chk[2]) + " limit " +
+                      std::to_string(chk[3]));
+    }
+  }
+#endif
+  const int e = *ctx->err_host;
+  if (e) {
+    int zero = 0;
+    cudaMemcpy(ctx->err_dev, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e & DEV_ERR_TIMEOUT)
+      return fail(ctx, FDLLM_ERR_TIMEOUT, "a device-side wait timed out; results are invalid");
+    if (e & DEV_ERR_TOKEN)
+      return fail(ctx, FDLLM_ERR_ARG, "a token id is out of range or the prompt holds the mask id");
+    return fail(ctx, FDLLM_ERR_CUDA, "device kernel reported an error");
+  }
+  return FDLLM_OK;
+}
+
+// One denoising step: forward for the mode + merge/select.  first = block start.
+int run_step(fdllm_ctx* ctx, int mode, bool first, int s, int B, int L, float tau, float* dbg) {
+  int n_part = 0, rc;
+  if (first || mode == FDLLM_CACHE_NONE) {
+    rc = forward(ctx, 0, L, L, s, B, dbg, &n_part);
+  } else if (mode == FDLLM_CACHE_DUAL) {
+    rc = forward(ctx, s, B, L, 0, B, dbg, &n_part);
+  } else {
+    rc = forward(ctx, s, L - s, L, 0, B, dbg, &n_part);
+  }
+  if (rc) return rc;
+  ProfScope ps(ctx, "merge_select", (double)n_part * B * 12.0, 0.0);
+  KL(launch_merge_select(ctx->lm_part, n_part, B, ctx->x, s, ctx->cfg.mask_id, tau, 1, ctx->conf,
+                         ctx->tok, ctx->unmask, ctx->state, ctx->stream));
+  return FDLLM_OK;
+}
+
+int check_gen_args(fdllm_ctx* ctx, int prompt_len, int gen_len, int block_size, float tau,
+                   int cache_mode) {
+  if (!ctx->weights_loaded) return fail(ctx, FDLLM_ERR_STATE, "weights are not loaded");
+  if (gen_len < 1 || block_size < 1 || gen_len % block_size)
+    return fail(ctx, FDLLM_ERR_ARG, "gen_len and block_size must be >= 1 with gen_len % block_size == 0");
+  if (block_size > kMaxLmRows) return fail(ctx, FDLLM_ERR_ARG, "block_size must be <= 256");
+  if (prompt_len < 0 || (long long)prompt_len + gen_len > ctx->cfg.max_seq)
+    return fail(ctx, FDLLM_ERR_ARG, "prompt_len + gen_len exceeds max_seq (or prompt_len < 0)");
+  if (std::isnan(tau)) return fail(ctx, FDLLM_ERR_ARG, "tau is NaN");
+  if (cache_mode < FDLLM_CACHE_NONE || cache_mode > FDLLM_CACHE_DUAL)
+    return fail(ctx, FDLLM_ERR_ARG, "unknown cache_mode");
+  return FDLLM_OK;
+}
+
+int generate_impl(fdllm_ctx* ctx, const int32_t* prompt, bool prompt_dev, int P, int G, int B,
+                  float tau, int mode, int32_t* out, bool out_dev, int* out_steps,
+                  fdllm_stats* stats) {
+  int rc = check_gen_args(ctx, P, G, B, tau, mode);
+  if (rc) return rc;
+  if (!out || !out_steps) return fail(ctx, FDLLM_ERR_ARG, "NULL output pointer");
+  if (P > 0 && !prompt) return fail(ctx, FDLLM_ERR_ARG, "NULL prompt");
+  const fdllm_config& c = ctx->cfg;
+  if (!prompt_dev) {
+    for (int i = 0; i < P; ++i)
+      if (prompt[i] < 0 || prompt[i] >= c.vocab || prompt[i] == c.mask_id)
+        return fail(ctx, FDLLM_ERR_ARG, "prompt id out of range or equal to the mask id");
+  }
+  CK(cudaSetDevice(ctx->device));
+  const int L = P + G;
+  if (P > 0)
+    CK(cudaMemcpyAsync(ctx->x, prompt, sizeof(int32_t) * P,
+                       prompt_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                       ctx->stream));
+  if (prompt_dev) KL(launch_check_prompt(ctx->x, P, c.vocab, c.mask_id, ctx->err_dev, ctx->stream));
+  KL(launch_fill_masked(ctx->x, P, L, c.mask_id, ctx->stream));
+  CK(cudaMemsetAsync(ctx->state, 0, sizeof(DecodeState), ctx->stream));
+  const int n_blocks = G / B;
+  int total = 0, refresh = 0, cached = 0;
+  double refresh_ms = 0, cached_ms = 0;
+  const bool timing = stats && stats->collect_timing;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (timing) {
+    CK(cudaEventCreate(&e0));
+    CK(cudaEventCreate(&e1));
+  }
+  for (int b = 0; b < n_blocks; ++b) {
+    const int s = P + b * B;
+    int nb = 0;
+    bool first = true;
+    for (;;) {
+      if (timing) CK(cudaEventRecord(e0, ctx->stream));
+      if ((rc = run_step(ctx, mode, first, s, B, L, tau, nullptr))) return rc;
+      if (timing) CK(cudaEventRecord(e1, ctx->stream));
+      if ((rc = sync_state(ctx))) return rc;
+      const bool full = first || mode == FDLLM_CACHE_NONE;
+      if (timing) {
+        float ms = 0;
+        CK(cudaEventElapsedTime(&ms, e0, e1));
+        (full ? refresh_ms : cached_ms) += ms;
+      }
+      (full ? refresh : cached) += 1;
+      first = false;
+      ++nb;
+      if (ctx->state_host->remaining == 0) break;
+      if (ctx->state_host->unmasked < 1 || nb >= B)
+        return fail(ctx, FDLLM_ERR_CUDA, "decode step made no progress");
+    }
+    total += nb;
+    if (stats && stats->steps_per_block) stats->steps_per_block[b] = nb;
+  }
+  CK(cudaMemcpyAsync(out, ctx->x + P, sizeof(int32_t) * G,
+                     out_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  if (timing) {
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+  }
+  *out_steps = total;
+  if (stats) {
+    stats->steps = total;
+    stats->refresh_steps = refresh;
+    stats->cached_steps = cached;
+    stats->n_blocks = n_blocks;
+    stats->refresh_ms = refresh_ms;
+    stats->cached_ms = cached_ms;
+  }
+  return FDLLM_OK;
+}
+
+}  // namespace
+
+// =============================================================== C ABI
+extern "C" {
+
+int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
+                 const fdllm_allocator* alloc, fdllm_ctx** out) {
+  std::string why;
+  if (!out) return fail(nullptr, FDLLM_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  int rc = check_config(cfg, &why);
+  if (rc) return fail(nullptr, rc, why);
+  if (alloc && (!alloc->alloc || !alloc->free))
+    return fail(nullptr, FDLLM_ERR_ARG, "allocator needs both alloc and free");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return fail(nullptr, FDLLM_ERR_ARG, "no such CUDA device");
+  }
+  fdllm_ctx* ctx = new fdllm_ctx();
+  ctx->cfg = *cfg;
+  ctx->device = device;
+  if (alloc) {
+    ctx->alloc = *alloc;
+    ctx->custom_alloc = true;
+  }
+  ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
+  ctx->tc = !ctx->f32;
+  ctx->esz = ctx->f32 ? 4 : 2;
+  auto bail = [&](int code, const std::string& m) {
+    g_create_error = m;
+    dfree_all(ctx);
+    if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
+    if (ctx->state_host) cudaFreeHost(ctx->state_host);
+    if (ctx->err_host) cudaFreeHost(ctx->err_host);
+    delete ctx;
+    return code;
+  };
+  if (cudaSetDevice(device) != cudaSuccess) return bail(FDLLM_ERR_CUDA, "cudaSetDevice failed");
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess)
+    return bail(FDLLM_ERR_CUDA, "cudaGetDeviceProperties failed");
+  ctx->num_sms = prop.multiProcessorCount;
+  if (ctx->tc && prop.major != 10)
+    return bail(FDLLM_ERR_ARG, "the bf16 path needs an sm_100 (B200-class) GPU");
+  if (cuda_stream) {
+    ctx->stream = static_cast<cudaStream_t>(cuda_stream);
+  } else {
+    // A blocking stream: ordered after work on the legacy default stream, so
+    // inputs a caller produced there are complete before the decoder reads them.
+    if (cudaStreamCreate(&ctx->stream) != cudaSuccess)
+      return bail(FDLLM_ERR_CUDA, "cudaStreamCreate failed");
+    ctx->own_stream = true;
+  }
+  if (ctx->tc) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess || !fn)
+      return bail(FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const fdllm_config& c = *cfg;
+  const int S = c.max_seq;
+  const int hq = c.n_heads * c.head_dim, hkv = c.n_kv_heads * c.head_dim;
+  ctx->n_pages = (S + KV_PAGE - 1) / KV_PAGE;
+  ctx->kv_planes = ctx->f32 ? 2 : 4;
+  const size_t kv_elems =
+      (size_t)c.n_layers * ctx->n_pages * ctx->kv_planes * c.n_kv_heads * KV_PAGE * c.head_dim;
+  const size_t rows = (size_t)S;
+  // activation matrices: plain rows (fp32) or two-term pair rows (bf16)
+  const size_t arows = ctx->f32 ? rows : pair_rows(rows);
+  ctx->q_plane = ctx->f32 ? 0 : rows * hq;
+  ctx->kv_pool = dalloc(ctx, kv_elems * ctx->esz);
+  ctx->page_table = (int*)dalloc(ctx, sizeof(int) * ctx->n_pages);
+  ctx->rope = (float2*)dalloc(ctx, sizeof(float2) * rows * (c.head_dim / 2));
+  ctx->x = (int*)dalloc(ctx, sizeof(int) * rows);
+  ctx->h = (float*)dalloc(ctx, sizeof(float) * rows * c.d_model);
+  ctx->a = dalloc(ctx, ctx->esz * arows * c.d_model);
+  ctx->q = dalloc(ctx, ctx->esz * rows * hq * (ctx->f32 ? 1 : 2));
+  ctx->o = dalloc(ctx, ctx->esz * arows * hq);
+  ctx->f = dalloc(ctx, ctx->esz * arows * c.ffn_dim);
+  const int max_n = std::max(std::max(c.vocab, 2 * c.ffn_dim), std::max(hq + 2 * hkv, c.d_model));
+  ctx->n_counters = ((max_n + 127) / 128) * ((S + 31) / 32);
+  ctx->counters = (int*)dalloc(ctx, sizeof(int) * ctx->n_counters);
+  if (ctx->tc) ctx->ws = (float*)dalloc(ctx, kWorkspaceBytes);
+  const size_t attn_rows = (size_t)kAttnSplitMaxM * c.n_heads;
+  ctx->attn_po = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * c.head_dim);
+  ctx->attn_ml = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * 2);
+  const size_t max_parts = std::max<size_t>((size_t)ctx->num_sms,
+                                            (size_t)((c.vocab + 127) / 128) * ((kMaxLmRows + 31) / 32));
+  ctx->lm_part_cap = max_parts * kMaxLmRows;
+  ctx->lm_part = (float*)dalloc(ctx, sizeof(SoftmaxState) * ctx->lm_part_cap);
+  ctx->conf = (float*)dalloc(ctx, sizeof(float) * kMaxLmRows);
+  ctx->tok = (int*)dalloc(ctx, sizeof(int) * kMaxLmRows);
+  ctx->unmask = (uint8_t*)dalloc(ctx, kMaxLmRows);
+  ctx->state = (DecodeState*)dalloc(ctx, sizeof(DecodeState));
+  ctx->err_dev = (int*)dalloc(ctx, sizeof(int));
+  ctx->check = (int*)dalloc(ctx, 4 * sizeof(int));
+  ctx->cap_h = rows * c.d_model;
+  ctx->cap_q = ctx->esz == 4 ? rows * hq : 2 * rows * hq;
+  ctx->cap_kv = kv_elems;
+  ctx->cap_f = arows * c.ffn_dim;
+  for (void* p : {(void*)ctx->kv_pool, (void*)ctx->page_table, (void*)ctx->rope, (void*)ctx->x,
+                  (void*)ctx->h, ctx->a, ctx->q, ctx->o, ctx->f, (void*)ctx->counters,
+                  (void*)ctx->attn_po, (void*)ctx->attn_ml, (void*)ctx->lm_part,
+                  (void*)ctx->conf, (void*)ctx->tok, (void*)ctx->unmask, (void*)ctx->state,
+                  (void*)ctx->err_dev, (void*)ctx->check})
+    if (!p) return bail(FDLLM_ERR_OOM, "device allocation failed");
+  if (ctx->tc && !ctx->ws) return bail(FDLLM_ERR_OOM, "device allocation failed");
+  if (cudaMallocHost(&ctx->state_host, sizeof(DecodeState)) != cudaSuccess ||
+      cudaMallocHost(&ctx->err_host, sizeof(int)) != cudaSuccess)
+    return bail(FDLLM_ERR_OOM, "pinned host allocation failed");
+  // page table (identity for one sequence), RoPE table (angles in double)
+  std::vector<int> pt(ctx->n_pages);
+  for (int i = 0; i < ctx->n_pages; ++i) pt[i] = i;
+  const int half = c.head_dim / 2;
+  std::vector<float2> rt(rows * half);
+  for (size_t p = 0; p < rows; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double inv = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
+      const double ang = (double)p * inv;
+      rt[p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  bool ok = cudaMemcpy(ctx->page_table, pt.data(), sizeof(int) * pt.size(),
+                       cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemcpy(ctx->rope, rt.data(), sizeof(float2) * rt.size(),
+                       cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemset(ctx->counters, 0, sizeof(int) * ctx->n_counters) == cudaSuccess &&
+            cudaMemset(ctx->err_dev, 0, sizeof(int)) == cudaSuccess &&
+            cudaMemset(ctx->check, 0, 4 * sizeof(int)) == cudaSuccess &&
+            cudaMemset(ctx->kv_pool, 0, kv_elems * ctx->esz) == cudaSuccess &&
+            cudaMemset(ctx->a, 0, ctx->esz * arows * c.d_model) == cudaSuccess &&
+            cudaMemset(ctx->o, 0, ctx->esz * arows * hq) == cudaSuccess &&
+            cudaMemset(ctx->f, 0, ctx->esz * arows * c.ffn_dim) == cudaSuccess;
+  if (!ok) return bail(FDLLM_ERR_CUDA, "initialising device buffers failed");
+  if (ctx->tc) {
+    for (int i = 0; i < 3; ++i) {
+      const int nt = kNtChoices[i];
+      if (!make_map(ctx, &ctx->m_a[i], ctx->a, arows, c.d_model, nt) ||
+          !make_map(ctx, &ctx->m_o[i], ctx->o, arows, hq, nt) ||
+          !make_map(ctx, &ctx->m_f[i], ctx->f, arows, c.ffn_dim, nt))
+        return bail(FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation buffer");
+    }
+  }
+  *out = ctx;
+  return FDLLM_OK;
+}
+
+int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensors) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (!tensors || n_tensors < 1) return fail(ctx, FDLLM_ERR_ARG, "no tensors");
+  if (ctx->weights_loaded) return fail(ctx, FDLLM_ERR_STATE, "weights are already loaded");
+  const fdllm_config& c = ctx->cfg;
+  const int d = c.d_model, hd = c.head_dim, F = c.ffn_dim, V = c.vocab;
+  const int hq = c.n_heads * hd, hkv = c.n_kv_heads * hd;
+  struct Want { std::string name; int64_t numel; const fdllm_tensor* got; };
+  std::vector<Want> want;
+  want.push_back({"embed", (int64_t)V * d, nullptr});
+  for (int l = 0; l < c.n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    want.push_back({p + "attn_norm", d, nullptr});
+    want.push_back({p + "wq", (int64_t)hq * d, nullptr});
+    want.push_back({p + "wk", (int64_t)hkv * d, nullptr});
+    want.push_back({p + "wv", (int64_t)hkv * d, nullptr});
+    want.push_back({p + "wo", (int64_t)d * hq, nullptr});
+    want.push_back({p + "ffn_norm", d, nullptr});
+    want.push_back({p + "w_gate", (int64_t)F * d, nullptr});
+    want.push_back({p + "w_up", (int64_t)F * d, nullptr});
+    want.push_back({p + "w_down", (int64_t)d * F, nullptr});
+  }
+  want.push_back({"final_norm", d, nullptr});
+  want.push_back({"lm_head", (int64_t)V * d, nullptr});
+  for (int i = 0; i < n_tensors; ++i) {
+    const fdllm_tensor& t = tensors[i];
+    if (!t.name || !t.data) return fail(ctx, FDLLM_ERR_SHAPE, "tensor with NULL name or data");
+    bool found = false;
+    for (Want& w : want) {
+      if (w.name != t.name) continue;
+      if (w.got) return fail(ctx, FDLLM_ERR_SHAPE, "duplicate tensor " + w.name);
+      if (t.numel != w.numel)
+        return fail(ctx, FDLLM_ERR_SHAPE, "wrong numel for " + w.name);
+      if (t.dtype != c.dtype) return fail(ctx, FDLLM_ERR_SHAPE, "wrong dtype for " + w.name);
+      w.got = &t;
+      found = true;
+      break;
+    }
+    if (!found) return fail(ctx, FDLLM_ERR_SHAPE, std::string("unknown tensor ") + t.name);
+  }
+  for (Want& w : want)
+    if (!w.got) return fail(ctx, FDLLM_ERR_SHAPE, "missing tensor " + w.name);
+  CK(cudaSetDevice(ctx->device));
+  const size_t es = ctx->esz;
+  const size_t per_layer = ((size_t)(hq + 2 * hkv) * d + (size_t)d * hq + 2ull * F * d +
+                            (size_t)d * F) * es + 2 * sizeof(float) * d;
+  const size_t total = 2ull * V * d * es + sizeof(float) * d + c.n_layers * (per_layer + 1024);
+  uint8_t* arena = (uint8_t*)dalloc(ctx, total + 4096);
+  if (!arena) return fail(ctx, FDLLM_ERR_OOM, "weight allocation failed");
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    void* p = arena + off;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  };
+  auto find = [&](const std::string& n) {
+    for (Want& w : want) if (w.name == n) return w.got;
+    return (const fdllm_tensor*)nullptr;
+  };
+  auto copy_to = [&](void* dst, const std::string& n, size_t bytes) {
+    return cudaMemcpy(dst, find(n)->data, bytes, cudaMemcpyDefault);
+  };
+  auto norm_to = [&](float* dst, const std::string& n) -> cudaError_t {
+    const fdllm_tensor* t = find(n);
+    std::vector<float> hv(d);
+    if (ctx->f32) {
+      cudaError_t e = cudaMemcpy(hv.data(), t->data, sizeof(float) * d, cudaMemcpyDefault);
+      if (e != cudaSuccess) return e;
+    } else {
+      std::vector<uint16_t> raw(d);
+      cudaError_t e = cudaMemcpy(raw.data(), t->data, 2 * d, cudaMemcpyDefault);
+      if (e != cudaSuccess) return e;
+      for (int i = 0; i < d; ++i) {
+        uint32_t u = (uint32_t)raw[i] << 16;
+        std::memcpy(&hv[i], &u, 4);
+      }
+    }
+    return cudaMemcpy(dst, hv.data(), sizeof(float) * d, cudaMemcpyHostToDevice);
+  };
+  ctx->embed = take((size_t)V * d * es);
+  ctx->lm_head = take((size_t)V * d * es);
+  ctx->final_norm = (float*)take(sizeof(float) * d);
+  CK(copy_to(ctx->embed, "embed", (size_t)V * d * es));
+  CK(copy_to(ctx->lm_head, "lm_head", (size_t)V * d * es));
+  CK(norm_to(ctx->final_norm, "final_norm"));
+  ctx->layers.assign(c.n_layers, LayerW());
+  for (int l = 0; l < c.n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    LayerW& lw = ctx->layers[l];
+    lw.wqkv = take((size_t)(hq + 2 * hkv) * d * es);
+    lw.wo = take((size_t)d * hq * es);
+    lw.wgu = take(2ull * F * d * es);
+    lw.wd = take((size_t)d * F * es);
+    lw.attn_norm = (float*)take(sizeof(float) * d);
+    lw.ffn_norm = (float*)take(sizeof(float) * d);
+    uint8_t* qkv = (uint8_t*)lw.wqkv;
+    CK(copy_to(qkv, p + "wq", (size_t)hq * d * es));
+    CK(copy_to(qkv + (size_t)hq * d * es, p + "wk", (size_t)hkv * d * es));
+    CK(copy_to(qkv + (size_t)(hq + hkv) * d * es, p + "wv", (size_t)hkv * d * es));
+    CK(copy_to(lw.wo, p + "wo", (size_t)d * hq * es));
+    CK(copy_to(lw.wd, p + "w_down", (size_t)d * F * es));
+    // gate/up interleaved in groups of 64 rows: [g0..g63, u0..u63, g64..g127, ...]
+    const size_t grp = 64ull * d * es;
+    CK(cudaMemcpy2D(lw.wgu, 2 * grp, find(p + "w_gate")->data, grp, grp, F / 64,
+                    cudaMemcpyDefault));
+    CK(cudaMemcpy2D((uint8_t*)lw.wgu + grp, 2 * grp, find(p + "w_up")->data, grp, grp, F / 64,
+                    cudaMemcpyDefault));
+    CK(norm_to(lw.attn_norm, p + "attn_norm"));
+    CK(norm_to(lw.ffn_norm, p + "ffn_norm"));
+    if (ctx->tc) {
+      if (!make_map(ctx, &lw.m_qkv, lw.wqkv, hq + 2 * hkv, d, 128) ||
+          !make_map(ctx, &lw.m_o, lw.wo, d, hq, 128) ||
+          !make_map(ctx, &lw.m_gu, lw.wgu, 2 * F, d, 128) ||
+          !make_map(ctx, &lw.m_d, lw.wd, d, F, 128))
+        return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight");
+    }
+  }
+  if (ctx->tc && !make_map(ctx, &ctx->m_head, ctx->lm_head, V, d, 128))
+    return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for lm_head");
+  CK(cudaDeviceSynchronize());
+  ctx->weights = arena;
+  ctx->weights_loaded = true;
+  return FDLLM_OK;
+}
+
+int fdllm_generate(fdllm_ctx* ctx, const int32_t* prompt_ids, int prompt_len, int gen_len,
+                   int block_size, float tau, int cache_mode, int32_t* out_tokens,
+                   int* out_steps, fdllm_stats* stats) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  return generate_impl(ctx, prompt_ids, false, prompt_len, gen_len, block_size, tau, cache_mode,
+                       out_tokens, false, out_steps, stats);
+}
+
+int fdllm_generate_device(fdllm_ctx* ctx, const int32_t* prompt_ids_dev, int prompt_len,
+                          int gen_len, int block_size, float tau, int cache_mode,
+                          int32_t* out_tokens_dev, int* out_steps, fdllm_stats* stats) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  return generate_impl(ctx, prompt_ids_dev, true, prompt_len, gen_len, block_size, tau,
+                       cache_mode, out_tokens_dev, true, out_steps, stats);
+}
+
+int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, const int32_t* current_ids,
+                     int L, int block_start, int block_size, float tau, int cache_mode,
+                     float* logits, float* conf, int32_t* tok, uint8_t* unmask) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (!ctx->weights_loaded) return fail(ctx, FDLLM_ERR_STATE, "weights are not loaded");
+  const fdllm_config& c = ctx->cfg;
+  if (!snapshot_ids || !current_ids || !conf || !tok || !unmask)
+    return fail(ctx, FDLLM_ERR_ARG, "NULL argument");
+  if (L < 1 || L > c.max_seq || block_size < 1 || block_size > kMaxLmRows || block_start < 0 ||
+      block_start + block_size > L)
+    return fail(ctx, FDLLM_ERR_ARG, "bad L / block range");
+  if (std::isnan(tau)) return fail(ctx, FDLLM_ERR_ARG, "tau is NaN");
+  if (cache_mode < FDLLM_CACHE_NONE || cache_mode > FDLLM_CACHE_DUAL)
+    return fail(ctx, FDLLM_ERR_ARG, "unknown cache_mode");
+  for (int i = 0; i < L; ++i)
+    if (snapshot_ids[i] < 0 || snapshot_ids[i] >= c.vocab || current_ids[i] < 0 ||
+        current_ids[i] >= c.vocab)
+      return fail(ctx, FDLLM_ERR_ARG, "token id out of range");
+  CK(cudaSetDevice(ctx->device));
+  const int B = block_size, s = block_start;
+  float* dbg = nullptr;
+  if (logits) {
+    const size_t need = (size_t)B * c.vocab;
+    if (need > ctx->dbg_cap) {
+      ctx->dbg = (float*)dalloc(ctx, sizeof(float) * need);
+      if (!ctx->dbg) return fail(ctx, FDLLM_ERR_OOM, "debug logits allocation failed");
+      ctx->dbg_cap = need;
+    }
+    dbg = ctx->dbg;
+  }
+  const bool same = std::memcmp(snapshot_ids, current_ids, sizeof(int32_t) * L) == 0;
+  CK(cudaMemsetAsync(ctx->state, 0, sizeof(DecodeState), ctx->stream));
+  CK(cudaMemcpyAsync(ctx->x, snapshot_ids, sizeof(int32_t) * L, cudaMemcpyHostToDevice,
+                     ctx->stream));
+  int rc, n_part = 0;
+  if (same || cache_mode == FDLLM_CACHE_NONE) {
+    if (!same)
+      CK(cudaMemcpyAsync(ctx->x, current_ids, sizeof(int32_t) * L, cudaMemcpyHostToDevice,
+                         ctx->stream));
+    if ((rc = forward(ctx, 0, L, L, s, B, dbg, &n_part))) return rc;
+  } else {
+    if ((rc = forward(ctx, 0, L, L, s, B, nullptr, &n_part))) return rc;
+    CK(cudaMemcpyAsync(ctx->x, current_ids, sizeof(int32_t) * L, cudaMemcpyHostToDevice,
+                       ctx->stream));
+    if (cache_mode == FDLLM_CACHE_DUAL) rc = forward(ctx, s, B, L, 0, B, dbg, &n_part);
+    else rc = forward(ctx, s, L - s, L, 0, B, dbg, &n_part);
+    if (rc) return rc;
+  }
+  KL(launch_merge_select(ctx->lm_part, n_part, B, ctx->x, s, c.mask_id, tau, 1, ctx->conf,
+                         ctx->tok, ctx->unmask, ctx->state, ctx->stream));
+  if ((rc = sync_state(ctx))) return rc;
+  CK(cudaMemcpy(conf, ctx->conf, sizeof(float) * B, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(tok, ctx->tok, sizeof(int32_t) * B, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(unmask, ctx->unmask, B, cudaMemcpyDeviceToHost));
+  if (logits) CK(cudaMemcpy(logits, dbg, sizeof(float) * B * c.vocab, cudaMemcpyDeviceToHost));
+  return FDLLM_OK;
+}
+
+int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k_out, float* v_out) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  const fdllm_config& c = ctx->cfg;
+  if (layer < 0 || layer >= c.n_layers || pos0 < 0 || n < 1 || pos0 + n > c.max_seq || !k_out ||
+      !v_out)
+    return fail(ctx, FDLLM_ERR_ARG, "bad layer / position range");
+  CK(cudaSetDevice(ctx->device));
+  CK(cudaStreamSynchronize(ctx->stream));
+  const int Hkv = c.n_kv_heads, hd = c.head_dim;
+  const int P = ctx->kv_planes;
+  const size_t page_elems = (size_t)P * Hkv * KV_PAGE * hd;
+  std::vector<int> pt(ctx->n_pages);
+  CK(cudaMemcpy(pt.data(), ctx->page_table, sizeof(int) * pt.size(), cudaMemcpyDeviceToHost));
+  std::vector<uint8_t> page(page_elems * ctx->esz);
+  int cur = -1;
+  for (int i = 0; i < n; ++i) {
+    const int pos = pos0 + i;
+    const int pg = pt[pos / KV_PAGE], slot = pos % KV_PAGE;
+    if (pg != cur) {
+      const size_t off = ((size_t)layer * ctx->n_pages + pg) * page_elems * ctx->esz;
+      CK(cudaMemcpy(page.data(), (uint8_t*)ctx->kv_pool + off, page.size(),
+                    cudaMemcpyDeviceToHost));
+      cur = pg;
+    }
+    auto elem = [&](int plane, int hh, int dd) -> float {
+      const size_t e = (((size_t)plane * Hkv + hh) * KV_PAGE + slot) * hd + dd;
+      float val;
+      if (ctx->f32) {
+        std::memcpy(&val, page.data() + e * 4, 4);
+        return val;
+      }
+      uint16_t raw;
+      std::memcpy(&raw, page.data() + e * 2, 2);
+      if (plane < 2) {  // bf16 K terms
+        uint32_t u = (uint32_t)raw << 16;
+        std::memcpy(&val, &u, 4);
+        return val;
+      }
+      __half_raw hr;  // fp16 V terms
+      hr.x = raw;
+      return __half2float(__half(hr));
+    };
+    for (int hh = 0; hh < Hkv; ++hh)
+      for (int dd = 0; dd < hd; ++dd) {
+        const size_t o = ((size_t)i * Hkv + hh) * hd + dd;
+        if (ctx->f32) {
+          k_out[o] = elem(0, hh, dd);
+          v_out[o] = elem(1, hh, dd);
+        } else {  // two-term: the stored value is hi + lo
+          k_out[o] = elem(0, hh, dd) + elem(1, hh, dd);
+          v_out[o] = elem(2, hh, dd) + elem(3, hh, dd);
+        }
+      }
+  }
+  return FDLLM_OK;
+}
+
+int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
+               int K, int splits) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (!w_dev || !x_dev || !y_dev || N < 1 || M < 1 || K < 1)
+    return fail(ctx, FDLLM_ERR_ARG, "bad GEMM arguments");
+  if (ctx->tc && (K % 64 || ((uintptr_t)w_dev | (uintptr_t)x_dev) % 16))
+    return fail(ctx, FDLLM_ERR_ARG, "bf16 GEMM needs K % 64 == 0 and 16-byte aligned operands");
+  if (splits < 0 || (splits > 0 && !ctx->tc))
+    return fail(ctx, FDLLM_ERR_ARG, "bad split count");
+  CK(cudaSetDevice(ctx->device));
+  GemmShape gs = plan_gemm(ctx, N, M, K, true);
+  if (splits > 0) {
+    if (splits > gs.kb_total) return fail(ctx, FDLLM_ERR_ARG, "more splits than K blocks");
+    gs.splits = splits;
+    gs.units = gs.n_tiles * gs.n_tt * splits;
+    gs.grid = std::min(gs.units, ctx->num_sms);
+    if ((size_t)gs.units * (gs.nt / 2) * 128 * sizeof(float) > kWorkspaceBytes)
+      return fail(ctx, FDLLM_ERR_ARG, "split workspace too large");
+  }
+  if (gs.n_tiles * gs.n_tt > ctx->n_counters)
+    return fail(ctx, FDLLM_ERR_ARG, "GEMM too large for the counter buffer");
+  EpiParams ep = epi_base(ctx, EPI_STORE);
+  ep.N = N;
+  ep.M = M;
+  ep.out = y_dev;
+  ep.ld_out = N;
+  ep.cap_out = (size_t)M * N;
+  ep.act_f32 = ctx->f32;
+  if (ctx->tc) {
+    CUtensorMap wm, xm;
+    if (!make_map(ctx, &wm, w_dev, N, K, 128) ||
+        !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt))
+      return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
+                   ctx->n_counters};
+    KL(launch_gemm_tc(&wm, &xm, gs, ep, sc, ctx->stream));
+  } else {
+    KL(launch_gemm_simt((const float*)w_dev, (const float*)x_dev, 0, K, gs, ep, ctx->stream));
+  }
+  return sync_state(ctx);
+}
+
+int fdllm_attention(fdllm_ctx* ctx, const void* q_dev, void* o_dev, int layer, int M, int L) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  const fdllm_config& c = ctx->cfg;
+  if (!q_dev || !o_dev || layer < 0 || layer >= c.n_layers || M < 1 || L < 1 || L > c.max_seq)
+    return fail(ctx, FDLLM_ERR_ARG, "bad attention arguments");
+  CK(cudaSetDevice(ctx->device));
+  int rc = run_attention(ctx, layer, M, L, q_dev, o_dev);
+  if (rc) return rc;
+  return sync_state(ctx);
+}
+
+int fdllm_profile_enable(fdllm_ctx* ctx, int enable) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  prof_harvest(ctx);
+  ctx->prof = enable != 0;
+  if (ctx->prof) ctx->prof_stats.clear();
+  return FDLLM_OK;
+}
+
+int fdllm_profile_read(fdllm_ctx* ctx, fdllm_kernel_stat* out, int max_stats, int* n_stats) {
+  if (!ctx || !n_stats || (max_stats > 0 && !out)) return FDLLM_ERR_ARG;
+  if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  prof_harvest(ctx);
+  *n_stats = (int)ctx->prof_stats.size();
+  for (int i = 0; i < max_stats && i < *n_stats; ++i) out[i] = ctx->prof_stats[i];
+  return FDLLM_OK;
+}
+
+const char* fdllm_last_error(const fdllm_ctx* ctx) {
+  return ctx ? ctx->err.c_str() : g_create_error.c_str();
+}
+
+int64_t fdllm_launch_count(fdllm_ctx* ctx, int reset) {
+  if (!ctx) return 0;
+  const int64_t n = ctx->launches;
+  if (reset) ctx->launches = 0;
+  return n;
+}
+
+int fdllm_destroy(fdllm_ctx* ctx) {
+  if (!ctx) return FDLLM_OK;
+  cudaSetDevice(ctx->device);
+  if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  prof_harvest(ctx);
+  for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
+  dfree_all(ctx);
+  if (ctx->state_host) cudaFreeHost(ctx->state_host);
+  if (ctx->err_host) cudaFreeHost(ctx->err_host);
+  if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
+  delete ctx;
+  return FDLLM_OK;
+}
+
+}  // extern "C"

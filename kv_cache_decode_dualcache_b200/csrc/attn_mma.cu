@@ -1,0 +1,301 @@
+// Bidirectional attention of the bfloat16 model on tensor cores (mma.sync).
+//
+// o = softmax(q K^T / sqrt(hd)) V over keys [0, L), no mask: block queries
+// (DualCache step), rows [s, L) (prefix-cache step) or every position (full
+// forward) all attend to the whole sequence, whose K/V come from the paged
+// cache (the step's own rows were written there by the QKV epilogue just
+// before).
+//
+// CTA = (row tile of 64 query rows, KV head, key split).  A query row is a
+// (position, head-in-group) pair, so the query heads that share a KV head in
+// GQA share the K/V tiles.  Four warps, 16 rows each.  K/V tiles of 64 keys
+// (one cache page) are double-buffered in shared memory with cp.async, in a
+// 16-byte-chunk XOR swizzle so ldmatrix is conflict-free.
+//
+// Every operand is two-term (hi + lo): q and K as bf16 pairs, V as fp16
+// pairs, and the softmax weights P are split the same way into fp16 pairs.
+// Each product takes the three significant cross terms:
+//   S  = q_hi K_hi + q_hi K_lo + q_lo K_hi        (bf16 MMAs, f32 accumulate)
+//   PV = P_hi V_hi + P_hi V_lo + P_lo V_hi        (fp16 MMAs, f32 accumulate)
+// so the attention output carries ~16 significant bits like every other
+// stored activation of the bf16 model (see split_bf16).  Online softmax in
+// f32, exp2 domain.  With n_split > 1 each split writes unnormalised partial
+// outputs and its (max, sum) per row; attn_combine merges them.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fd {
+
+namespace {
+
+FD_DEV void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+FD_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+FD_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+FD_DEV void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+FD_DEV void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+FD_DEV void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+FD_DEV void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `ch` of row `r` in a [64][HD] 2-byte tile.
+template <int HD>
+FD_DEV uint32_t swz(int r, int ch) {
+  return (uint32_t)(r * HD * 2 + ((ch ^ (r & 7)) << 4));
+}
+
+template <int HD>
+__global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
+  constexpr int TILE = 64 * HD * 2;  // bytes of one [64][HD] 2-byte tile
+  constexpr int CH = HD / 8;         // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t sm[];
+  // layout: Q hi, Q lo, then per buffer b: K hi, K lo, V hi, V lo
+  const uint32_t q_s = smem_u32(sm);
+  auto kv_s = [&](int buf, int plane) { return q_s + (2 + buf * 4 + plane) * TILE; };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.n_heads, Hkv = p.n_kv_heads, rep = H / Hkv;
+  const int g = blockIdx.y;
+  const int rows_total = p.M * rep;
+  const int row0 = blockIdx.x * 64;
+  const int key_lo = blockIdx.z * p.keys_per_split;
+  const int key_hi = min(p.L, key_lo + p.keys_per_split);
+  const int n_kt = (key_hi - key_lo + 63) / 64;
+
+  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q);
+  const uint16_t* pool = reinterpret_cast<const uint16_t*>(p.kv_pool);
+
+  // ---- Q tiles (hi and lo planes)
+  for (int idx = tid; idx < 64 * CH; idx += 128) {
+    const int i = idx / CH, ch = idx % CH;
+    const int r = row0 + i;
+    const bool ok = r < rows_total;
+    const int m = ok ? r / rep : 0, jj = ok ? r % rep : 0;
+    const __nv_bfloat16* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
+    cp_async16(q_s + swz<HD>(i, ch), src, ok ? 16 : 0);
+    cp_async16(q_s + TILE + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
+  }
+  auto load_kv = [&](int kt, int buf) {
+    const int k0 = key_lo + kt * 64;
+    const int page = p.page_table[k0 / KV_PAGE];
+    const size_t plane = (size_t)Hkv * KV_PAGE * HD;
+    const size_t base = ((size_t)p.layer * p.n_pages + page) * 4 * plane + (size_t)g * KV_PAGE * HD;
+    for (int idx = tid; idx < 64 * CH; idx += 128) {
+      const int i = idx / CH, ch = idx % CH;
+      const bool ok = (k0 + i) < key_hi;
+      const size_t e = base + (size_t)(ok ? i : 0) * HD + ch * 8;
+#pragma unroll
+      for (int pl = 0; pl < 4; ++pl)
+        cp_async16(kv_s(buf, pl) + swz<HD>(i, ch), pool + e + pl * plane, ok ? 16 : 0);
+    }
+  };
+  load_kv(0, 0);
+  cp_async_commit();
+
+  const bool warp_active = row0 + warp * 16 < rows_total;
+  const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // 1/sqrt(hd) * log2(e)
+  float oacc[HD / 8][4];
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.0f;
+  float mrow[2] = {-INFINITY, -INFINITY};
+  float lrow[2] = {0.0f, 0.0f};
+
+  for (int kt = 0; kt < n_kt; ++kt) {
+    if (kt + 1 < n_kt) load_kv(kt + 1, (kt + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const int buf = kt & 1;
+    if (warp_active) {
+      // ---- S = Q K^T for 64 keys (8 n-tiles of 8)
+      float s[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        uint32_t qh[4], ql[4];
+        const uint32_t qa = swz<HD>(warp * 16 + (lane & 15), 2 * kk + (lane >> 4));
+        ldsm_x4(q_s + qa, qh);
+        ldsm_x4(q_s + TILE + qa, ql);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t kh[4], kl[4];
+          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const uint32_t ka = swz<HD>(key, 2 * kk + ((lane >> 3) & 1));
+          ldsm_x4(kv_s(buf, 0) + ka, kh);
+          ldsm_x4(kv_s(buf, 1) + ka, kl);
+          mma_bf16(s[2 * np], qh, kh[0], kh[1]);
+          mma_bf16(s[2 * np + 1], qh, kh[2], kh[3]);
+          mma_bf16(s[2 * np], qh, kl[0], kl[1]);
+          mma_bf16(s[2 * np + 1], qh, kl[2], kl[3]);
+          mma_bf16(s[2 * np], ql, kh[0], kh[1]);
+          mma_bf16(s[2 * np + 1], ql, kh[2], kh[3]);
+        }
+      }
+      // ---- online softmax (rows lane/4 and lane/4 + 8)
+      const int kbase = key_lo + kt * 64 + 2 * (lane & 3);
+      float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool ok = kbase + nt * 8 + (c & 1) < key_hi;
+          s[nt][c] = ok ? s[nt][c] * sl2 : -INFINITY;
+          tmax[c >> 1] = fmaxf(tmax[c >> 1], s[nt][c]);
+        }
+      }
+      float alpha[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+        tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+        const float mnew = fmaxf(mrow[r], tmax[r]);
+        alpha[r] = (mrow[r] == -INFINITY) ? 0.0f : exp2f(mrow[r] - mnew);
+        mrow[r] = mnew;
+        lrow[r] *= alpha[r];
+      }
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        oacc[j][0] *= alpha[0];
+        oacc[j][1] *= alpha[0];
+        oacc[j][2] *= alpha[1];
+        oacc[j][3] *= alpha[1];
+      }
+      uint32_t ph[8][2], pl[8][2];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float p0 = exp2f(s[nt][2 * r] - mrow[r]);
+          const float p1 = exp2f(s[nt][2 * r + 1] - mrow[r]);
+          const __half2 hi = __floats2half2_rn(p0, p1);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
+          ph[nt][r] = *reinterpret_cast<const uint32_t*>(&hi);
+          pl[nt][r] = *reinterpret_cast<const uint32_t*>(&lo);
+          lrow[r] += p0 + p1;
+        }
+      }
+      // ---- O += P V
+#pragma unroll
+      for (int kk2 = 0; kk2 < 4; ++kk2) {
+        const uint32_t ah[4] = {ph[2 * kk2][0], ph[2 * kk2][1], ph[2 * kk2 + 1][0],
+                                ph[2 * kk2 + 1][1]};
+        const uint32_t al[4] = {pl[2 * kk2][0], pl[2 * kk2][1], pl[2 * kk2 + 1][0],
+                                pl[2 * kk2 + 1][1]};
+#pragma unroll
+        for (int j = 0; j < HD / 8; j += 2) {
+          uint32_t vh[4], vl[4];
+          const int key = kk2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+          const uint32_t va = swz<HD>(key, j + (lane >> 4));
+          ldsm_x4_t(kv_s(buf, 2) + va, vh);
+          ldsm_x4_t(kv_s(buf, 3) + va, vl);
+          mma_f16(oacc[j], ah, vh[0], vh[1]);
+          mma_f16(oacc[j + 1], ah, vh[2], vh[3]);
+          mma_f16(oacc[j], ah, vl[0], vl[1]);
+          mma_f16(oacc[j + 1], ah, vl[2], vl[3]);
+          mma_f16(oacc[j], al, vh[0], vh[1]);
+          mma_f16(oacc[j + 1], al, vh[2], vh[3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  if (!warp_active) return;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
+    lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
+  }
+  const int rows_all = p.M * H;
+  const int hq = H * HD;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int rr = row0 + warp * 16 + (lane >> 2) + 8 * r;
+    if (rr >= rows_total) continue;
+    const int m = rr / rep, head = g * rep + rr % rep;
+    const size_t orow = (size_t)m * H + head;
+    if (p.n_split == 1) {
+      const float inv = 1.0f / lrow[r];
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
+      const size_t hi_off = (size_t)pair_row(m) * hq + (size_t)head * HD;
+      const size_t lo_off = hi_off + (size_t)PAIR_LO * hq;
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        const int d = j * 8 + 2 * (lane & 3);
+        __nv_bfloat16 h0, l0, h1, l1;
+        split_bf16(oacc[j][2 * r] * inv, h0, l0);
+        split_bf16(oacc[j][2 * r + 1] * inv, h1, l1);
+        *reinterpret_cast<__nv_bfloat162*>(o + hi_off + d) = __halves2bfloat162(h0, h1);
+        *reinterpret_cast<__nv_bfloat162*>(o + lo_off + d) = __halves2bfloat162(l0, l1);
+      }
+    } else {
+      float* po = p.part_o + ((size_t)blockIdx.z * rows_all + orow) * HD;
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        const int d = j * 8 + 2 * (lane & 3);
+        *reinterpret_cast<float2*>(po + d) = make_float2(oacc[j][2 * r], oacc[j][2 * r + 1]);
+      }
+      if ((lane & 3) == 0) {
+        float* ml = p.part_ml + ((size_t)blockIdx.z * rows_all + orow) * 2;
+        ml[0] = mrow[r];
+        ml[1] = lrow[r];
+      }
+    }
+  }
+}
+
+template <int HD>
+cudaError_t launch_hd(const AttnParams& p, cudaStream_t st) {
+  constexpr int smem = 10 * 64 * HD * 2;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<HD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int rows = p.M * (p.n_heads / p.n_kv_heads);
+  dim3 grid((rows + 63) / 64, p.n_kv_heads, p.n_split);
+  attn_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st) {
+  if (p.kv_planes != 4) return cudaErrorInvalidValue;
+  switch (p.head_dim) {
+    case 64: return launch_hd<64>(p, st);
+    case 128: return launch_hd<128>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fd

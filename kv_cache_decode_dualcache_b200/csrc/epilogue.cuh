@@ -1,0 +1,187 @@
+// GEMM epilogues shared by the tcgen05 GEMM (bf16 model) and the CUDA-core
+// GEMM (fp32 model).
+//
+// Both GEMMs hand the epilogue output tiles of 128 features x 32 tokens,
+// staged in shared memory as float tile[t * 128 + e] (t = token row in the
+// chunk, e = feature within the 128-feature tile).  The 128 epilogue threads
+// call epi_chunk with e = their feature index.  Control flow is uniform
+// within each warp (the LM-head reduction uses warp shuffles).
+//
+// Stores of the bf16 model are two-term (hi + lo, see split_bf16): the q
+// planes, the K/V cache planes and the SwiGLU output in pair rows.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fd {
+
+constexpr int EPI_THREADS = 128;
+constexpr int CHUNK_T = 32;
+
+FD_DEV size_t kv_offset(const EpiParams& ep, int pos, int plane, int head, int dim) {
+  const int page = ep.page_table[pos / KV_PAGE];
+  const int slot = pos % KV_PAGE;
+  return ((((size_t)ep.layer * ep.n_pages + page) * ep.kv_planes + plane) * ep.n_kv_heads +
+          head) * (size_t)(KV_PAGE * ep.head_dim) +
+         (size_t)slot * ep.head_dim + dim;
+}
+
+// One 32-token chunk of a 128-feature output tile.
+//   tile: [32][128] float in shared memory, fully written before the call.
+//   n0:   first feature of the tile; t0: token row of tile row 0.
+//   lm:   per-token softmax states of this CTA (EPI_LMHEAD only).
+template <bool F32>
+FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, int e,
+                      SoftmaxState* lm) {
+  const int n = n0 + e;
+  switch (ep.kind) {
+    case EPI_STORE: {
+      if (n < ep.N)
+        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t)
+        {
+          const size_t i = (size_t)(t0 + t) * ep.ld_out + n;
+          if (FD_CHECK(i < ep.cap_out, ep.check, 1, i, ep.cap_out)) ep.out[i] = tile[t * 128 + e];
+        }
+      break;
+    }
+    case EPI_RESID: {
+      if (n < ep.N)
+        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t)
+        {
+          const size_t i = (size_t)(t0 + t) * ep.N + n;
+          if (FD_CHECK(i < ep.cap_h, ep.check, 2, i, ep.cap_h)) ep.h[i] += tile[t * 128 + e];
+        }
+      break;
+    }
+    case EPI_SWIGLU: {
+      // Rows [128j, 128j+64) of the fused weight are gate rows [64j, 64j+64),
+      // rows [128j+64, 128j+128) the matching up rows.
+      const int F = ep.N / 2;
+      const int j = (n0 / 128) * 64 + e;
+      if (e < 64 && j < F)
+        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
+          const float g = tile[t * 128 + e];
+          const float u = tile[t * 128 + e + 64];
+          const float y = silu_f(g) * u;
+          const int tok = t0 + t;
+          if (F32) {
+            const size_t i = (size_t)tok * F + j;
+            if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f))
+              reinterpret_cast<float*>(ep.f_out)[i] = y;
+          } else {
+            __nv_bfloat16 hi, lo;
+            split_bf16(y, hi, lo);
+            __nv_bfloat16* f = reinterpret_cast<__nv_bfloat16*>(ep.f_out);
+            const size_t r = (size_t)pair_row(tok);
+            const size_t i = (r + PAIR_LO) * F + j;
+            if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f)) {
+              f[r * F + j] = hi;
+              f[i] = lo;
+            }
+          }
+        }
+      break;
+    }
+    case EPI_QKV: {
+      if (n >= ep.N) break;
+      const int hd = ep.head_dim, half = hd / 2;
+      const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
+      const int dh = n % hd;
+      const bool is_q = n < hq, is_v = n >= hq + hk;
+      for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
+        const int tok = t0 + t;
+        const int pos = ep.pos0 + tok;
+        float y = tile[t * 128 + e];
+        if (!is_v) {
+          const float2 cs = ep.rope[(size_t)pos * half + (dh % half)];
+          if (dh < half) {
+            const float x2 = tile[t * 128 + e + half];
+            y = y * cs.x - x2 * cs.y;
+          } else {
+            const float x1 = tile[t * 128 + e - half];
+            y = y * cs.x + x1 * cs.y;
+          }
+        }
+        if (F32) {
+          float* kv = reinterpret_cast<float*>(ep.kv_pool);
+          if (is_q) {
+            const size_t i = (size_t)tok * hq + n;
+            if (FD_CHECK(i < ep.cap_q, ep.check, 4, i, ep.cap_q))
+              reinterpret_cast<float*>(ep.q_out)[i] = y;
+          } else {
+            const size_t i = is_v ? kv_offset(ep, pos, 1, (n - hq - hk) / hd, dh)
+                                  : kv_offset(ep, pos, 0, (n - hq) / hd, dh);
+            if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
+          }
+        } else if (is_q) {
+          __nv_bfloat16 hi, lo;
+          split_bf16(y, hi, lo);
+          __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(ep.q_out);
+          const size_t i = (size_t)tok * hq + n;
+          if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
+            q[i] = hi;
+            q[ep.q_plane + i] = lo;
+          }
+        } else if (!is_v) {
+          __nv_bfloat16 hi, lo;
+          split_bf16(y, hi, lo);
+          __nv_bfloat16* k = reinterpret_cast<__nv_bfloat16*>(ep.kv_pool);
+          const int head = (n - hq) / hd;
+          const size_t i0 = kv_offset(ep, pos, 0, head, dh), i1 = kv_offset(ep, pos, 1, head, dh);
+          if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
+            k[i0] = hi;
+            k[i1] = lo;
+          }
+        } else {
+          __half hi, lo;
+          split_f16(y, hi, lo);
+          __half* v = reinterpret_cast<__half*>(ep.kv_pool);
+          const int head = (n - hq - hk) / hd;
+          const size_t i0 = kv_offset(ep, pos, 2, head, dh), i1 = kv_offset(ep, pos, 3, head, dh);
+          if (FD_CHECK(i1 < ep.cap_kv, ep.check, 6, i1, ep.cap_kv)) {
+            v[i0] = hi;
+            v[i1] = lo;
+          }
+        }
+      }
+      break;
+    }
+    case EPI_LMHEAD: {
+      const int warp = e >> 5, lane = e & 31;
+      for (int t = warp; t < CHUNK_T; t += EPI_THREADS / 32) {
+        const int tok = t0 + t;
+        if (tok >= ep.M) break;  // uniform across the warp
+        float z[4];
+        float mx = -INFINITY;
+        int arg = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = lane + 32 * j;
+          const int nn = n0 + r;
+          z[j] = ep.logit_scale * tile[t * 128 + r];
+          if (ep.dbg_logits && nn < ep.N) {
+            const size_t i = (size_t)tok * ep.N + nn;
+            if (FD_CHECK(i < ep.cap_dbg, ep.check, 7, i, ep.cap_dbg)) ep.dbg_logits[i] = z[j];
+          }
+          const bool ok = nn < ep.N && nn != ep.mask_id;
+          if (!ok) z[j] = -INFINITY;
+          if (z[j] > mx) { mx = z[j]; arg = nn; }  // j ascending: lowest id kept on ties
+        }
+        warp_argmax(mx, arg);
+        float s = 0.0f;
+        if (mx != -INFINITY) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) s += (z[j] == -INFINITY) ? 0.0f : expf(z[j] - mx);
+        }
+        s = warp_sum(s);
+        if (lane == 0) lm[tok] = sm_merge(lm[tok], SoftmaxState{mx, s, arg});
+      }
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+}  // namespace fd

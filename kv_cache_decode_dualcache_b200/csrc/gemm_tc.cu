@@ -1,0 +1,315 @@
+// Persistent tcgen05 GEMM for the bfloat16 model: Y[t, n] = sum_k X[t, k] W[n, k].
+//
+// The weight matrix is the 128-row A operand (the "swap-AB" arrangement: the
+// model's output features fill the MMA's M = 128; the few block tokens are
+// the MMA's N), so a block step with 32 tokens still issues full 128-row
+// MMAs while it streams the weights once from HBM.  The activations are
+// two-term (hi + lo bf16) in pair rows: every 64 rows hold the hi and the lo
+// term of 32 tokens, so a token tile of NT rows covers NT/2 tokens and the
+// lo term costs tensor work only (the weights are read once).  Both operands
+// are K-major, staged by TMA with the 128-byte swizzle into a STAGES-deep
+// ring of shared-memory buffers; one thread issues tcgen05.mma into a
+// double-buffered TMEM accumulator (128 lanes x NT columns each), and four
+// epilogue warps drain the accumulator with tcgen05.ld, 64 columns (hi and
+// lo of 32 tokens, summed) at a time, through the shared epilogue (RoPE +
+// KV-cache write, residual add, SwiGLU, or the fused LM-head
+// max/argmax/sum-exp).
+//
+// Work units are (feature tile, token tile, K split).  CTAs loop over units
+// with a stride of gridDim.x.  With more than one split, each split writes
+// its float partial tile to a workspace and the last split to arrive (an
+// atomic counter per tile, reset by that CTA) sums the partials in split
+// order, so results do not depend on arrival order.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
+// MMA issuer, warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
+#include <type_traits>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace fd {
+
+namespace {
+
+constexpr int BK = 64;                    // K elements per stage (128 bytes of bf16)
+constexpr int A_STAGE_BYTES = 128 * BK * 2;
+constexpr int LM_MAX_ROWS = 256;          // largest M for the LM-head epilogue
+
+template <int NT> struct TcCfg;
+template <> struct TcCfg<64> { static constexpr int STAGES = 8; };
+template <> struct TcCfg<128> { static constexpr int STAGES = 6; };
+template <> struct TcCfg<256> { static constexpr int STAGES = 4; };
+
+template <int NT>
+struct TcLayout {
+  static constexpr int STAGES = TcCfg<NT>::STAGES;
+  static constexpr int B_STAGE_BYTES = NT * BK * 2;
+  static constexpr int A_OFF = 0;
+  static constexpr int B_OFF = A_OFF + STAGES * A_STAGE_BYTES;
+  static constexpr int TILE_OFF = B_OFF + STAGES * B_STAGE_BYTES;
+  static constexpr int BAR_OFF = TILE_OFF + CHUNK_T * 128 * 4;
+  static constexpr int N_BARS = 2 * STAGES + 4;
+  static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
+  static constexpr int LM_OFF = MISC_OFF + 16;
+  static constexpr int END = LM_OFF + LM_MAX_ROWS * (int)sizeof(SoftmaxState);
+  static constexpr int SMEM = END + 1024;  // slack for 1024-byte alignment
+  static_assert(B_STAGE_BYTES % 1024 == 0, "B stages must stay 1024-byte aligned");
+  static_assert(SMEM <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
+};
+
+struct UnitCoord {
+  int tile, tt, split, kb_lo, kb_hi;
+};
+
+FD_DEV UnitCoord decode_unit(const GemmShape& gs, int u) {
+  UnitCoord c;
+  c.split = u % gs.splits;
+  const int rest = u / gs.splits;
+  c.tt = rest % gs.n_tt;
+  c.tile = rest / gs.n_tt;
+  c.kb_lo = (int)((long long)c.split * gs.kb_total / gs.splits);
+  c.kb_hi = (int)((long long)(c.split + 1) * gs.kb_total / gs.splits);
+  return c;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap,
+                   const __grid_constant__ CUtensorMap amap, GemmShape gs, EpiParams ep,
+                   GemmScratch sc) {
+  constexpr int TOK = NT / 2;  // tokens per token tile
+  using Lay = TcLayout<NT>;
+  constexpr int STAGES = Lay::STAGES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(NT);
+  constexpr uint32_t TMEM_COLS = 2 * NT;
+  constexpr uint32_t STAGE_TX = A_STAGE_BYTES + Lay::B_STAGE_BYTES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* a_st = smem + Lay::A_OFF;
+  uint8_t* b_st = smem + Lay::B_OFF;
+  float* tile = reinterpret_cast<float*>(smem + Lay::TILE_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 2);
+  SoftmaxState* lm = reinterpret_cast<SoftmaxState*>(smem + Lay::LM_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool lmhead = ep.kind == EPI_LMHEAD;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], EPI_THREADS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&wmap);
+    tma_prefetch_desc(&amap);
+  }
+  if (warp == 1) tmem_alloc(misc, TMEM_COLS);
+  if (lmhead && warp >= 2) {
+    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_THREADS)
+      lm[t] = sm_empty();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x) {
+        const UnitCoord c = decode_unit(gs, u);
+        for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, sc.err, abort_flag)) { ok = false; break; }
+          FD_CHECK(kb >= 0 && kb < gs.kb_total && c.tile < gs.n_tiles && c.tt < gs.n_tt, ep.check,
+                   20, kb, c.tile * 65536 + c.tt);
+          mbar_arrive_expect_tx(&full[s], STAGE_TX);
+          tma_load_2d(a_st + s * A_STAGE_BYTES, &wmap, &full[s], kb * BK, c.tile * 128);
+          tma_load_2d(b_st + s * Lay::B_STAGE_BYTES, &amap, &full[s], kb * BK, c.tt * NT);
+        }
+      }
+      if (!ok || *abort_flag) {
+        // Let every copy already issued land before the CTA can exit.
+        const uint32_t n = it < (uint32_t)STAGES ? it : (uint32_t)STAGES;
+        for (uint32_t j = 0; j < n; ++j) {
+          const uint32_t i2 = it - 1 - j;
+          mbar_wait(&full[i2 % STAGES], (i2 / STAGES) & 1u, sc.err, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x, ++local) {
+        const UnitCoord c = decode_unit(gs, u);
+        const uint32_t buf = local & 1u;
+        if (!mbar_wait(&acc_empty[buf], ((local >> 1) & 1u) ^ 1u, sc.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * NT;
+        for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1u, sc.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(a_st + s * A_STAGE_BYTES);
+          const uint32_t b0 = smem_u32(b_st + s * Lay::B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_bf16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), IDESC,
+                        (kb > c.kb_lo || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int e = quad * 32 + lane;  // feature row = TMEM lane
+    uint32_t local = 0;
+    for (int u = blockIdx.x; u < gs.units; u += gridDim.x, ++local) {
+      const UnitCoord c = decode_unit(gs, u);
+      const uint32_t buf = local & 1u;
+      const bool got = mbar_wait(&acc_full[buf], (local >> 1) & 1u, sc.err, abort_flag);
+      tc_fence_after();
+      const int n0 = c.tile * 128;
+      const int tile_id = c.tile * gs.n_tt + c.tt;
+      float* ws_unit = sc.ws + ((size_t)tile_id * gs.splits + c.split) * (TOK * 128);
+      for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
+        // columns [64ch, 64ch+32) hold the hi term, [64ch+32, 64ch+64) the lo term
+        float v[32], vl[32];
+        FD_CHECK(buf * NT + ch * 64 + 64 <= TMEM_COLS, ep.check, 21, buf * NT + ch * 64, TMEM_COLS);
+        const uint32_t col = tmem + ((uint32_t)(quad * 32) << 16) + buf * NT + ch * 64;
+        tmem_ld32(col, v);
+        tmem_ld32(col + 32, vl);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] += vl[t];
+        if (gs.splits == 1) {
+          named_bar(1, EPI_THREADS);  // previous chunk's epilogue is done with `tile`
+#pragma unroll
+          for (int t = 0; t < 32; ++t) tile[t * 128 + e] = v[t];
+          named_bar(1, EPI_THREADS);
+          if (got) epi_chunk<false>(ep, tile, n0, c.tt * TOK + ch * CHUNK_T, e, lm);
+        } else {
+          const size_t wi = (size_t)(ws_unit - sc.ws) + (ch * CHUNK_T + 31) * 128 + e;
+          if (FD_CHECK(wi < sc.ws_elems, ep.check, 22, wi, sc.ws_elems)) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ws_unit[(ch * CHUNK_T + t) * 128 + e] = v[t];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      if (gs.splits > 1) {
+        __threadfence();
+        named_bar(1, EPI_THREADS);
+        if (e == 0) {
+          int prev = -1;
+          if (FD_CHECK(tile_id < sc.n_counters, ep.check, 23, tile_id, sc.n_counters))
+            prev = atomicAdd(&sc.counters[tile_id], 1);
+          *last_flag = (prev == gs.splits - 1);
+        }
+        named_bar(1, EPI_THREADS);
+        if (*last_flag) {
+          __threadfence();
+          const float* ws_tile = sc.ws + (size_t)tile_id * gs.splits * (TOK * 128);
+          for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
+            float acc[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) acc[t] = 0.0f;
+            for (int sp = 0; sp < gs.splits; ++sp) {
+              const float* p = ws_tile + (size_t)sp * (TOK * 128) + ch * CHUNK_T * 128 + e;
+              const size_t wi = (size_t)(p - sc.ws) + 31 * 128;
+              if (!FD_CHECK(wi < sc.ws_elems, ep.check, 24, wi, sc.ws_elems)) continue;
+#pragma unroll
+              for (int t = 0; t < 32; ++t) acc[t] += __ldcg(p + t * 128);
+            }
+            named_bar(1, EPI_THREADS);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) tile[t * 128 + e] = acc[t];
+            named_bar(1, EPI_THREADS);
+            if (got) epi_chunk<false>(ep, tile, n0, c.tt * TOK + ch * CHUNK_T, e, lm);
+          }
+          if (e == 0) sc.counters[tile_id] = 0;
+        }
+        named_bar(1, EPI_THREADS);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (lmhead && warp >= 2) {
+    SoftmaxState* out = reinterpret_cast<SoftmaxState*>(ep.lm_part) + (size_t)blockIdx.x * gs.M;
+    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_THREADS) {
+      const size_t i = (size_t)blockIdx.x * gs.M + t;
+      if (FD_CHECK(i < ep.cap_lm, ep.check, 25, i, ep.cap_lm)) out[t] = lm[t];
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int NT>
+cudaError_t launch_nt(const CUtensorMap* w_map, const CUtensorMap* act_map, const GemmShape& gs,
+                      const EpiParams& ep, const GemmScratch& sc, cudaStream_t st) {
+  static bool attr_set = false;
+  const int smem = TcLayout<NT>::SMEM;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  gemm_tc_kernel<NT><<<gs.grid, 192, smem, st>>>(*w_map, *act_map, gs, ep, sc);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_tc_smem_bytes(int nt) {
+  switch (nt) {
+    case 64: return TcLayout<64>::SMEM;
+    case 128: return TcLayout<128>::SMEM;
+    case 256: return TcLayout<256>::SMEM;
+    default: return -1;
+  }
+}
+
+cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
+                           const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
+                           cudaStream_t st) {
+  if (ep.kind == EPI_LMHEAD && gs.M > LM_MAX_ROWS) return cudaErrorInvalidValue;
+  switch (gs.nt) {
+    case 64: return launch_nt<64>(w_map, act_map, gs, ep, sc, st);
+    case 128: return launch_nt<128>(w_map, act_map, gs, ep, sc, st);
+    case 256: return launch_nt<256>(w_map, act_map, gs, ep, sc, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fd

@@ -1,0 +1,133 @@
+// Internal interface between the host orchestration (api.cu) and the kernel
+// translation units.  Not part of the public C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fd {
+
+enum EpiKind : int {
+  EPI_STORE = 0,   // out[t, n] = y (float)
+  EPI_QKV = 1,     // RoPE on q and k; q -> q buffer, k and v -> KV cache pages
+  EPI_RESID = 2,   // h[t, n] += y  (float residual stream)
+  EPI_SWIGLU = 3,  // 64-row gate/up groups: f[t, j] = silu(gate) * up
+  EPI_LMHEAD = 4,  // online max / argmax / sum-exp over vocab tiles
+};
+
+// Everything a GEMM epilogue needs.  Token index t is the row within the
+// GEMM's activation operand (0..M-1); feature index n is the output column.
+struct EpiParams {
+  int kind;
+  int N;             // output features (rows of the weight matrix)
+  int M;             // valid token rows
+  int act_f32;       // 1: activations / outputs are float (fp32 model); 0: bf16
+  // EPI_STORE
+  float* out;
+  int ld_out;
+  // EPI_QKV
+  void* q_out;       // fp32: [M, H*hd]; bf16: hi plane then lo plane, each [rows, H*hd]
+  size_t q_plane;    // elements per q plane (bf16)
+  void* kv_pool;     // [layers][pages][planes][Hkv][KV_PAGE][hd]; planes: fp32 K,V;
+                     // bf16 K hi, K lo (bf16), V hi, V lo (fp16)
+  int kv_planes;
+  const int* page_table;
+  int n_pages;
+  int layer;
+  int pos0;          // absolute position of token row 0
+  const float2* rope;  // [max_seq][hd/2] (cos, sin)
+  int n_heads, n_kv_heads, head_dim;
+  // EPI_RESID
+  float* h;          // [M, N]
+  // EPI_SWIGLU
+  void* f_out;       // [M, N/2] (fp32) or two-term pair rows (bf16)
+  // EPI_LMHEAD
+  float logit_scale;
+  int mask_id;
+  float* lm_part;    // [n_part][M] of (m, s, arg) triples
+  float* dbg_logits; // optional [M, N] float logits (mask id included)
+  // Capacities (elements) of the output buffers, used only by builds with
+  // FDLLM_CHECKS, where every store is bounds-checked and a violation is
+  // recorded in check[0..3] (count, code, index, aux) instead of performed.
+  size_t cap_out, cap_h, cap_q, cap_kv, cap_f, cap_dbg, cap_lm;
+  int* check;
+};
+
+// Bookkeeping shared by both GEMM implementations.
+struct GemmShape {
+  int N, M, K;
+  int nt;            // token tile width
+  int splits;        // K splits (deterministic reduction when > 1)
+  int n_tiles;       // ceil(N / 128)
+  int n_tt;          // ceil(M / nt)
+  int kb_total;      // ceil(K / 64)
+  int units;         // n_tiles * n_tt * splits
+  int grid;          // CTAs launched
+};
+
+struct GemmScratch {
+  float* ws;         // split-K partial tiles
+  int* counters;     // per tile arrival counters (self-resetting)
+  int* err;          // device error word
+  size_t ws_elems;   // capacities (checked in FDLLM_CHECKS builds)
+  int n_counters;
+};
+
+// Launchers (return cudaError_t of the launch).
+// bf16 model: activations in two-term pair rows, token tiles of nt/2 tokens.
+cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
+                           const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
+                           cudaStream_t st);
+// fp32 model: plain [M, K] activations starting at row act_row0.
+cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int K,
+                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st);
+int gemm_tc_smem_bytes(int nt);
+
+struct AttnParams {
+  const void* q;       // [M, H, hd] (fp32) or hi/lo planes of [M, H, hd] (bf16)
+  size_t q_plane;      // elements per q plane (bf16)
+  void* o;             // [M, H*hd] (fp32) or two-term pair rows (bf16)
+  const void* kv_pool;
+  int kv_planes;
+  const int* page_table;
+  int n_pages, layer;
+  int M;               // query positions
+  int L;               // keys [0, L)
+  int n_heads, n_kv_heads, head_dim;
+  int n_split;         // key splits (1 = write o directly)
+  int keys_per_split;  // multiple of 64
+  float* part_o;       // [n_split][M*H][hd]
+  float* part_ml;      // [n_split][M*H][2]
+};
+
+cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st);
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st);
+cudaError_t launch_attn_combine(const AttnParams& p, int f32, cudaStream_t st);
+
+// h[i] = embed[x[r0+i]]; a[i] = RMSNorm(h[i]) * g, i in [0, M).
+cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
+                                 int vocab, const float* g, float eps, float* h, void* a,
+                                 int f32, int* err, cudaStream_t st);
+// a[i] = RMSNorm(h[h_row0 + i]) * g, i in [0, M).  bf16: two-term pair rows.
+cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
+                           void* a, int f32, cudaStream_t st);
+
+struct DecodeState {
+  int remaining;     // masked positions left in the block after the step
+  int unmasked;      // positions unmasked by the step
+  int steps;         // steps taken so far (incremented by every select)
+  int pad;
+};
+
+// Merge LM-head partials into conf/tok for n rows and, when select != 0,
+// apply the threshold-or-fallback unmask rule to x[s .. s+n).
+cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,
+                                int mask_id, float tau, int select, float* conf, int* tok,
+                                uint8_t* unmask, DecodeState* state, cudaStream_t st);
+
+cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st);
+cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
+                                cudaStream_t st);
+
+}  // namespace fd

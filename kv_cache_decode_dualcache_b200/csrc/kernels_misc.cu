@@ -1,0 +1,358 @@
+// CUDA-core kernels: embedding + RMSNorm, RMSNorm, the LM-head partial
+// merge fused with the threshold/unmask/scatter step, the float32 GEMM and
+// attention of the fp32 model, and the split-KV attention combine.
+#include <type_traits>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace fd {
+
+namespace {
+
+// Deterministic block sum (fixed tree) for blockDim.x a multiple of 32.
+FD_DEV float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.0f;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+FD_DEV float block_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = -INFINITY;
+  for (int i = 0; i < nw; ++i) t = fmaxf(t, red[i]);
+  return t;
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// a[row] = h[h_row0 + row] / sqrt(mean(h^2) + eps) * g; one CTA per row.  With
+// `x` given, h[row] is first gathered from the embedding table at token
+// x[r0 + row].  fp32 model: a is [M, d] float; bf16 model: a is two-term in
+// pair rows.
+template <typename T>
+__global__ void rmsnorm_kernel(const int* x, int r0, const T* embed, int vocab, float* h,
+                               int h_row0, int d, const float* g, float eps, T* a, int* err) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  float* hr = h + (size_t)(h_row0 + row) * d;
+  if (x) {
+    int tok = x[r0 + row];
+    if (tok < 0 || tok >= vocab) {
+      if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
+      tok = 0;
+    }
+    const T* er = embed + (size_t)tok * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) hr[j] = to_f(er[j]);
+  }
+  float ss = 0.0f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const float v = hr[j];
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  if (std::is_same<T, float>::value) {
+    for (int j = threadIdx.x; j < d; j += blockDim.x)
+      a[(size_t)row * d + j] = from_f<T>(hr[j] * inv * g[j]);
+  } else {
+    __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(a);
+    const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      __nv_bfloat16 hi, lo;
+      split_bf16(hr[j] * inv * g[j], hi, lo);
+      ab[r_hi + j] = hi;
+      ab[r_lo + j] = lo;
+    }
+  }
+}
+
+// ------------------------------------------------------- merge + select
+__global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
+                                    int mask_id, float tau, int select, float* conf, int* tok,
+                                    uint8_t* unmask, DecodeState* state) {
+  __shared__ float s_conf[256];
+  __shared__ int s_tok[256];
+  __shared__ int s_best;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = warp; t < n; t += blockDim.x >> 5) {
+    SoftmaxState st = sm_empty();
+    for (int q = lane; q < n_part; q += 32) st = sm_merge(st, part[(size_t)q * n + t]);
+    st = warp_sm_merge(st);
+    if (lane == 0) {
+      // conf = exp(z_max - logsumexp) = 1 / sum exp(z - z_max)
+      const float c = (st.s > 0.0f) ? 1.0f / st.s : 0.0f;
+      s_conf[t] = c;
+      s_tok[t] = st.arg;
+      conf[t] = c;
+      tok[t] = st.arg;
+    }
+  }
+  __syncthreads();
+  if (!select) return;
+  const int i = threadIdx.x;
+  const bool valid = i < n;
+  const bool masked = valid && x[s + i] == mask_id;
+  const float ci = valid ? s_conf[i] : 0.0f;
+  const bool pass = masked && (ci >= tau);
+  const int n_pass = __syncthreads_count(pass);
+  if (threadIdx.x == 0) {
+    int best = -1;
+    float bc = -INFINITY;
+    if (n_pass == 0) {
+      for (int j = 0; j < n; ++j) {
+        if (x[s + j] != mask_id) continue;
+        const float cj = (s_conf[j] == s_conf[j]) ? s_conf[j] : -1.0f;  // NaN last
+        if (best < 0 || cj > bc) { best = j; bc = cj; }
+      }
+    }
+    s_best = best;
+  }
+  __syncthreads();
+  const bool u = pass || (n_pass == 0 && i == s_best);
+  if (valid) unmask[i] = u ? 1 : 0;
+  const int n_left = __syncthreads_count(masked && !u);
+  const int n_un = __syncthreads_count(u);
+  if (u) x[s + i] = s_tok[i];
+  if (threadIdx.x == 0) {
+    state->remaining = n_left;
+    state->unmasked = n_un;
+    state->steps += 1;
+  }
+}
+
+__global__ void fill_kernel(int* x, int from, int to, int v) {
+  const int i = from + blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < to) x[i] = v;
+}
+
+__global__ void check_prompt_kernel(const int* x, int n, int vocab, int mask_id, int* err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const int t = x[i];
+    if (t < 0 || t >= vocab || t == mask_id) atomicOr(err, DEV_ERR_TOKEN);
+  }
+}
+
+// ------------------------------------------------------- CUDA-core GEMM
+// One CTA computes one 128-feature x 32-token chunk; 128 threads, thread e
+// owns feature n0 + e.  Used by the float32 model (float32 FMAs; tensor-core
+// tf32 would round the inputs to 10 significant bits).
+__global__ void __launch_bounds__(128)
+    gemm_simt_kernel(const float* w, const float* act, int act_row0, int K, GemmShape gs,
+                     EpiParams ep) {
+  __shared__ float ws_[32][129];
+  __shared__ float as_[32][33];
+  __shared__ float tile[32 * 128];
+  __shared__ SoftmaxState lm[32];
+  const int e = threadIdx.x;
+  const int tile_idx = blockIdx.x % gs.n_tiles;
+  const int tt = blockIdx.x / gs.n_tiles;
+  const int n0 = tile_idx * 128, t0 = tt * 32;
+  float acc[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.0f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int idx = e; idx < 128 * 32; idx += 128) {
+      const int r = idx / 32, kk = idx % 32;
+      const int n = n0 + r, k = k0 + kk;
+      ws_[kk][r] = (n < gs.N && k < K) ? w[(size_t)n * K + k] : 0.0f;
+    }
+    for (int idx = e; idx < 32 * 32; idx += 128) {
+      const int t = idx / 32, kk = idx % 32;
+      const int k = k0 + kk;
+      as_[t][kk] = (t0 + t < gs.M && k < K) ? act[(size_t)(act_row0 + t0 + t) * K + k] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 32; ++kk) {
+      const float wv = ws_[kk][e];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) acc[t] = fmaf(wv, as_[t][kk], acc[t]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int t = 0; t < 32; ++t) tile[t * 128 + e] = acc[t];
+  SoftmaxState* lmp = lm - t0;  // index by absolute token row
+  if (ep.kind == EPI_LMHEAD && e < 32) lm[e] = sm_empty();
+  __syncthreads();
+  epi_chunk<true>(ep, tile, n0, t0, e, lmp);
+  __syncthreads();
+  if (ep.kind == EPI_LMHEAD) {
+    SoftmaxState* out = reinterpret_cast<SoftmaxState*>(ep.lm_part) + (size_t)blockIdx.x * gs.M;
+    for (int t = e; t < gs.M; t += 128) out[t] = (t >= t0 && t < t0 + 32) ? lm[t - t0] : sm_empty();
+  }
+}
+
+// ------------------------------------------------------- CUDA-core attention
+// One CTA per (query row, head): softmax(q K^T / sqrt(hd)) V over keys [0, L),
+// float32 model (K and V planes of float).
+__global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
+  using T = float;
+  using VT = float;
+  extern __shared__ float sh[];
+  __shared__ float red[32];
+  float* qs = sh;               // [hd]
+  float* sc = sh + p.head_dim;  // [L]
+  const int m = blockIdx.x, head = blockIdx.y;
+  const int hd = p.head_dim, H = p.n_heads, Hkv = p.n_kv_heads;
+  const int g = head / (H / Hkv);
+  const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)m * H + head) * hd;
+  for (int d = threadIdx.x; d < hd; d += blockDim.x) qs[d] = to_f(q[d]);
+  __syncthreads();
+  const float scale = 1.0f / sqrtf((float)hd);
+  const T* kp = reinterpret_cast<const T*>(p.kv_pool);
+  const VT* vp = reinterpret_cast<const VT*>(p.kv_pool);
+  auto off = [&](int pos, int kv) {
+    const int page = p.page_table[pos / KV_PAGE];
+    return ((((size_t)p.layer * p.n_pages + page) * p.kv_planes + kv) * Hkv + g) *
+               (size_t)(KV_PAGE * hd) +
+           (size_t)(pos % KV_PAGE) * hd;
+  };
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j < p.L; j += blockDim.x) {
+    const T* kr = kp + off(j, 0);
+    float dot = 0.0f;
+    for (int d = 0; d < hd; ++d) dot = fmaf(qs[d], to_f(kr[d]), dot);
+    sc[j] = dot * scale;
+    mx = fmaxf(mx, sc[j]);
+  }
+  mx = block_max(mx, red);
+  float sum = 0.0f;
+  for (int j = threadIdx.x; j < p.L; j += blockDim.x) {
+    const float e = expf(sc[j] - mx);
+    sc[j] = e;
+    sum += e;
+  }
+  sum = block_sum(sum, red);
+  __syncthreads();
+  T* o = reinterpret_cast<T*>(p.o) + ((size_t)m * H + head) * hd;
+  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
+    float acc = 0.0f;
+    for (int j = 0; j < p.L; ++j) acc = fmaf(sc[j], to_f(vp[off(j, 1) + d]), acc);
+    o[d] = from_f<T>(acc / sum);
+  }
+}
+
+// Combine split-KV partial attention outputs (log2-domain maxima).
+template <typename T>
+__global__ void attn_combine_kernel(AttnParams p) {
+  const int row = blockIdx.x;  // m * H + head
+  const int rows = p.M * p.n_heads;
+  const int hd = p.head_dim;
+  float mstar = -INFINITY;
+  for (int c = 0; c < p.n_split; ++c) mstar = fmaxf(mstar, p.part_ml[((size_t)c * rows + row) * 2]);
+  float den = 0.0f;
+  for (int c = 0; c < p.n_split; ++c) {
+    const float m = p.part_ml[((size_t)c * rows + row) * 2];
+    if (m != -INFINITY) den += exp2f(m - mstar) * p.part_ml[((size_t)c * rows + row) * 2 + 1];
+  }
+  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
+    float num = 0.0f;
+    for (int c = 0; c < p.n_split; ++c) {
+      const float m = p.part_ml[((size_t)c * rows + row) * 2];
+      if (m != -INFINITY) num += exp2f(m - mstar) * p.part_o[((size_t)c * rows + row) * hd + d];
+    }
+    const float y = num / den;
+    if (std::is_same<T, float>::value) {
+      reinterpret_cast<float*>(p.o)[(size_t)row * hd + d] = y;
+    } else {
+      // two-term pair rows of [M, H*hd]
+      const int m = row / p.n_heads, head = row % p.n_heads;
+      const size_t hq = (size_t)p.n_heads * hd;
+      const size_t off = (size_t)pair_row(m) * hq + (size_t)head * hd + d;
+      __nv_bfloat16 hi, lo;
+      split_bf16(y, hi, lo);
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
+      o[off] = hi;
+      o[off + (size_t)PAIR_LO * hq] = lo;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
+                                 int vocab, const float* g, float eps, float* h, void* a,
+                                 int f32, int* err, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  if (f32)
+    rmsnorm_kernel<float><<<M, 256, 0, st>>>(x, r0, (const float*)embed, vocab, h, 0, d, g, eps,
+                                             (float*)a, err);
+  else
+    rmsnorm_kernel<__nv_bfloat16><<<M, 256, 0, st>>>(x, r0, (const __nv_bfloat16*)embed, vocab,
+                                                     h, 0, d, g, eps, (__nv_bfloat16*)a, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
+                           void* a, int f32, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  if (f32)
+    rmsnorm_kernel<float><<<M, 256, 0, st>>>(nullptr, 0, nullptr, 0, const_cast<float*>(h),
+                                             h_row0, d, g, eps, (float*)a, nullptr);
+  else
+    rmsnorm_kernel<__nv_bfloat16><<<M, 256, 0, st>>>(nullptr, 0, nullptr, 0,
+                                                     const_cast<float*>(h), h_row0, d, g, eps,
+                                                     (__nv_bfloat16*)a, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,
+                                int mask_id, float tau, int select, float* conf, int* tok,
+                                uint8_t* unmask, DecodeState* state, cudaStream_t st) {
+  if (n <= 0 || n > 256) return cudaErrorInvalidValue;
+  merge_select_kernel<<<1, 256, 0, st>>>(reinterpret_cast<const SoftmaxState*>(lm_part), n_part,
+                                         n, x, s, mask_id, tau, select, conf, tok, unmask, state);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st) {
+  if (to <= from) return cudaSuccess;
+  fill_kernel<<<(to - from + 255) / 256, 256, 0, st>>>(x, from, to, mask_id);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
+                                cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  check_prompt_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, n, vocab, mask_id, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int K,
+                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st) {
+  const int grid = gs.n_tiles * ((gs.M + 31) / 32);
+  gemm_simt_kernel<<<grid, 128, 0, st>>>(w, act, act_row0, K, gs, ep);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st) {
+  if (p.kv_planes != 2) return cudaErrorInvalidValue;
+  dim3 grid(p.M, p.n_heads);
+  const size_t smem = (size_t)(p.head_dim + p.L) * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  attn_simt_kernel<<<grid, 128, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const AttnParams& p, int f32, cudaStream_t st) {
+  const int rows = p.M * p.n_heads;
+  if (f32)
+    attn_combine_kernel<float><<<rows, 128, 0, st>>>(p);
+  else
+    attn_combine_kernel<__nv_bfloat16><<<rows, 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace fd

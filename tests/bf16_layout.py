@@ -1,0 +1,27 @@
+"""Builders for the two-term (hi + lo) bf16 layouts the bf16 decoder uses,
+written with plain torch ops for the GPU kernel tests."""
+import torch
+
+
+def split(x: torch.Tensor):
+    hi = x.to(torch.bfloat16)
+    lo = (x - hi.float()).to(torch.bfloat16)
+    return hi, lo
+
+
+def pair_rows(x: torch.Tensor) -> torch.Tensor:
+    """[M, K] float -> [2*ceil(M/32)*32, K] bf16: per group of 32 tokens the
+    32 hi rows, then the 32 lo rows."""
+    M, K = x.shape
+    G = (M + 31) // 32
+    pad = torch.zeros(G * 32, K, device=x.device, dtype=x.dtype)
+    pad[:M] = x
+    hi, lo = split(pad)
+    return torch.stack([hi.view(G, 32, K), lo.view(G, 32, K)], dim=1).reshape(G * 64, K)
+
+
+def from_pair_rows(y: torch.Tensor, M: int) -> torch.Tensor:
+    """Inverse of pair_rows: hi + lo as float [M, K]."""
+    G = y.shape[0] // 64
+    v = y.float().view(G, 2, 32, -1)
+    return (v[:, 0] + v[:, 1]).reshape(G * 32, -1)[:M]

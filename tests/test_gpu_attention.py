@@ -1,0 +1,48 @@
+"""The decoder's attention kernel in isolation: random queries against the
+K/V the GPU cached for a sequence, checked against the oracle's attention
+(float64) on exactly those K/V.  Covers the no-split path (many rows) and
+the split-KV path (block-sized M), MHA and GQA, ragged key counts."""
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_decode_dualcache_b200 import fdllm, synth
+from oracle.model import attention
+from tests.bf16_layout import from_pair_rows, split
+from tests.gpu_util import make_decoder, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", params=["small-bf16", "small-gqa-bf16"])
+def setup(request):
+    require_gpu()
+    shape = synth.SHAPES[request.param]
+    dec = make_decoder(shape, synth.make_weights(shape, device="cpu"), 256)
+    prompt = synth.make_prompt(shape, 150).numpy()
+    x = np.concatenate([prompt, np.full(50, shape.mask_id)])
+    dec.step_debug(x, x, 150, 32, 0.9, "dual", logits=False)   # fills the cache for 200 positions
+    return shape, dec
+
+
+@pytest.mark.parametrize("M,L", [(32, 200), (200, 200), (7, 65), (64, 128), (100, 37)])
+@pytest.mark.parametrize("qscale", [1.0, 4.0, 16.0])
+def test_attention_matches_oracle(setup, M, L, qscale):
+    shape, dec = setup
+    H, hd = shape.n_heads, shape.head_dim
+    g = torch.Generator(device="cuda").manual_seed(M * 1000 + L)
+    q = torch.randn(M, H, hd, generator=g, device="cuda") * qscale
+    qh, ql = split(q)
+    qd = torch.stack([qh, ql]).contiguous()
+    rows = 2 * ((M + 31) // 32) * 32
+    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.bfloat16)
+    fdllm.fdllm_attention(dec.ctx, qd, o, 0, L)
+    torch.cuda.synchronize()
+    k, v = dec.read_kv(0, 0, L)
+    qx = (qh.double() + ql.double()).cpu().numpy()
+    ref = attention(qx, k.astype(np.float64), v.astype(np.float64)).reshape(M, H * hd)
+    got = from_pair_rows(o, M).double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    tol = 1e-4 * max(1.0, np.abs(ref).max())
+    assert err <= tol, (err, tol)
