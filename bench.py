@@ -1,0 +1,386 @@
+"""Benchmark of the Fast-dLLM DualCache decoder on the LLaDA-8B shape.
+
+One "step" = one full block-wise generation (every block-start refresh and
+every DualCache block step: the whole hot path) of gen_len tokens after a
+prompt, with random N(0, 0.02) bf16 weights of the LLaDA-8B shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fdllm|reference]
+
+Prints one JSON line.  value = generated tokens/s of the whole job (all
+ranks), timed with CUDA events on the decoder's stream around K generations
+with the prompt already in HBM (max over ranks).  e2e = the same metric
+through the host-buffer C call (prompt copied in, tokens copied out every
+step).  roofline = the dominant kernel class of a separate profiled
+generation (per-launch CUDA events), against MEASURED_PEAKS.json.
+cpu_baseline = the float64 oracle on the host cores on a bounded sample.
+Multi-GPU runs are independent replicas (one sequence per rank).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gen tokens/s (LLaDA-8B shape, DualCache, tau=0.9)"
+WORKLOAD = "llada8b-p256-g256"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _config(wl, n):
+    return {"workload": wl.name, "model_shape": wl.shape.name, "prompt_len": wl.prompt_len,
+            "gen_len": wl.gen_len, "block_size": wl.block_size, "tau": wl.tau,
+            "cache_mode": wl.cache_mode, "batch_per_gpu": 1, "global_batch": n,
+            "weights": "random N(0,0.02) bf16, seed 1",
+            "l2": "no flush needed: each step streams ~16 GB of weights (> 126 MB L2)",
+            "parallelism": "replicas" if n > 1 else "single"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = sorted(v for v in (num(r[1]) for r in rows) if v is not None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "samples": len(rows), "reasons": reasons}
+
+
+def roofline_from_profile(stats, hbm, tf_sustained, peak_kind, traffic):
+    """Dominant kernel class: block-step GEMMs (HBM-bound, M <= 64 tokens) or
+    full-forward GEMMs (tensor-bound).  achieved = algorithmic bytes (flops)
+    of its launches / their summed event time."""
+    groups = {"step": [s for s in stats if s["name"].startswith("gemm.") and s["name"].endswith(".step")],
+              "full": [s for s in stats if s["name"].startswith("gemm.") and s["name"].endswith(".full")]}
+    tot = {k: sum(s["total_ms"] for s in v) for k, v in groups.items()}
+    total_all = sum(s["total_ms"] for s in stats) or 1.0
+    key = max(tot, key=tot.get)
+    g = groups[key]
+    ms = tot[key]
+    launches = sum(s["launches"] for s in g)
+    if key == "step":
+        achieved = sum(s["bytes"] for s in g) / (ms * 1e-3) / 1e9
+        out = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s"}
+        per_launch_bytes = sum(s["bytes"] for s in g) / max(1, launches)
+    else:
+        achieved = sum(s["flops"] for s in g) / (ms * 1e-3) / 1e12
+        out = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tf_sustained,
+               "unit": "TFLOP/s"}
+        per_launch_bytes = sum(s["bytes"] for s in g) / max(1, launches)
+    out["frac"] = round(out["achieved"] / out["peak"], 4)
+    out["traffic"] = traffic
+    out["kernel"] = "gemm_tc_kernel (%s-forward launches)" % ("DualCache block-step" if key == "step"
+                                                           else "full")
+    out["share_of_kernel_time"] = round(ms / total_all, 3)
+    out["launches"] = launches
+    out["algorithmic_bytes_per_launch"] = round(per_launch_bytes)
+    out["peak_source"] = peak_kind
+    out["classes"] = {s["name"]: {"launches": s["launches"], "ms": round(s["total_ms"], 3),
+                                  "GBps": round(s["bytes"] / (s["total_ms"] * 1e-3) / 1e9, 1)
+                                  if s["total_ms"] else None,
+                                  "TFps": round(s["flops"] / (s["total_ms"] * 1e-3) / 1e12, 1)
+                                  if s["total_ms"] else None} for s in stats}
+    return out
+
+
+def _traffic_record():
+    """ncu DRAM bytes per launch recorded for the current GEMM source, if any."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
+    try:
+        rec = json.load(open(path))
+        src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", "gemm_tc.cu"),
+                    "rb").read()
+        if rec.get("gemm_tc_sha256") == hashlib.sha256(src).hexdigest():
+            return rec.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, weights_host, step_counts, sample_layers=4):
+    """The float64 oracle, as it stands, on a bounded sample: one block-start
+    full forward and one DualCache block step of a model with the first
+    `sample_layers` layers, each scaled to the full depth.  Returns the
+    oracle's generated tokens/s estimated with the GPU run's step counts."""
+    import numpy as np
+    import torch
+    from kv_cache_decode_dualcache_b200 import synth
+    from oracle.model import Model
+
+    shape = synth.with_layers(wl.shape, sample_layers)
+    w = {k: v for k, v in weights_host.items()
+         if not k.startswith("layers.") or int(k.split(".")[1]) < sample_layers}
+    model = Model(shape.as_dict(), w)
+    P, G, B = wl.prompt_len, wl.gen_len, wl.block_size
+    L = P + G
+    prompt = synth.make_prompt(wl.shape, P).numpy()
+    x = np.concatenate([prompt, np.full(G, wl.shape.mask_id)])
+    t0 = time.perf_counter()
+    _, kv = model.forward(x, range(L), return_kv=True, head_rows=range(P, P + B))  # refresh
+    t_refresh = time.perf_counter() - t0
+    cur = x.copy()
+    cur[P:P + B // 2] = prompt[:B // 2]
+    t0 = time.perf_counter()
+    model.forward(cur, range(P, P + B), cache=kv)                                  # DualCache step
+    t_step = time.perf_counter() - t0
+    scale = wl.shape.n_layers / sample_layers
+    n_ref, n_cached = step_counts
+    total = scale * (n_ref * t_refresh + n_cached * t_step)
+    return {"tok_s": G / total, "t_refresh_s": t_refresh * scale, "t_step_s": t_step * scale,
+            "sample_s": t_refresh + t_step, "threads": torch.get_num_threads()}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from kv_cache_decode_dualcache_b200 import synth
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    sample_layers = 4
+    w = synth.make_weights(wl.shape, device=dev)
+    w = {k: v.cpu() for k, v in w.items()
+         if not k.startswith("layers.") or int(k.split(".")[1]) < sample_layers}
+    # step counts of this workload's decode (8 blocks; the GPU run measured
+    # 3.25 steps per block on average); the oracle runs the same schedule
+    n_blocks = wl.gen_len // wl.block_size
+    counts = (n_blocks, args.ref_cached_steps)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(wl, w, counts, sample_layers)
+        if i >= args.warmup:
+            vals.append(r)
+    v = sum(r["tok_s"] for r in vals) / len(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * wl.gen_len / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(wl, 1),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["threads"],
+                             "kind": "oracle",
+                             "sample": f"per step: one block-start full forward and one DualCache "
+                                       f"block step of the first {sample_layers} of "
+                                       f"{wl.shape.n_layers} layers, scaled x"
+                                       f"{wl.shape.n_layers // sample_layers}; "
+                                       f"{counts[0]} refresh + {counts[1]} cached steps"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_fdllm(args, wl):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from kv_cache_decode_dualcache_b200 import build, fdllm, synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    shape = wl.shape
+    P, G, B, tau = wl.prompt_len, wl.gen_len, wl.block_size, wl.tau
+    stream = torch.cuda.Stream()
+    dec = fdllm.Decoder(shape, P + G, device=local, stream=stream.cuda_stream)
+    w = synth.make_weights(shape, device="cuda")
+    dec.load_weights(w)
+    want_cpu = (not args.no_cpu_baseline) and world == 1 and rank == 0
+    w_host = None
+    if want_cpu:
+        w_host = {k: v.cpu() for k, v in w.items()
+                  if not k.startswith("layers.") or int(k.split(".")[1]) < 4}
+    del w
+    torch.cuda.empty_cache()
+    prompt = synth.make_prompt(shape, P, salt=rank).numpy()
+    prompt_host = torch.from_numpy(prompt).pin_memory()
+    prompt_dev = prompt_host.to(f"cuda:{local}")
+    out_dev = torch.empty(G, dtype=torch.int32, device=f"cuda:{local}")
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        dec.generate_device(prompt_dev, G, B, tau, out_dev, wl.cache_mode)
+    torch.cuda.synchronize()
+
+    # ---- timed region: device-resident prompt
+    sampler = ClockSampler(local) if rank == 0 else None
+    dec.launch_count(reset=True)
+    steps_total = 0
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        steps_total += dec.generate_device(prompt_dev, G, B, tau, out_dev, wl.cache_mode)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    launches = dec.launch_count(reset=True)
+    clocks = sampler.stop() if sampler else None
+    t = torch.tensor([ms], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = world * args.steps * G / (ms_max * 1e-3)
+    tokens = out_dev.cpu().numpy()
+
+    # ---- end to end: host buffers through the C call
+    out_host = torch.empty(G, dtype=torch.int32).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    e2e_steps = 0
+    stats = None
+    for _ in range(args.steps):
+        res, nsteps, stats = dec.generate(prompt_host.numpy(), G, B, tau, wl.cache_mode)
+        out_host.numpy()[:] = res
+        e2e_steps += nsteps
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t2 = torch.tensor([e2.elapsed_time(e3)], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_value = world * args.steps * G / (float(t2.item()) * 1e-3)
+    steps_per_gen = e2e_steps / args.steps
+    h2d = P * 4
+    d2h = G * 4 + int(round(steps_per_gen)) * 20   # tokens + per-step state / error words
+
+    # ---- roofline: one profiled generation (per-launch events)
+    fdllm.fdllm_profile_enable(dec.ctx, True)
+    dec.generate_device(prompt_dev, G, B, tau, out_dev, wl.cache_mode)
+    prof = fdllm.fdllm_profile_read(dec.ctx)
+    fdllm.fdllm_profile_enable(dec.ctx, False)
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, _traffic_record())
+    timing = dec.generate(prompt, G, B, tau, wl.cache_mode, timing=True)[2]
+
+    cpu = None
+    if want_cpu:
+        cores = len(os.sched_getaffinity(0))
+        torch.set_num_threads(cores)
+        r = oracle_sample(wl, w_host, (timing.refresh_steps, timing.cached_steps))
+        cpu = {"value": r["tok_s"], "unit": "tokens/s", "cores": r["threads"], "kind": "oracle",
+               "sample": "one block-start full forward and one DualCache block step of the "
+                         "first 4 of 32 layers (float64 oracle), scaled x8 and weighted by "
+                         f"this run's {timing.refresh_steps} refresh + {timing.cached_steps} "
+                         f"cached steps ({r['sample_s']:.1f} s of CPU work)",
+               "t_refresh_s": round(r["t_refresh_s"], 3), "t_step_s": round(r["t_step_s"], 3)}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": _config(wl, world),
+                "decode": {"denoising_steps_per_generation": steps_total / args.steps,
+                           "steps_per_block": timing.steps_per_block,
+                           "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
+                           "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3),
+                           "tokens_checksum": int(np.asarray(tokens, dtype=np.int64).sum())},
+                "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches,
+                "roofline": roof,
+                "clocks": clocks,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fdllm", choices=["fdllm", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-cached-steps", type=int, default=18,
+                    help="cached steps per generation assumed by the reference arm")
+    args = ap.parse_args()
+    from kv_cache_decode_dualcache_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_fdllm(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

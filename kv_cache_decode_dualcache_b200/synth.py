@@ -94,6 +94,14 @@ WORKLOADS = {
     "llada8b-p1024-g1024": Workload("llada8b-p1024-g1024", LLADA_8B, 1024, 1024, 32, 0.9, "dual"),
     "dream7b-p512-g512": Workload("dream7b-p512-g512", DREAM_7B, 512, 512, 32, 0.9, "dual"),
     "llada8b-batch16": Workload("llada8b-batch16", LLADA_8B, 0, 256, 32, 0.9, "dual", batch=16),
+    # Two layers of the LLaDA-8B shape (~3 GB of weights): the same GEMM,
+    # attention and LM-head shapes per launch, small enough for a full ncu
+    # capture of single launches.
+    "llada8b-2layer-p256-g32": Workload("llada8b-2layer-p256-g32",
+                                        ModelShape("llada-8b-shape-2layer", 2, 4096, 32, 32, 128,
+                                                   12288, 126464, 126463, 1e4, 1e-5, 30.0, "bf16",
+                                                   1),
+                                        256, 32, 32, 0.9, "dual"),
 }
 
 
