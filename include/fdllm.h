@@ -221,6 +221,33 @@ FDLLM_API int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, f
 FDLLM_API int fdllm_attention(fdllm_ctx* ctx, const void* q_dev, void* o_dev, int layer, int M,
                               int L);
 
+/* The same GEMM as fdllm_gemm on the bf16 model (tcgen05, two-term x in
+ * the 32-token pair-row layout described there, float y), for callers that
+ * cannot allocate device memory: code that runs inside a host framework
+ * which has reserved the device memory up front (a cudaMalloc here would
+ * fail or break its accounting), or that must not take the implicit
+ * synchronisation an allocation can cause.  It needs no ctx and allocates
+ * nothing: the split-K scratch (8 MiB of partial tiles, 4096 tile counters,
+ * an error word) is a fixed device array inside the library, present on
+ * every GPU that loads the library until the process exits.  The Fast-dLLM
+ * pages have no counterpart of this call; it is an interface convenience.
+ *   - Runs on the current CUDA device, on stream cuda_stream (NULL = the
+ *     legacy default stream), and returns when the result is in y_dev.
+ *   - The first call on each device looks the scratch array's address up
+ *     and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the same scratch array: calls whose GPU
+ *     work overlaps (two host threads, or two streams) race and give wrong
+ *     results.  The tile counters and the error word are cleared on the
+ *     stream at the start of every call.
+ *   - Maximum size: the planned (or forced) K splits must fit their partial
+ *     tiles in 8 MiB (units x tokens-per-tile x 128 floats) and the output
+ *     must have at most 4096 tiles of 128 features x one token tile; larger
+ *     requests return FDLLM_ERR_ARG (message via fdllm_last_error(NULL)).
+ * Errors: ARG (NULL pointers, sizes <= 0, K % 64 != 0, misaligned operands,
+ * too many splits, beyond the maximum, not an sm_100 GPU), CUDA, TIMEOUT. */
+FDLLM_API int fdllm_gemm_noalloc(const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
+                                 int K, int splits, void* cuda_stream);
+
 /* Per-kernel-class timing.  While enabled, every launch the ctx makes is
  * bracketed by CUDA events on the ctx's stream and accumulated per class
  * (e.g. "gemm.ffn_up.step", "attn.full"), together with the launch's

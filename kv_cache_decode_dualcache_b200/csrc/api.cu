@@ -275,50 +275,18 @@ int check_config(const fdllm_config* c, std::string* why) {
 // balance the per-CTA K blocks over the persistent grid (deterministic
 // reduction of the splits).  Plans are memoised per shape.
 GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split) {
+  if (ctx->tc) return plan_gemm_tc(ctx->num_sms, N, M, K, allow_split, kWorkspaceBytes);
   GemmShape g{};
   g.N = N;
   g.M = M;
   g.K = K;
   g.n_tiles = (N + 127) / 128;
   g.kb_total = (K + 63) / 64;
-  if (!ctx->tc) {
-    g.nt = 32;
-    g.splits = 1;
-    g.n_tt = (M + 31) / 32;
-    g.units = g.n_tiles * g.n_tt;
-    g.grid = g.units;
-    return g;
-  }
-  int nt = 64;
-  while (nt / 2 < M && nt < 256) nt *= 2;
-  g.nt = nt;
-  g.n_tt = (M + nt / 2 - 1) / (nt / 2);
-  const int base_units = g.n_tiles * g.n_tt;
-  const int max_split = allow_split ? std::min(16, std::max(1, g.kb_total / 4)) : 1;
-  double best = 1e300;
-  int best_s = 1;
-  for (int s = 1; s <= max_split; ++s) {
-    const long long units = (long long)base_units * s;
-    if (s > 1 && (size_t)units * (nt / 2) * 128 * sizeof(float) > kWorkspaceBytes) break;
-    const int grid = (int)std::min<long long>(units, ctx->num_sms);
-    // per-CTA cost in K blocks of its units, +2 per unit (pipeline fill and
-    // epilogue), +1 per unit when split (partial tile write and reduction)
-    std::vector<double> load(grid, 0.0);
-    for (long long u = 0; u < units; ++u) {
-      const int sp = (int)(u % s);
-      const int kb = (int)((long long)(sp + 1) * g.kb_total / s - (long long)sp * g.kb_total / s);
-      load[u % grid] += kb + 2.0 + (s > 1 ? 1.0 : 0.0);
-    }
-    double mx = 0.0;
-    for (double v : load) mx = std::max(mx, v);
-    if (mx < best * 0.995) {
-      best = mx;
-      best_s = s;
-    }
-  }
-  g.splits = best_s;
-  g.units = base_units * best_s;
-  g.grid = std::min(g.units, ctx->num_sms);
+  g.nt = 32;
+  g.splits = 1;
+  g.n_tt = (M + 31) / 32;
+  g.units = g.n_tiles * g.n_tt;
+  g.grid = g.units;
   return g;
 }
 
@@ -640,6 +608,53 @@ int generate_impl(fdllm_ctx* ctx, const int32_t* prompt, bool prompt_dev, int P,
 }
 
 }  // namespace
+
+namespace fd {
+
+// Error message for calls without a ctx (fdllm_last_error(NULL)).
+void set_thread_error(const std::string& msg) { g_create_error = msg; }
+
+GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes) {
+  GemmShape g{};
+  g.N = N;
+  g.M = M;
+  g.K = K;
+  g.n_tiles = (N + 127) / 128;
+  g.kb_total = (K + 63) / 64;
+  int nt = 64;
+  while (nt / 2 < M && nt < 256) nt *= 2;
+  g.nt = nt;
+  g.n_tt = (M + nt / 2 - 1) / (nt / 2);
+  const int base_units = g.n_tiles * g.n_tt;
+  const int max_split = allow_split ? std::min(16, std::max(1, g.kb_total / 4)) : 1;
+  double best = 1e300;
+  int best_s = 1;
+  for (int s = 1; s <= max_split; ++s) {
+    const long long units = (long long)base_units * s;
+    if (s > 1 && (size_t)units * (nt / 2) * 128 * sizeof(float) > ws_bytes) break;
+    const int grid = (int)std::min<long long>(units, num_sms);
+    // per-CTA cost in K blocks of its units, +2 per unit (pipeline fill and
+    // epilogue), +1 per unit when split (partial tile write and reduction)
+    std::vector<double> load(grid, 0.0);
+    for (long long u = 0; u < units; ++u) {
+      const int sp = (int)(u % s);
+      const int kb = (int)((long long)(sp + 1) * g.kb_total / s - (long long)sp * g.kb_total / s);
+      load[u % grid] += kb + 2.0 + (s > 1 ? 1.0 : 0.0);
+    }
+    double mx = 0.0;
+    for (double v : load) mx = std::max(mx, v);
+    if (mx < best * 0.995) {
+      best = mx;
+      best_s = s;
+    }
+  }
+  g.splits = best_s;
+  g.units = base_units * best_s;
+  g.grid = std::min(g.units, num_sms);
+  return g;
+}
+
+}  // namespace fd
 
 // =============================================================== C ABI
 extern "C" {

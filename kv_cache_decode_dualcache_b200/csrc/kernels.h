@@ -74,6 +74,12 @@ struct GemmScratch {
   int n_counters;
 };
 
+// Tile / split plan of the tcgen05 GEMM for N output features, M tokens and
+// reduction length K on a GPU with num_sms SMs: token tile of nt rows (nt/2
+// tokens of two-term activations), K split chosen to balance the per-CTA K
+// blocks over the persistent grid, within ws_bytes of split-K workspace.
+GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes);
+
 // Launchers (return cudaError_t of the launch).
 // bf16 model: activations in two-term pair rows, token tiles of nt/2 tokens.
 cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,

@@ -29,8 +29,8 @@ DTYPES = {"fp32": 0, "bf16": 1}
 
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
             "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention",
-            "fdllm_profile_enable", "fdllm_profile_read", "fdllm_last_error",
-            "fdllm_launch_count", "fdllm_destroy")
+            "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
+            "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
 
 
 class FdllmConfig(ctypes.Structure):
@@ -103,6 +103,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_read_kv.argtypes = [vp, i32, i32, i32, P(ctypes.c_float), P(ctypes.c_float)]
     lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32]
     lib.fdllm_attention.argtypes = [vp, vp, vp, i32, i32, i32]
+    lib.fdllm_gemm_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
     lib.fdllm_profile_enable.argtypes = [vp, i32]
     lib.fdllm_profile_read.argtypes = [vp, P(FdllmKernelStat), i32, P(i32)]
     lib.fdllm_last_error.argtypes = [vp]
@@ -111,8 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_launch_count.restype = ctypes.c_int64
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
-                 "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_profile_enable",
-                 "fdllm_profile_read", "fdllm_destroy"):
+                 "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -265,6 +266,23 @@ def fdllm_gemm(ctx, w_dev, x_dev, y_dev, splits: int = 0) -> None:
         raise ValueError(f"x_dev must be a contiguous [{need}, {K}] tensor")
     _check(load_library().fdllm_gemm(ctx, w_dev.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(), N,
                                      M, K, splits), ctx)
+
+
+def fdllm_gemm_noalloc(w_dev, x_dev, y_dev, splits: int = 0, stream=None) -> None:
+    """Allocation-free variant of fdllm_gemm (bf16 model only; no ctx): same
+    operands and layouts, scratch from the library's fixed device array.
+    Runs on the current device and the given stream handle (None = legacy
+    default stream)."""
+    N, K = w_dev.shape
+    M = int(y_dev.shape[0])
+    if tuple(y_dev.shape) != (M, N) or not y_dev.is_contiguous():
+        raise ValueError("y_dev must be a contiguous [M, N] tensor")
+    need = _pair_rows(M)
+    if x_dev.shape[0] < need or x_dev.shape[1] != K or not x_dev.is_contiguous():
+        raise ValueError(f"x_dev must be a contiguous [{need}, {K}] tensor")
+    _check(load_library().fdllm_gemm_noalloc(w_dev.data_ptr(), x_dev.data_ptr(),
+                                             y_dev.data_ptr(), N, M, K, splits,
+                                             ctypes.c_void_p(stream) if stream else None), None)
 
 
 def fdllm_attention(ctx, q_dev, o_dev, layer: int, L: int) -> None:
