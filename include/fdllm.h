@@ -203,12 +203,13 @@ FDLLM_API int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k
  * hi = bf16(x), lo = bf16(x - hi)) grouped by 32 tokens: group j occupies
  * rows [64j, 64j+32) with the hi terms of tokens 32j.. and rows
  * [64j+32, 64j+64) with their lo terms (2 * ceil(M/32) * 32 rows in all).
- * y_dev is a device [M, N] float buffer.  splits = 0 lets the planner pick
- * the K split; splits > 0 forces it (bf16 only).  Needs K % 64 == 0 and
- * 16-byte aligned w_dev / x_dev on the bf16 model.  Errors: ARG, CUDA,
- * TIMEOUT. */
+ * y_dev is a device [M, N] float buffer: y = x W^T, or y += x W^T when
+ * accumulate != 0 (the residual-add epilogue of the decoder's O and down
+ * projections).  splits = 0 lets the planner pick the K split; splits > 0
+ * forces it (bf16 only).  Needs K % 64 == 0 and 16-byte aligned w_dev /
+ * x_dev on the bf16 model.  Errors: ARG, CUDA, TIMEOUT. */
 FDLLM_API int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev,
-                         int N, int M, int K, int splits);
+                         int N, int M, int K, int splits, int accumulate);
 
 /* Kernel-level check of the decoder's attention over the ctx's KV cache:
  * o = softmax(q K^T / sqrt(head_dim)) V with keys [0, L) of layer `layer`

@@ -36,6 +36,7 @@ constexpr size_t kWorkspaceBytes = 64ull << 20;
 constexpr int kMaxLmRows = 256;
 constexpr int kMaxAttnSplit = 16;
 constexpr int kAttnSplitMaxM = 64;
+constexpr int kSpRing = 8;
 
 thread_local std::string g_create_error = "no error";
 
@@ -100,6 +101,7 @@ struct fdllm_ctx {
   int n_counters = 0;
   float* attn_po = nullptr;
   float* attn_ml = nullptr;
+  int* attn_cnt = nullptr;      // split-merge counters of the attention kernel
   float* lm_part = nullptr;
   size_t lm_part_cap = 0;   // SoftmaxState entries
   float* conf = nullptr;
@@ -116,6 +118,17 @@ struct fdllm_ctx {
   CUtensorMap m_a[3], m_o[3], m_f[3];
   std::map<std::tuple<int, int, int, int>, GemmShape> plans;
   int64_t launches = 0;
+  bool pdl = true;              // programmatic dependent launch between kernels
+  bool graphs = true;           // replay each step kind from a captured CUDA graph
+  StepParams* sp = nullptr;     // device step scalars (read by the kernels)
+  StepParams* sp_host = nullptr;  // pinned ring of kSpRing slots: a pending async copy
+  int sp_slot = 0;                // never reads a slot overwritten after it was queued
+  struct StepGraph {
+    cudaGraphExec_t exec;
+    int n_part;
+    int launches;
+  };
+  std::map<std::tuple<int, int, int>, StepGraph> step_graphs;
   // per-kernel-class timing (fdllm_profile_enable)
   struct ProfPending {
     cudaEvent_t a, b;
@@ -249,7 +262,8 @@ int check_config(const fdllm_config* c, std::string* why) {
   auto bad = [&](const char* m) { *why = m; return FDLLM_ERR_ARG; };
   if (!c) return bad("config is NULL");
   if (c->n_layers < 1) return bad("n_layers must be >= 1");
-  if (c->d_model < 64 || c->d_model % 64) return bad("d_model must be a positive multiple of 64");
+  if (c->d_model < 64 || c->d_model % 64 || c->d_model > 8192)
+    return bad("d_model must be a multiple of 64 in [64, 8192]");
   if (c->ffn_dim < 64 || c->ffn_dim % 64) return bad("ffn_dim must be a positive multiple of 64");
   if (!(c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 128))
     return bad("head_dim must be 32, 64 or 128");
@@ -328,9 +342,10 @@ int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* 
   if (ctx->tc) {
     GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
                    ctx->n_counters};
-    KL(launch_gemm_tc(wmap, act_map(amaps, gs.nt), gs, ep, sc, ctx->stream));
+    KL(launch_gemm_tc(wmap, act_map(amaps, gs.nt), gs, ep, sc, ctx->stream, ctx->pdl));
   } else {
-    KL(launch_gemm_simt((const float*)w, (const float*)act, act_row0, K, gs, ep, ctx->stream));
+    KL(launch_gemm_simt((const float*)w, (const float*)act, act_row0, K, gs, ep, ctx->stream,
+                        ctx->pdl));
   }
   if (n_part_out) *n_part_out = gs.grid;
   return FDLLM_OK;
@@ -346,6 +361,7 @@ EpiParams epi_base(fdllm_ctx* ctx, int kind) {
   ep.cap_f = ctx->cap_f;
   ep.cap_dbg = ctx->dbg_cap;
   ep.cap_lm = ctx->lm_part_cap;
+  ep.sp = ctx->sp;
   ep.kv_pool = ctx->kv_pool;
   ep.kv_planes = ctx->kv_planes;
   ep.q_plane = ctx->q_plane;
@@ -379,6 +395,7 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   ap.head_dim = c.head_dim;
   ap.part_o = ctx->attn_po;
   ap.part_ml = ctx->attn_ml;
+  ap.counters = ctx->attn_cnt;
   ap.n_split = 1;
   ap.keys_per_split = ((L + 63) / 64) * 64;
   const double es = (double)ctx->esz;
@@ -388,28 +405,29 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   const std::string att_tag = M <= 64 ? "attn.step" : "attn.full";
   if (!ctx->tc) {
     ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
-    KL(launch_attn_simt(ap, ctx->stream));
+    KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
     return FDLLM_OK;
   }
+  // Key splits only when one CTA would stream many key tiles (long
+  // sequences, few query rows): enough CTAs to cover the SMs twice, at least
+  // 4 key tiles per split.
   const int rep = c.n_heads / c.n_kv_heads;
-  const int ctas = ((M * rep + 63) / 64) * c.n_kv_heads;
+  const int rows_per_cta = attn_rows_per_cta(M, c.n_heads, c.n_kv_heads);
+  const int ctas = ((M * rep + rows_per_cta - 1) / rows_per_cta) * c.n_kv_heads;
   const int key_tiles = (L + 63) / 64;
-  if (M <= kAttnSplitMaxM) {
+  if (M <= kAttnSplitMaxM && key_tiles > 8) {
     int want = std::max(1, (2 * ctx->num_sms) / std::max(1, ctas));
-    want = std::min(want, std::min(kMaxAttnSplit, key_tiles));
-    const int tiles_per = (key_tiles + want - 1) / want;
-    ap.keys_per_split = tiles_per * 64;
-    ap.n_split = (key_tiles + tiles_per - 1) / tiles_per;
+    want = std::min(want, std::min(kMaxAttnSplit, key_tiles / 4));
+    if (want > 1) {
+      const int tiles_per = (key_tiles + want - 1) / want;
+      ap.keys_per_split = tiles_per * 64;
+      ap.n_split = (key_tiles + tiles_per - 1) / tiles_per;
+    }
   }
   {
     const double part = ap.n_split > 1 ? (double)ap.n_split * M * c.n_heads * c.head_dim * 4.0 : 0;
     ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes + part, att_flops);
-    KL(launch_attn_mma(ap, ctx->stream));
-  }
-  if (ap.n_split > 1) {
-    ProfScope ps(ctx, "attn.combine", (double)ap.n_split * M * c.n_heads * c.head_dim * 4.0 +
-                                          qo_bytes / 2, 0.0);
-    KL(launch_attn_combine(ap, ctx->f32, ctx->stream));
+    KL(launch_attn_mma(ap, ctx->stream, ctx->pdl));
   }
   return FDLLM_OK;
 }
@@ -424,7 +442,8 @@ int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg,
   {
     ProfScope ps(ctx, "embed_rmsnorm", (double)M * d * (2.0 * es + 4.0), 0.0);
     KL(launch_embed_rmsnorm(ctx->x, r0, M, ctx->embed, d, c.vocab, ctx->layers[0].attn_norm,
-                            c.rms_eps, ctx->h, ctx->a, ctx->f32, ctx->err_dev, ctx->stream));
+                            c.rms_eps, ctx->h, ctx->a, ctx->f32, ctx->err_dev, ctx->sp,
+                            ctx->stream, ctx->pdl));
   }
   int rc;
   for (int l = 0; l < c.n_layers; ++l) {
@@ -440,7 +459,8 @@ int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg,
     if ((rc = run_gemm(ctx, "o", lw.wo, &lw.m_o, ctx->o, ctx->m_o, 0, d, M, hq, ep))) return rc;
     {
       ProfScope ps(ctx, "rmsnorm", (double)M * d * (es + 4.0), 0.0);
-      KL(launch_rmsnorm(ctx->h, 0, M, d, lw.ffn_norm, c.rms_eps, ctx->a, ctx->f32, ctx->stream));
+      KL(launch_rmsnorm(ctx->h, 0, M, d, lw.ffn_norm, c.rms_eps, ctx->a, ctx->f32, nullptr, false,
+                        ctx->stream, ctx->pdl));
     }
     ep = epi_base(ctx, EPI_SWIGLU);
     ep.f_out = ctx->f;
@@ -457,7 +477,7 @@ int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg,
       ProfScope ps(ctx, "rmsnorm", (double)nr * d * (es + 4.0), 0.0);
       KL(launch_rmsnorm(ctx->h, last ? lm0 : 0, nr, d,
                         last ? ctx->final_norm : ctx->layers[l + 1].attn_norm, c.rms_eps, ctx->a,
-                        ctx->f32, ctx->stream));
+                        ctx->f32, ctx->sp, last, ctx->stream, ctx->pdl));
     }
   }
   EpiParams ep = epi_base(ctx, EPI_LMHEAD);
@@ -501,20 +521,72 @@ int sync_state(fdllm_ctx* ctx) {
   return FDLLM_OK;
 }
 
-// One denoising step: forward for the mode + merge/select.  first = block start.
-int run_step(fdllm_ctx* ctx, int mode, bool first, int s, int B, int L, float tau, float* dbg) {
-  int n_part = 0, rc;
-  if (first || mode == FDLLM_CACHE_NONE) {
-    rc = forward(ctx, 0, L, L, s, B, dbg, &n_part);
-  } else if (mode == FDLLM_CACHE_DUAL) {
-    rc = forward(ctx, s, B, L, 0, B, dbg, &n_part);
-  } else {
-    rc = forward(ctx, s, L - s, L, 0, B, dbg, &n_part);
-  }
+// Write the step scalars the kernels read (r0, lm0, s, tau).  Each update
+// uses the next slot of a pinned ring; every call path synchronises the
+// stream before kSpRing updates are outstanding.
+int set_step_params(fdllm_ctx* ctx, int r0, int lm0, int s, float tau) {
+  StepParams* slot = ctx->sp_host + ctx->sp_slot;
+  ctx->sp_slot = (ctx->sp_slot + 1) % kSpRing;
+  *slot = StepParams{r0, lm0, s, tau};
+  CK(cudaMemcpyAsync(ctx->sp, slot, sizeof(StepParams), cudaMemcpyHostToDevice, ctx->stream));
+  return FDLLM_OK;
+}
+
+// The launches of one step: forward over rows [r0, r0+M) (r0 and lm0 come
+// from the step scalars) and the merge/select kernel.
+int enqueue_step(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int B, float tau, float* dbg,
+                 int* n_part) {
+  int rc = forward(ctx, r0, M, L, lm0, B, dbg, n_part);
   if (rc) return rc;
-  ProfScope ps(ctx, "merge_select", (double)n_part * B * 12.0, 0.0);
-  KL(launch_merge_select(ctx->lm_part, n_part, B, ctx->x, s, ctx->cfg.mask_id, tau, 1, ctx->conf,
-                         ctx->tok, ctx->unmask, ctx->state, ctx->stream));
+  ProfScope ps(ctx, "merge_select", (double)*n_part * B * 12.0, 0.0);
+  KL(launch_merge_select(ctx->lm_part, *n_part, B, ctx->x, 0, ctx->cfg.mask_id, tau, 1, ctx->conf,
+                         ctx->tok, ctx->unmask, ctx->state, ctx->sp, ctx->stream, ctx->pdl));
+  return FDLLM_OK;
+}
+
+// One denoising step: forward for the mode + merge/select.  first = block
+// start.  Steps of the same shape replay one captured CUDA graph (the kernel
+// sequence depends only on the row count, the key count and the block size;
+// the per-step scalars live in device memory).
+int run_step(fdllm_ctx* ctx, int mode, bool first, int s, int B, int L, float tau, float* dbg) {
+  int r0, M, lm0;
+  if (first || mode == FDLLM_CACHE_NONE) {
+    r0 = 0; M = L; lm0 = s;
+  } else if (mode == FDLLM_CACHE_DUAL) {
+    r0 = s; M = B; lm0 = 0;
+  } else {
+    r0 = s; M = L - s; lm0 = 0;
+  }
+  int rc = set_step_params(ctx, r0, lm0, s, tau);
+  if (rc) return rc;
+  int n_part = 0;
+  if (!ctx->graphs || ctx->prof || dbg) return enqueue_step(ctx, r0, M, L, lm0, B, tau, dbg, &n_part);
+  const auto key = std::make_tuple(M, L, B);
+  auto it = ctx->step_graphs.find(key);
+  if (it == ctx->step_graphs.end()) {
+    cudaGraph_t g = nullptr;
+    CK(cudaStreamBeginCapture(ctx->stream, cudaStreamCaptureModeRelaxed));
+    const int64_t before = ctx->launches;
+    rc = enqueue_step(ctx, r0, M, L, lm0, B, tau, nullptr, &n_part);
+    cudaError_t e = cudaStreamEndCapture(ctx->stream, &g);
+    if (rc) {
+      if (g) cudaGraphDestroy(g);
+      return rc;
+    }
+    if (e != cudaSuccess)
+      return fail(ctx, FDLLM_ERR_CUDA, std::string("graph capture: ") + cudaGetErrorString(e));
+    fdllm_ctx::StepGraph sg{};
+    e = cudaGraphInstantiate(&sg.exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess)
+      return fail(ctx, FDLLM_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
+    sg.n_part = n_part;
+    sg.launches = (int)(ctx->launches - before);
+    ctx->launches = before;
+    it = ctx->step_graphs.emplace(key, sg).first;
+  }
+  CK(cudaGraphLaunch(it->second.exec, ctx->stream));
+  ctx->launches += it->second.launches;
   return FDLLM_OK;
 }
 
@@ -634,16 +706,20 @@ GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_
     if (s > 1 && (size_t)units * (nt / 2) * 128 * sizeof(float) > ws_bytes) break;
     const int grid = (int)std::min<long long>(units, num_sms);
     // per-CTA cost in K blocks of its units, +2 per unit (pipeline fill and
-    // epilogue), +1 per unit when split (partial tile write and reduction)
+    // epilogue); a split unit also writes its float partial tile and the last
+    // one reads all of them back: (1 + s) tiles of nt/2 x 128 floats, costed
+    // in K blocks of the same bytes (one K block moves (128 + nt) x 64 bf16).
+    const double kb_bytes = (128.0 + nt) * 64 * 2;
+    const double split_cost = s > 1 ? (1.0 + s) * (nt / 2) * 128 * 4 / kb_bytes : 0.0;
     std::vector<double> load(grid, 0.0);
     for (long long u = 0; u < units; ++u) {
       const int sp = (int)(u % s);
       const int kb = (int)((long long)(sp + 1) * g.kb_total / s - (long long)sp * g.kb_total / s);
-      load[u % grid] += kb + 2.0 + (s > 1 ? 1.0 : 0.0);
+      load[u % grid] += kb + 2.0 + split_cost;
     }
     double mx = 0.0;
     for (double v : load) mx = std::max(mx, v);
-    if (mx < best * 0.995) {
+    if (mx < best * 0.9) {
       best = mx;
       best_s = s;
     }
@@ -689,6 +765,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
     if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
     if (ctx->state_host) cudaFreeHost(ctx->state_host);
     if (ctx->err_host) cudaFreeHost(ctx->err_host);
+    if (ctx->sp_host) cudaFreeHost(ctx->sp_host);
     delete ctx;
     return code;
   };
@@ -743,6 +820,9 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   const size_t attn_rows = (size_t)kAttnSplitMaxM * c.n_heads;
   ctx->attn_po = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * c.head_dim);
   ctx->attn_ml = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * 2);
+  // one counter per (query row tile of >= 16 rows, KV head) of a split launch (M <= 64)
+  const int attn_cnt_n = ((kAttnSplitMaxM * (c.n_heads / c.n_kv_heads) + 15) / 16) * c.n_kv_heads;
+  ctx->attn_cnt = (int*)dalloc(ctx, sizeof(int) * attn_cnt_n);
   const size_t max_parts = std::max<size_t>((size_t)ctx->num_sms,
                                             (size_t)((c.vocab + 127) / 128) * ((kMaxLmRows + 31) / 32));
   ctx->lm_part_cap = max_parts * kMaxLmRows;
@@ -753,6 +833,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->state = (DecodeState*)dalloc(ctx, sizeof(DecodeState));
   ctx->err_dev = (int*)dalloc(ctx, sizeof(int));
   ctx->check = (int*)dalloc(ctx, 4 * sizeof(int));
+  ctx->sp = (StepParams*)dalloc(ctx, sizeof(StepParams));
   ctx->cap_h = rows * c.d_model;
   ctx->cap_q = ctx->esz == 4 ? rows * hq : 2 * rows * hq;
   ctx->cap_kv = kv_elems;
@@ -761,12 +842,16 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
                   (void*)ctx->h, ctx->a, ctx->q, ctx->o, ctx->f, (void*)ctx->counters,
                   (void*)ctx->attn_po, (void*)ctx->attn_ml, (void*)ctx->lm_part,
                   (void*)ctx->conf, (void*)ctx->tok, (void*)ctx->unmask, (void*)ctx->state,
-                  (void*)ctx->err_dev, (void*)ctx->check})
+                  (void*)ctx->err_dev, (void*)ctx->check, (void*)ctx->sp,
+                  (void*)ctx->attn_cnt})
     if (!p) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (ctx->tc && !ctx->ws) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (cudaMallocHost(&ctx->state_host, sizeof(DecodeState)) != cudaSuccess ||
-      cudaMallocHost(&ctx->err_host, sizeof(int)) != cudaSuccess)
+      cudaMallocHost(&ctx->err_host, sizeof(int)) != cudaSuccess ||
+      cudaMallocHost(&ctx->sp_host, kSpRing * sizeof(StepParams)) != cudaSuccess)
     return bail(FDLLM_ERR_OOM, "pinned host allocation failed");
+  if (ctx->tc && init_kernel_attributes() != cudaSuccess)
+    return bail(FDLLM_ERR_CUDA, "setting kernel shared-memory limits failed");
   // page table (identity for one sequence), RoPE table (angles in double)
   std::vector<int> pt(ctx->n_pages);
   for (int i = 0; i < ctx->n_pages; ++i) pt[i] = i;
@@ -785,6 +870,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
             cudaMemset(ctx->counters, 0, sizeof(int) * ctx->n_counters) == cudaSuccess &&
             cudaMemset(ctx->err_dev, 0, sizeof(int)) == cudaSuccess &&
             cudaMemset(ctx->check, 0, 4 * sizeof(int)) == cudaSuccess &&
+            cudaMemset(ctx->attn_cnt, 0, sizeof(int) * attn_cnt_n) == cudaSuccess &&
             cudaMemset(ctx->kv_pool, 0, kv_elems * ctx->esz) == cudaSuccess &&
             cudaMemset(ctx->a, 0, ctx->esz * arows * c.d_model) == cudaSuccess &&
             cudaMemset(ctx->o, 0, ctx->esz * arows * hq) == cudaSuccess &&
@@ -983,17 +1069,22 @@ int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, const int32_t*
     if (!same)
       CK(cudaMemcpyAsync(ctx->x, current_ids, sizeof(int32_t) * L, cudaMemcpyHostToDevice,
                          ctx->stream));
-    if ((rc = forward(ctx, 0, L, L, s, B, dbg, &n_part))) return rc;
+    if ((rc = set_step_params(ctx, 0, s, s, tau))) return rc;
+    if ((rc = enqueue_step(ctx, 0, L, L, s, B, tau, dbg, &n_part))) return rc;
   } else {
+    if ((rc = set_step_params(ctx, 0, s, s, tau))) return rc;
     if ((rc = forward(ctx, 0, L, L, s, B, nullptr, &n_part))) return rc;
     CK(cudaMemcpyAsync(ctx->x, current_ids, sizeof(int32_t) * L, cudaMemcpyHostToDevice,
                        ctx->stream));
-    if (cache_mode == FDLLM_CACHE_DUAL) rc = forward(ctx, s, B, L, 0, B, dbg, &n_part);
-    else rc = forward(ctx, s, L - s, L, 0, B, dbg, &n_part);
+    if (cache_mode == FDLLM_CACHE_DUAL) {
+      if ((rc = set_step_params(ctx, s, 0, s, tau))) return rc;
+      rc = enqueue_step(ctx, s, B, L, 0, B, tau, dbg, &n_part);
+    } else {
+      if ((rc = set_step_params(ctx, s, 0, s, tau))) return rc;
+      rc = enqueue_step(ctx, s, L - s, L, 0, B, tau, dbg, &n_part);
+    }
     if (rc) return rc;
   }
-  KL(launch_merge_select(ctx->lm_part, n_part, B, ctx->x, s, c.mask_id, tau, 1, ctx->conf,
-                         ctx->tok, ctx->unmask, ctx->state, ctx->stream));
   if ((rc = sync_state(ctx))) return rc;
   CK(cudaMemcpy(conf, ctx->conf, sizeof(float) * B, cudaMemcpyDeviceToHost));
   CK(cudaMemcpy(tok, ctx->tok, sizeof(int32_t) * B, cudaMemcpyDeviceToHost));
@@ -1060,7 +1151,7 @@ int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k_out, floa
 }
 
 int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
-               int K, int splits) {
+               int K, int splits, int accumulate) {
   if (!ctx) return FDLLM_ERR_ARG;
   if (!w_dev || !x_dev || !y_dev || N < 1 || M < 1 || K < 1)
     return fail(ctx, FDLLM_ERR_ARG, "bad GEMM arguments");
@@ -1080,23 +1171,30 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
   }
   if (gs.n_tiles * gs.n_tt > ctx->n_counters)
     return fail(ctx, FDLLM_ERR_ARG, "GEMM too large for the counter buffer");
-  EpiParams ep = epi_base(ctx, EPI_STORE);
+  EpiParams ep = epi_base(ctx, accumulate ? EPI_RESID : EPI_STORE);
   ep.N = N;
   ep.M = M;
   ep.out = y_dev;
   ep.ld_out = N;
   ep.cap_out = (size_t)M * N;
+  ep.h = y_dev;
+  ep.cap_h = (size_t)M * N;
   ep.act_f32 = ctx->f32;
-  if (ctx->tc) {
-    CUtensorMap wm, xm;
-    if (!make_map(ctx, &wm, w_dev, N, K, 128) ||
-        !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt))
-      return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
-                   ctx->n_counters};
-    KL(launch_gemm_tc(&wm, &xm, gs, ep, sc, ctx->stream));
-  } else {
-    KL(launch_gemm_simt((const float*)w_dev, (const float*)x_dev, 0, K, gs, ep, ctx->stream));
+  {
+    ProfScope ps(ctx, "gemm.check",
+                 (double)N * K * ctx->esz + 2.0 * M * K * ctx->esz + 4.0 * M * N,
+                 2.0 * (ctx->tc ? 2 : 1) * M * N * K);
+    if (ctx->tc) {
+      CUtensorMap wm, xm;
+      if (!make_map(ctx, &wm, w_dev, N, K, 128) ||
+          !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt))
+        return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+      GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
+                     ctx->n_counters};
+      KL(launch_gemm_tc(&wm, &xm, gs, ep, sc, ctx->stream));
+    } else {
+      KL(launch_gemm_simt((const float*)w_dev, (const float*)x_dev, 0, K, gs, ep, ctx->stream));
+    }
   }
   return sync_state(ctx);
 }
@@ -1147,9 +1245,12 @@ int fdllm_destroy(fdllm_ctx* ctx) {
   if (ctx->stream) cudaStreamSynchronize(ctx->stream);
   prof_harvest(ctx);
   for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
+  for (auto& kv : ctx->step_graphs) cudaGraphExecDestroy(kv.second.exec);
+  ctx->step_graphs.clear();
   dfree_all(ctx);
   if (ctx->state_host) cudaFreeHost(ctx->state_host);
   if (ctx->err_host) cudaFreeHost(ctx->err_host);
+  if (ctx->sp_host) cudaFreeHost(ctx->sp_host);
   if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
   delete ctx;
   return FDLLM_OK;

@@ -6,11 +6,15 @@
 // cache (the step's own rows were written there by the QKV epilogue just
 // before).
 //
-// CTA = (row tile of 64 query rows, KV head, key split).  A query row is a
-// (position, head-in-group) pair, so the query heads that share a KV head in
-// GQA share the K/V tiles.  Four warps, 16 rows each.  K/V tiles of 64 keys
-// (one cache page) are double-buffered in shared memory with cp.async, in a
-// 16-byte-chunk XOR swizzle so ldmatrix is conflict-free.
+// CTA = (row tile of up to 64 query rows, KV head, key split).  A query row
+// is a (position, head-in-group) pair, so the query heads that share a KV
+// head in GQA share the K/V tiles.  K/V tiles of 64 keys (one cache page)
+// are double-buffered in shared memory with cp.async, in a 16-byte-chunk XOR
+// swizzle so ldmatrix is conflict-free.  The four warps are NKG key groups x
+// (4 / NKG) row groups of 16 rows: with few query rows (a 32-token block,
+// MHA: NKG = 2) the warps split every key tile between them instead of
+// idling, and merge their online-softmax states through shared memory at
+// the end.
 //
 // Every operand is two-term (hi + lo): q and K as bf16 pairs, V as fp16
 // pairs, and the softmax weights P are split the same way into fp16 pairs.
@@ -19,14 +23,20 @@
 //   PV = P_hi V_hi + P_hi V_lo + P_lo V_hi        (fp16 MMAs, f32 accumulate)
 // so the attention output carries ~16 significant bits like every other
 // stored activation of the bf16 model (see split_bf16).  Online softmax in
-// f32, exp2 domain.  With n_split > 1 each split writes unnormalised partial
-// outputs and its (max, sum) per row; attn_combine merges them.
+// f32, exp2 domain.
+//
+// With n_split > 1 (long sequences) each split writes unnormalised partial
+// outputs and its (max, sum) per row; the last split CTA of a (row tile, KV
+// head) to arrive (a self-resetting counter) merges all splits in split
+// order and writes o, so the result does not depend on arrival order.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace fd {
 
 namespace {
+
+constexpr int kMaxSplit = 16;
 
 FD_DEV void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
@@ -69,29 +79,35 @@ FD_DEV uint32_t swz(int r, int ch) {
   return (uint32_t)(r * HD * 2 + ((ch ^ (r & 7)) << 4));
 }
 
-template <int HD>
+template <int HD, int NKG>
 __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   constexpr int TILE = 64 * HD * 2;  // bytes of one [64][HD] 2-byte tile
   constexpr int CH = HD / 8;         // 16-byte chunks per row
+  constexpr int NRG = 4 / NKG;       // row groups of 16 rows
+  constexpr int KEYS = 64 / NKG;     // keys of a tile per key group
+  constexpr int NNT = KEYS / 8;      // 8-key n-tiles per key group
   extern __shared__ __align__(128) uint8_t sm[];
   // layout: Q hi, Q lo, then per buffer b: K hi, K lo, V hi, V lo
   const uint32_t q_s = smem_u32(sm);
   auto kv_s = [&](int buf, int plane) { return q_s + (2 + buf * 4 + plane) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rg = warp % NRG, kg = warp / NRG;
   const int H = p.n_heads, Hkv = p.n_kv_heads, rep = H / Hkv;
   const int g = blockIdx.y;
   const int rows_total = p.M * rep;
-  const int row0 = blockIdx.x * 64;
+  const int row0 = blockIdx.x * (16 * NRG);
   const int key_lo = blockIdx.z * p.keys_per_split;
   const int key_hi = min(p.L, key_lo + p.keys_per_split);
   const int n_kt = (key_hi - key_lo + 63) / 64;
 
   const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q);
   const uint16_t* pool = reinterpret_cast<const uint16_t*>(p.kv_pool);
+  pdl_trigger();
+  pdl_wait();
 
-  // ---- Q tiles (hi and lo planes)
-  for (int idx = tid; idx < 64 * CH; idx += 128) {
+  // ---- Q tiles (hi and lo planes), 16 * NRG rows
+  for (int idx = tid; idx < 16 * NRG * CH; idx += 128) {
     const int i = idx / CH, ch = idx % CH;
     const int r = row0 + i;
     const bool ok = r < rows_total;
@@ -117,7 +133,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   load_kv(0, 0);
   cp_async_commit();
 
-  const bool warp_active = row0 + warp * 16 < rows_total;
+  const bool warp_active = row0 + rg * 16 < rows_total;
   const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // 1/sqrt(hd) * log2(e)
   float oacc[HD / 8][4];
 #pragma unroll
@@ -132,20 +148,20 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     __syncthreads();
     const int buf = kt & 1;
     if (warp_active) {
-      // ---- S = Q K^T for 64 keys (8 n-tiles of 8)
-      float s[8][4];
+      // ---- S = Q K^T for this warp's KEYS keys of the tile
+      float s[NNT][4];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+      for (int nt = 0; nt < NNT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
         uint32_t qh[4], ql[4];
-        const uint32_t qa = swz<HD>(warp * 16 + (lane & 15), 2 * kk + (lane >> 4));
+        const uint32_t qa = swz<HD>(rg * 16 + (lane & 15), 2 * kk + (lane >> 4));
         ldsm_x4(q_s + qa, qh);
         ldsm_x4(q_s + TILE + qa, ql);
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
+        for (int np = 0; np < NNT / 2; ++np) {
           uint32_t kh[4], kl[4];
-          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int key = kg * KEYS + np * 16 + (lane & 7) + ((lane >> 4) << 3);
           const uint32_t ka = swz<HD>(key, 2 * kk + ((lane >> 3) & 1));
           ldsm_x4(kv_s(buf, 0) + ka, kh);
           ldsm_x4(kv_s(buf, 1) + ka, kl);
@@ -158,10 +174,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
         }
       }
       // ---- online softmax (rows lane/4 and lane/4 + 8)
-      const int kbase = key_lo + kt * 64 + 2 * (lane & 3);
+      const int kbase = key_lo + kt * 64 + kg * KEYS + 2 * (lane & 3);
       float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < NNT; ++nt) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const bool ok = kbase + nt * 8 + (c & 1) < key_hi;
@@ -175,6 +191,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
         tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
         tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
         const float mnew = fmaxf(mrow[r], tmax[r]);
+        // a key group may see only masked keys in a ragged last tile
         alpha[r] = (mrow[r] == -INFINITY) ? 0.0f : exp2f(mrow[r] - mnew);
         mrow[r] = mnew;
         lrow[r] *= alpha[r];
@@ -186,13 +203,13 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
         oacc[j][2] *= alpha[1];
         oacc[j][3] *= alpha[1];
       }
-      uint32_t ph[8][2], pl[8][2];
+      uint32_t ph[NNT][2], pl[NNT][2];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < NNT; ++nt) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const float p0 = exp2f(s[nt][2 * r] - mrow[r]);
-          const float p1 = exp2f(s[nt][2 * r + 1] - mrow[r]);
+          const float p0 = mrow[r] == -INFINITY ? 0.0f : exp2f(s[nt][2 * r] - mrow[r]);
+          const float p1 = mrow[r] == -INFINITY ? 0.0f : exp2f(s[nt][2 * r + 1] - mrow[r]);
           const __half2 hi = __floats2half2_rn(p0, p1);
           const float2 hf = __half22float2(hi);
           const __half2 lo = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
@@ -203,7 +220,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
       }
       // ---- O += P V
 #pragma unroll
-      for (int kk2 = 0; kk2 < 4; ++kk2) {
+      for (int kk2 = 0; kk2 < NNT / 2; ++kk2) {
         const uint32_t ah[4] = {ph[2 * kk2][0], ph[2 * kk2][1], ph[2 * kk2 + 1][0],
                                 ph[2 * kk2 + 1][1]};
         const uint32_t al[4] = {pl[2 * kk2][0], pl[2 * kk2][1], pl[2 * kk2 + 1][0],
@@ -211,7 +228,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
 #pragma unroll
         for (int j = 0; j < HD / 8; j += 2) {
           uint32_t vh[4], vl[4];
-          const int key = kk2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+          const int key = kg * KEYS + kk2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
           const uint32_t va = swz<HD>(key, j + (lane >> 4));
           ldsm_x4_t(kv_s(buf, 2) + va, vh);
           ldsm_x4_t(kv_s(buf, 3) + va, vl);
@@ -227,7 +244,46 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     __syncthreads();
   }
 
-  if (!warp_active) return;
+  // ---- merge the key groups of each row group (shared memory, fixed order)
+  if (NKG > 1) {
+    // per warp: 32 lanes x (HD/2 accumulators + 2 max + 2 sums) floats,
+    // placed over the (now unused) K/V buffers
+    constexpr int PER_LANE = HD / 2 + 4;
+    float* xch = reinterpret_cast<float*>(sm + 2 * TILE);
+    float* mine = xch + (size_t)(warp * 32 + lane) * PER_LANE;
+    if (kg > 0) {
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mine[j * 4 + c] = oacc[j][c];
+      mine[HD / 2] = mrow[0];
+      mine[HD / 2 + 1] = mrow[1];
+      mine[HD / 2 + 2] = lrow[0];
+      mine[HD / 2 + 3] = lrow[1];
+    }
+    __syncthreads();
+    if (kg == 0) {
+      for (int k = 1; k < NKG; ++k) {
+        const float* other = xch + (size_t)((k * NRG + rg) * 32 + lane) * PER_LANE;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float mo = other[HD / 2 + r], lo_ = other[HD / 2 + 2 + r];
+          const float mn = fmaxf(mrow[r], mo);
+          const float a = (mrow[r] == -INFINITY) ? 0.0f : exp2f(mrow[r] - mn);
+          const float b = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+#pragma unroll
+          for (int j = 0; j < HD / 8; ++j) {
+            oacc[j][2 * r] = oacc[j][2 * r] * a + other[j * 4 + 2 * r] * b;
+            oacc[j][2 * r + 1] = oacc[j][2 * r + 1] * a + other[j * 4 + 2 * r + 1] * b;
+          }
+          lrow[r] = lrow[r] * a + lo_ * b;
+          mrow[r] = mn;
+        }
+      }
+    }
+  }
+  const bool writer = warp_active && kg == 0;
+
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
@@ -237,7 +293,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   const int hq = H * HD;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int rr = row0 + warp * 16 + (lane >> 2) + 8 * r;
+    if (!writer) break;
+    const int rr = row0 + rg * 16 + (lane >> 2) + 8 * r;
     if (rr >= rows_total) continue;
     const int m = rr / rep, head = g * rep + rr % rep;
     const size_t orow = (size_t)m * H + head;
@@ -269,33 +326,136 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
       }
     }
   }
+  if (p.n_split == 1) return;
+
+  // ---- split merge by the last split CTA of this (row tile, KV head)
+  __shared__ int s_last;
+  __shared__ float s_w[64][kMaxSplit];
+  __shared__ float s_inv[64];
+  __threadfence();
+  __syncthreads();
+  int* cnt = p.counters + blockIdx.y * gridDim.x + blockIdx.x;
+  if (tid == 0) {
+    const int prev = atomicAdd(cnt, 1);
+    s_last = (prev == p.n_split - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int n_rows = min(16 * NRG, rows_total - row0);
+  if (tid < n_rows) {  // per-row split weights
+    const int rr = row0 + tid;
+    const size_t orow = (size_t)(rr / rep) * H + g * rep + rr % rep;
+    float mc[kMaxSplit], lc[kMaxSplit];
+    float mstar = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxSplit; ++c) {
+      mc[c] = c < p.n_split ? __ldcg(p.part_ml + ((size_t)c * rows_all + orow) * 2) : -INFINITY;
+      lc[c] = c < p.n_split ? __ldcg(p.part_ml + ((size_t)c * rows_all + orow) * 2 + 1) : 0.0f;
+      mstar = fmaxf(mstar, mc[c]);
+    }
+    float den = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kMaxSplit; ++c) {
+      const float w = mc[c] == -INFINITY ? 0.0f : exp2f(mc[c] - mstar);
+      s_w[tid][c] = w;
+      den += w * lc[c];
+    }
+    s_inv[tid] = 1.0f / den;
+  }
+  __syncthreads();
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
+  // 8 outputs per thread per pass, every partial load issued before any store
+  for (int base = 0; base < n_rows * HD; base += 128 * 8) {
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    for (int c = 0; c < p.n_split; ++c) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int idx = base + e * 128 + tid;
+        if (idx < n_rows * HD) {
+          const int i = idx / HD, d = idx % HD;
+          const int rr = row0 + i;
+          const size_t orow = (size_t)(rr / rep) * H + g * rep + rr % rep;
+          acc[e] += s_w[i][c] * __ldcg(p.part_o + ((size_t)c * rows_all + orow) * HD + d);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int idx = base + e * 128 + tid;
+      if (idx < n_rows * HD) {
+        const int i = idx / HD, d = idx % HD;
+        const int rr = row0 + i;
+        const int m = rr / rep, head = g * rep + rr % rep;
+        __nv_bfloat16 hi, lo;
+        split_bf16(acc[e] * s_inv[i], hi, lo);
+        const size_t off = (size_t)pair_row(m) * hq + (size_t)head * HD + d;
+        o[off] = hi;
+        o[off + (size_t)PAIR_LO * hq] = lo;
+      }
+    }
+  }
+  if (tid == 0) *cnt = 0;
 }
 
-template <int HD>
-cudaError_t launch_hd(const AttnParams& p, cudaStream_t st) {
+template <int HD, int NKG>
+cudaError_t set_attr() {
+  return cudaFuncSetAttribute(attn_mma_kernel<HD, NKG>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, 10 * 64 * HD * 2);
+}
+
+template <int HD, int NKG>
+cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
   constexpr int smem = 10 * 64 * HD * 2;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<HD>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_attr<HD, NKG>();
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
-  dim3 grid((rows + 63) / 64, p.n_kv_heads, p.n_split);
-  attn_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
-  return cudaGetLastError();
+  const int rows_per_cta = 16 * (4 / NKG);
+  dim3 grid((rows + rows_per_cta - 1) / rows_per_cta, p.n_kv_heads, p.n_split);
+  return launch_k(pdl, attn_mma_kernel<HD, NKG>, grid, dim3(128), (size_t)smem, st, p);
+}
+
+template <int HD>
+cudaError_t launch_nkg(const AttnParams& p, cudaStream_t st, bool pdl) {
+  const int rows = p.M * (p.n_heads / p.n_kv_heads);
+  if (rows <= 16) return launch_hd<HD, 4>(p, st, pdl);
+  if (rows <= 32) return launch_hd<HD, 2>(p, st, pdl);
+  return launch_hd<HD, 1>(p, st, pdl);
 }
 
 }  // namespace
 
-cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st) {
-  if (p.kv_planes != 4) return cudaErrorInvalidValue;
+int attn_rows_per_cta(int M, int n_heads, int n_kv_heads) {
+  const int rows = M * (n_heads / n_kv_heads);
+  return rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
+}
+
+cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl) {
+  if (p.kv_planes != 4 || p.n_split < 1 || p.n_split > kMaxSplit) return cudaErrorInvalidValue;
   switch (p.head_dim) {
-    case 64: return launch_hd<64>(p, st);
-    case 128: return launch_hd<128>(p, st);
+    case 64: return launch_nkg<64>(p, st, pdl);
+    case 128: return launch_nkg<128>(p, st, pdl);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t gemm_tc_init_attributes();
+
+cudaError_t init_kernel_attributes() {
+  cudaError_t e = set_attr<64, 1>();
+  if (e == cudaSuccess) e = set_attr<64, 2>();
+  if (e == cudaSuccess) e = set_attr<64, 4>();
+  if (e == cudaSuccess) e = set_attr<128, 1>();
+  if (e == cudaSuccess) e = set_attr<128, 2>();
+  if (e == cudaSuccess) e = set_attr<128, 4>();
+  if (e == cudaSuccess) e = gemm_tc_init_attributes();
+  return e;
 }
 
 }  // namespace fd

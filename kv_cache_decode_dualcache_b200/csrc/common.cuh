@@ -146,6 +146,17 @@ FD_DEV uint64_t global_timer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel in the
+// stream is still running.  pdl_wait() blocks until that kernel has completed
+// and its memory is visible: every read of data the previous kernel wrote,
+// and every write the previous kernel might still read, comes after it.
+// pdl_trigger() lets the next kernel launch once every CTA of this grid has
+// issued it (or exited).  Without the attribute both are no-ops.
+FD_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+FD_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 FD_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

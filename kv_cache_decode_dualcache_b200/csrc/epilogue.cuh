@@ -19,8 +19,9 @@ namespace fd {
 constexpr int EPI_THREADS = 128;
 constexpr int CHUNK_T = 32;
 
-FD_DEV size_t kv_offset(const EpiParams& ep, int pos, int plane, int head, int dim) {
-  const int page = ep.page_table[pos / KV_PAGE];
+// Element offset of (position, plane, kv head, dim) in the paged cache, with
+// the position's page already looked up.
+FD_DEV size_t kv_offset_pg(const EpiParams& ep, int page, int pos, int plane, int head, int dim) {
   const int slot = pos % KV_PAGE;
   return ((((size_t)ep.layer * ep.n_pages + page) * ep.kv_planes + plane) * ep.n_kv_heads +
           head) * (size_t)(KV_PAGE * ep.head_dim) +
@@ -46,12 +47,22 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
       break;
     }
     case EPI_RESID: {
-      if (n < ep.N)
-        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t)
-        {
+      // All 32 loads of h are issued before any store: interleaving them
+      // would serialise one memory round trip per token row (the compiler
+      // cannot prove the stores do not alias the next loads).
+      if (n < ep.N) {
+        const int nt = min(CHUNK_T, ep.M - t0);
+        float hv[CHUNK_T];
+#pragma unroll
+        for (int t = 0; t < CHUNK_T; ++t)
+          hv[t] = (t < nt) ? ep.h[(size_t)(t0 + t) * ep.N + n] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < CHUNK_T; ++t) {
+          if (t >= nt) break;
           const size_t i = (size_t)(t0 + t) * ep.N + n;
-          if (FD_CHECK(i < ep.cap_h, ep.check, 2, i, ep.cap_h)) ep.h[i] += tile[t * 128 + e];
+          if (FD_CHECK(i < ep.cap_h, ep.check, 2, i, ep.cap_h)) ep.h[i] = hv[t] + tile[t * 128 + e];
         }
+      }
       break;
     }
     case EPI_SWIGLU: {
@@ -89,20 +100,41 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
       const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
       const int dh = n % hd;
       const bool is_q = n < hq, is_v = n >= hq + hk;
-      for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
+      const int pos0 = ep.sp ? ep.sp->r0 : ep.pos0;
+      const int nt = min(CHUNK_T, ep.M - t0);
+      if (nt <= 0) break;  // chunk past the last token row of the tile
+      // Loads first (RoPE table for the chunk's 32 positions), stores after:
+      // see EPI_RESID.
+      float2 cs[CHUNK_T];
+      if (!is_v) {
+#pragma unroll
+        for (int t = 0; t < CHUNK_T; ++t)
+          cs[t] = (t < nt) ? __ldg(&ep.rope[(size_t)(pos0 + t0 + t) * half + (dh % half)])
+                           : make_float2(1.0f, 0.0f);
+      }
+      // the chunk's 32 positions span at most two cache pages
+      const int pidx0 = (pos0 + t0) / KV_PAGE;
+      int page0 = 0, page1 = 0;
+      if (!is_q) {
+        page0 = __ldg(&ep.page_table[pidx0]);
+        page1 = __ldg(&ep.page_table[(pos0 + t0 + nt - 1) / KV_PAGE]);
+      }
+#pragma unroll
+      for (int t = 0; t < CHUNK_T; ++t) {
+        if (t >= nt) break;
         const int tok = t0 + t;
-        const int pos = ep.pos0 + tok;
+        const int pos = pos0 + tok;
         float y = tile[t * 128 + e];
         if (!is_v) {
-          const float2 cs = ep.rope[(size_t)pos * half + (dh % half)];
           if (dh < half) {
             const float x2 = tile[t * 128 + e + half];
-            y = y * cs.x - x2 * cs.y;
+            y = y * cs[t].x - x2 * cs[t].y;
           } else {
             const float x1 = tile[t * 128 + e - half];
-            y = y * cs.x + x1 * cs.y;
+            y = y * cs[t].x + x1 * cs[t].y;
           }
         }
+        const int page = (pos / KV_PAGE == pidx0) ? page0 : page1;
         if (F32) {
           float* kv = reinterpret_cast<float*>(ep.kv_pool);
           if (is_q) {
@@ -110,8 +142,8 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
             if (FD_CHECK(i < ep.cap_q, ep.check, 4, i, ep.cap_q))
               reinterpret_cast<float*>(ep.q_out)[i] = y;
           } else {
-            const size_t i = is_v ? kv_offset(ep, pos, 1, (n - hq - hk) / hd, dh)
-                                  : kv_offset(ep, pos, 0, (n - hq) / hd, dh);
+            const size_t i = is_v ? kv_offset_pg(ep, page, pos, 1, (n - hq - hk) / hd, dh)
+                                  : kv_offset_pg(ep, page, pos, 0, (n - hq) / hd, dh);
             if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
           }
         } else if (is_q) {
@@ -128,7 +160,8 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
           split_bf16(y, hi, lo);
           __nv_bfloat16* k = reinterpret_cast<__nv_bfloat16*>(ep.kv_pool);
           const int head = (n - hq) / hd;
-          const size_t i0 = kv_offset(ep, pos, 0, head, dh), i1 = kv_offset(ep, pos, 1, head, dh);
+          const size_t i0 = kv_offset_pg(ep, page, pos, 0, head, dh);
+          const size_t i1 = kv_offset_pg(ep, page, pos, 1, head, dh);
           if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
             k[i0] = hi;
             k[i1] = lo;
@@ -138,7 +171,8 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
           split_f16(y, hi, lo);
           __half* v = reinterpret_cast<__half*>(ep.kv_pool);
           const int head = (n - hq - hk) / hd;
-          const size_t i0 = kv_offset(ep, pos, 2, head, dh), i1 = kv_offset(ep, pos, 3, head, dh);
+          const size_t i0 = kv_offset_pg(ep, page, pos, 2, head, dh);
+          const size_t i1 = kv_offset_pg(ep, page, pos, 3, head, dh);
           if (FD_CHECK(i1 < ep.cap_kv, ep.check, 6, i1, ep.cap_kv)) {
             v[i0] = hi;
             v[i1] = lo;

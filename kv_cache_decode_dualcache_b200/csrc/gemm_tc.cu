@@ -129,17 +129,43 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  pdl_trigger();  // the next kernel may launch onto SMs this grid is not using
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
+      // The weight tiles do not depend on the previous kernel: the first
+      // STAGES of them are requested before waiting for it; activation tiles
+      // only after.
       uint32_t it = 0;
       bool ok = true;
+      int pre = 0;  // stages whose weight tile was prefetched
+      {
+        int u = blockIdx.x, kb = 0;
+        if (u < gs.units) kb = decode_unit(gs, u).kb_lo;
+        while (u < gs.units && pre < STAGES) {
+          const UnitCoord c = decode_unit(gs, u);
+          if (kb >= c.kb_hi) {
+            u += gridDim.x;
+            if (u < gs.units) kb = decode_unit(gs, u).kb_lo;
+            continue;
+          }
+          mbar_arrive_expect_tx(&full[pre], STAGE_TX);
+          tma_load_2d(a_st + pre * A_STAGE_BYTES, &wmap, &full[pre], kb * BK, c.tile * 128);
+          ++pre;
+          ++kb;
+        }
+      }
+      pdl_wait();
       for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x) {
         const UnitCoord c = decode_unit(gs, u);
         for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
+          if (it < (uint32_t)pre) {  // weight tile already requested
+            tma_load_2d(b_st + s * Lay::B_STAGE_BYTES, &amap, &full[s], kb * BK, c.tt * NT);
+            continue;
+          }
           if (!mbar_wait(&empty[s], ph ^ 1u, sc.err, abort_flag)) { ok = false; break; }
           FD_CHECK(kb >= 0 && kb < gs.kb_total && c.tile < gs.n_tiles && c.tt < gs.n_tt, ep.check,
                    20, kb, c.tile * 65536 + c.tt);
@@ -188,6 +214,7 @@ __global__ void __launch_bounds__(192, 1)
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;
     const int e = quad * 32 + lane;  // feature row = TMEM lane
+    pdl_wait();                      // reads / writes of the previous kernel's data follow
     uint32_t local = 0;
     for (int u = blockIdx.x; u < gs.units; u += gridDim.x, ++local) {
       const UnitCoord c = decode_unit(gs, u);
@@ -275,18 +302,22 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int NT>
+cudaError_t set_attr_nt() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcLayout<NT>::SMEM);
+}
+
+template <int NT>
 cudaError_t launch_nt(const CUtensorMap* w_map, const CUtensorMap* act_map, const GemmShape& gs,
-                      const EpiParams& ep, const GemmScratch& sc, cudaStream_t st) {
+                      const EpiParams& ep, const GemmScratch& sc, cudaStream_t st, bool pdl) {
   static bool attr_set = false;
-  const int smem = TcLayout<NT>::SMEM;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_attr_nt<NT>();
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  gemm_tc_kernel<NT><<<gs.grid, 192, smem, st>>>(*w_map, *act_map, gs, ep, sc);
-  return cudaGetLastError();
+  return launch_k(pdl, gemm_tc_kernel<NT>, dim3(gs.grid), dim3(192), (size_t)TcLayout<NT>::SMEM,
+                  st, *w_map, *act_map, gs, ep, sc);
 }
 
 }  // namespace
@@ -302,14 +333,21 @@ int gemm_tc_smem_bytes(int nt) {
 
 cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
                            const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl) {
   if (ep.kind == EPI_LMHEAD && gs.M > LM_MAX_ROWS) return cudaErrorInvalidValue;
   switch (gs.nt) {
-    case 64: return launch_nt<64>(w_map, act_map, gs, ep, sc, st);
-    case 128: return launch_nt<128>(w_map, act_map, gs, ep, sc, st);
-    case 256: return launch_nt<256>(w_map, act_map, gs, ep, sc, st);
+    case 64: return launch_nt<64>(w_map, act_map, gs, ep, sc, st, pdl);
+    case 128: return launch_nt<128>(w_map, act_map, gs, ep, sc, st, pdl);
+    case 256: return launch_nt<256>(w_map, act_map, gs, ep, sc, st, pdl);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t gemm_tc_init_attributes() {
+  cudaError_t e = set_attr_nt<64>();
+  if (e == cudaSuccess) e = set_attr_nt<128>();
+  if (e == cudaSuccess) e = set_attr_nt<256>();
+  return e;
 }
 
 }  // namespace fd

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace fd {
 
 enum EpiKind : int {
@@ -14,6 +16,16 @@ enum EpiKind : int {
   EPI_RESID = 2,   // h[t, n] += y  (float residual stream)
   EPI_SWIGLU = 3,  // 64-row gate/up groups: f[t, j] = silu(gate) * up
   EPI_LMHEAD = 4,  // online max / argmax / sum-exp over vocab tiles
+};
+
+// Per-step scalars read by the kernels from device memory, so that one
+// captured CUDA graph serves every block of a generation: the host writes
+// them (one small copy) before each replay.
+struct StepParams {
+  int r0;            // absolute position of the forward's first row
+  int lm0;           // first LM-head row within the forward
+  int s;             // block start position (unmask target)
+  float tau;         // confidence threshold
 };
 
 // Everything a GEMM epilogue needs.  Token index t is the row within the
@@ -47,6 +59,7 @@ struct EpiParams {
   int mask_id;
   float* lm_part;    // [n_part][M] of (m, s, arg) triples
   float* dbg_logits; // optional [M, N] float logits (mask id included)
+  const StepParams* sp;  // when set, pos0 = sp->r0 (device-side step scalars)
   // Capacities (elements) of the output buffers, used only by builds with
   // FDLLM_CHECKS, where every store is bounds-checked and a violation is
   // recorded in check[0..3] (count, code, index, aux) instead of performed.
@@ -80,14 +93,36 @@ struct GemmScratch {
 // blocks over the persistent grid, within ws_bytes of split-K workspace.
 GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes);
 
+// Launch with the programmatic stream-serialization attribute (when pdl).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Sets the dynamic shared-memory limits of every kernel (call once per
+// device before any launch, outside stream capture).
+cudaError_t init_kernel_attributes();
+
 // Launchers (return cudaError_t of the launch).
 // bf16 model: activations in two-term pair rows, token tiles of nt/2 tokens.
 cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
                            const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
-                           cudaStream_t st);
+                           cudaStream_t st, bool pdl = false);
 // fp32 model: plain [M, K] activations starting at row act_row0.
 cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int K,
-                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st);
+                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st,
+                             bool pdl = false);
 int gemm_tc_smem_bytes(int nt);
 
 struct AttnParams {
@@ -105,19 +140,25 @@ struct AttnParams {
   int keys_per_split;  // multiple of 64
   float* part_o;       // [n_split][M*H][hd]
   float* part_ml;      // [n_split][M*H][2]
+  int* counters;       // [row tiles * Hkv] arrival counters of the splits (self-resetting)
 };
 
-cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st);
-cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st);
-cudaError_t launch_attn_combine(const AttnParams& p, int f32, cudaStream_t st);
+cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl = false);
+// Query rows per CTA of launch_attn_mma for M query positions (16, 32 or 64).
+int attn_rows_per_cta(int M, int n_heads, int n_kv_heads);
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl = false);
 
-// h[i] = embed[x[r0+i]]; a[i] = RMSNorm(h[i]) * g, i in [0, M).
+// h[i] = embed[x[r0+i]]; a[i] = RMSNorm(h[i]) * g, i in [0, M).  With sp,
+// r0 = sp->r0.
 cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
                                  int vocab, const float* g, float eps, float* h, void* a,
-                                 int f32, int* err, cudaStream_t st);
+                                 int f32, int* err, const StepParams* sp, cudaStream_t st,
+                                 bool pdl = false);
 // a[i] = RMSNorm(h[h_row0 + i]) * g, i in [0, M).  bf16: two-term pair rows.
+// With sp and rows_from_lm0, h_row0 = sp->lm0.
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
-                           void* a, int f32, cudaStream_t st);
+                           void* a, int f32, const StepParams* sp, bool rows_from_lm0,
+                           cudaStream_t st, bool pdl = false);
 
 struct DecodeState {
   int remaining;     // masked positions left in the block after the step
@@ -128,12 +169,15 @@ struct DecodeState {
 
 // Merge LM-head partials into conf/tok for n rows and, when select != 0,
 // apply the threshold-or-fallback unmask rule to x[s .. s+n).
+// With sp, s = sp->s and tau = sp->tau.
 cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,
                                 int mask_id, float tau, int select, float* conf, int* tok,
-                                uint8_t* unmask, DecodeState* state, cudaStream_t st);
+                                uint8_t* unmask, DecodeState* state, const StepParams* sp,
+                                cudaStream_t st, bool pdl = false);
 
-cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st);
+cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st,
+                               bool pdl = false);
 cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
-                                cudaStream_t st);
+                                cudaStream_t st, bool pdl = false);
 
 }  // namespace fd

@@ -1,6 +1,6 @@
 // CUDA-core kernels: embedding + RMSNorm, RMSNorm, the LM-head partial
-// merge fused with the threshold/unmask/scatter step, the float32 GEMM and
-// attention of the fp32 model, and the split-KV attention combine.
+// merge fused with the threshold/unmask/scatter step, and the float32 GEMM
+// and attention of the fp32 model.
 #include <type_traits>
 
 #include "common.cuh"
@@ -10,6 +10,8 @@
 namespace fd {
 
 namespace {
+
+constexpr int RMS_VPT = 32;   // values per thread: d_model up to 8192 with 256 threads
 
 // Deterministic block sum (fixed tree) for blockDim.x a multiple of 32.
 FD_DEV float block_sum(float v, float* red) {
@@ -40,11 +42,25 @@ FD_DEV float block_max(float v, float* red) {
 // x[r0 + row].  fp32 model: a is [M, d] float; bf16 model: a is two-term in
 // pair rows.
 template <typename T>
-__global__ void rmsnorm_kernel(const int* x, int r0, const T* embed, int vocab, float* h,
-                               int h_row0, int d, const float* g, float eps, T* a, int* err) {
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x, int r0,
+                                                      const T* __restrict__ embed, int vocab,
+                                                      float* __restrict__ h, int h_row0, int d,
+                                                      const float* __restrict__ g, float eps,
+                                                      T* __restrict__ a, int* err,
+                                                      const StepParams* sp, int rows_from_lm0) {
+  // The row stays in registers (d <= 256 * RMS_VPT): every load is issued
+  // before any store.
+  constexpr int VPT = RMS_VPT;
   __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;
+  if (sp) {
+    if (x) r0 = sp->r0;
+    if (rows_from_lm0) h_row0 = sp->lm0;
+  }
   float* hr = h + (size_t)(h_row0 + row) * d;
+  float v[VPT];
   if (x) {
     int tok = x[r0 + row];
     if (tok < 0 || tok >= vocab) {
@@ -52,26 +68,46 @@ __global__ void rmsnorm_kernel(const int* x, int r0, const T* embed, int vocab, 
       tok = 0;
     }
     const T* er = embed + (size_t)tok * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) hr[j] = to_f(er[j]);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int j = threadIdx.x + k * 256;
+      v[k] = j < d ? to_f(er[j]) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int j = threadIdx.x + k * 256;
+      if (j < d) hr[j] = v[k];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int j = threadIdx.x + k * 256;
+      v[k] = j < d ? hr[j] : 0.0f;
+    }
   }
   float ss = 0.0f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    const float v = hr[j];
-    ss += v * v;
-  }
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) ss += v[k] * v[k];
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
   if (std::is_same<T, float>::value) {
-    for (int j = threadIdx.x; j < d; j += blockDim.x)
-      a[(size_t)row * d + j] = from_f<T>(hr[j] * inv * g[j]);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int j = threadIdx.x + k * 256;
+      if (j < d) a[(size_t)row * d + j] = from_f<T>(v[k] * inv * __ldg(&g[j]));
+    }
   } else {
     __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(a);
     const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-      __nv_bfloat16 hi, lo;
-      split_bf16(hr[j] * inv * g[j], hi, lo);
-      ab[r_hi + j] = hi;
-      ab[r_lo + j] = lo;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int j = threadIdx.x + k * 256;
+      if (j < d) {
+        __nv_bfloat16 hi, lo;
+        split_bf16(v[k] * inv * __ldg(&g[j]), hi, lo);
+        ab[r_hi + j] = hi;
+        ab[r_lo + j] = lo;
+      }
     }
   }
 }
@@ -79,10 +115,16 @@ __global__ void rmsnorm_kernel(const int* x, int r0, const T* embed, int vocab, 
 // ------------------------------------------------------- merge + select
 __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
                                     int mask_id, float tau, int select, float* conf, int* tok,
-                                    uint8_t* unmask, DecodeState* state) {
+                                    uint8_t* unmask, DecodeState* state, const StepParams* sp) {
   __shared__ float s_conf[256];
   __shared__ int s_tok[256];
   __shared__ int s_best;
+  pdl_trigger();
+  pdl_wait();
+  if (sp) {
+    s = sp->s;
+    tau = sp->tau;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int t = warp; t < n; t += blockDim.x >> 5) {
     SoftmaxState st = sm_empty();
@@ -131,11 +173,15 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
 }
 
 __global__ void fill_kernel(int* x, int from, int to, int v) {
+  pdl_trigger();
+  pdl_wait();
   const int i = from + blockIdx.x * blockDim.x + threadIdx.x;
   if (i < to) x[i] = v;
 }
 
 __global__ void check_prompt_kernel(const int* x, int n, int vocab, int mask_id, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     const int t = x[i];
@@ -154,6 +200,8 @@ __global__ void __launch_bounds__(128)
   __shared__ float as_[32][33];
   __shared__ float tile[32 * 128];
   __shared__ SoftmaxState lm[32];
+  pdl_trigger();
+  pdl_wait();
   const int e = threadIdx.x;
   const int tile_idx = blockIdx.x % gs.n_tiles;
   const int tt = blockIdx.x / gs.n_tiles;
@@ -202,6 +250,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   using VT = float;
   extern __shared__ float sh[];
   __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
   float* qs = sh;               // [hd]
   float* sc = sh + p.head_dim;  // [L]
   const int m = blockIdx.x, head = blockIdx.y;
@@ -244,115 +294,71 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   }
 }
 
-// Combine split-KV partial attention outputs (log2-domain maxima).
-template <typename T>
-__global__ void attn_combine_kernel(AttnParams p) {
-  const int row = blockIdx.x;  // m * H + head
-  const int rows = p.M * p.n_heads;
-  const int hd = p.head_dim;
-  float mstar = -INFINITY;
-  for (int c = 0; c < p.n_split; ++c) mstar = fmaxf(mstar, p.part_ml[((size_t)c * rows + row) * 2]);
-  float den = 0.0f;
-  for (int c = 0; c < p.n_split; ++c) {
-    const float m = p.part_ml[((size_t)c * rows + row) * 2];
-    if (m != -INFINITY) den += exp2f(m - mstar) * p.part_ml[((size_t)c * rows + row) * 2 + 1];
-  }
-  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
-    float num = 0.0f;
-    for (int c = 0; c < p.n_split; ++c) {
-      const float m = p.part_ml[((size_t)c * rows + row) * 2];
-      if (m != -INFINITY) num += exp2f(m - mstar) * p.part_o[((size_t)c * rows + row) * hd + d];
-    }
-    const float y = num / den;
-    if (std::is_same<T, float>::value) {
-      reinterpret_cast<float*>(p.o)[(size_t)row * hd + d] = y;
-    } else {
-      // two-term pair rows of [M, H*hd]
-      const int m = row / p.n_heads, head = row % p.n_heads;
-      const size_t hq = (size_t)p.n_heads * hd;
-      const size_t off = (size_t)pair_row(m) * hq + (size_t)head * hd + d;
-      __nv_bfloat16 hi, lo;
-      split_bf16(y, hi, lo);
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
-      o[off] = hi;
-      o[off + (size_t)PAIR_LO * hq] = lo;
-    }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
                                  int vocab, const float* g, float eps, float* h, void* a,
-                                 int f32, int* err, cudaStream_t st) {
+                                 int f32, int* err, const StepParams* sp, cudaStream_t st,
+                                 bool pdl) {
   if (M <= 0) return cudaSuccess;
   if (f32)
-    rmsnorm_kernel<float><<<M, 256, 0, st>>>(x, r0, (const float*)embed, vocab, h, 0, d, g, eps,
-                                             (float*)a, err);
-  else
-    rmsnorm_kernel<__nv_bfloat16><<<M, 256, 0, st>>>(x, r0, (const __nv_bfloat16*)embed, vocab,
-                                                     h, 0, d, g, eps, (__nv_bfloat16*)a, err);
-  return cudaGetLastError();
+    return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, x, r0,
+                    (const float*)embed, vocab, h, 0, d, g, eps, (float*)a, err, sp, 0);
+  return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, x, r0,
+                  (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, (__nv_bfloat16*)a, err, sp,
+                  0);
 }
 
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
-                           void* a, int f32, cudaStream_t st) {
+                           void* a, int f32, const StepParams* sp, bool rows_from_lm0,
+                           cudaStream_t st, bool pdl) {
   if (M <= 0) return cudaSuccess;
+  const int* nx = nullptr;
   if (f32)
-    rmsnorm_kernel<float><<<M, 256, 0, st>>>(nullptr, 0, nullptr, 0, const_cast<float*>(h),
-                                             h_row0, d, g, eps, (float*)a, nullptr);
-  else
-    rmsnorm_kernel<__nv_bfloat16><<<M, 256, 0, st>>>(nullptr, 0, nullptr, 0,
-                                                     const_cast<float*>(h), h_row0, d, g, eps,
-                                                     (__nv_bfloat16*)a, nullptr);
-  return cudaGetLastError();
+    return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, nx, 0,
+                    (const float*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, (float*)a,
+                    (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+  return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
+                  (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps,
+                  (__nv_bfloat16*)a, (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
 }
 
 cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,
                                 int mask_id, float tau, int select, float* conf, int* tok,
-                                uint8_t* unmask, DecodeState* state, cudaStream_t st) {
+                                uint8_t* unmask, DecodeState* state, const StepParams* sp,
+                                cudaStream_t st, bool pdl) {
   if (n <= 0 || n > 256) return cudaErrorInvalidValue;
-  merge_select_kernel<<<1, 256, 0, st>>>(reinterpret_cast<const SoftmaxState*>(lm_part), n_part,
-                                         n, x, s, mask_id, tau, select, conf, tok, unmask, state);
-  return cudaGetLastError();
+  return launch_k(pdl, merge_select_kernel, dim3(1), dim3(256), 0, st,
+                  reinterpret_cast<const SoftmaxState*>(lm_part), n_part, n, x, s, mask_id, tau,
+                  select, conf, tok, unmask, state, sp);
 }
 
-cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st) {
+cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st, bool pdl) {
   if (to <= from) return cudaSuccess;
-  fill_kernel<<<(to - from + 255) / 256, 256, 0, st>>>(x, from, to, mask_id);
-  return cudaGetLastError();
+  return launch_k(pdl, fill_kernel, dim3((to - from + 255) / 256), dim3(256), 0, st, x, from, to,
+                  mask_id);
 }
 
 cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
-                                cudaStream_t st) {
+                                cudaStream_t st, bool pdl) {
   if (n <= 0) return cudaSuccess;
-  check_prompt_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, n, vocab, mask_id, err);
-  return cudaGetLastError();
+  return launch_k(pdl, check_prompt_kernel, dim3((n + 255) / 256), dim3(256), 0, st, x, n, vocab,
+                  mask_id, err);
 }
 
 cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int K,
-                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st) {
+                             const GemmShape& gs, const EpiParams& ep, cudaStream_t st, bool pdl) {
   const int grid = gs.n_tiles * ((gs.M + 31) / 32);
-  gemm_simt_kernel<<<grid, 128, 0, st>>>(w, act, act_row0, K, gs, ep);
-  return cudaGetLastError();
+  return launch_k(pdl, gemm_simt_kernel, dim3(grid), dim3(128), 0, st, w, act, act_row0, K, gs,
+                  ep);
 }
 
-cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st) {
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl) {
   if (p.kv_planes != 2) return cudaErrorInvalidValue;
-  dim3 grid(p.M, p.n_heads);
   const size_t smem = (size_t)(p.head_dim + p.L) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  attn_simt_kernel<<<grid, 128, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_k(pdl, attn_simt_kernel, dim3(p.M, p.n_heads), dim3(128), smem, st, p);
 }
 
-cudaError_t launch_attn_combine(const AttnParams& p, int f32, cudaStream_t st) {
-  const int rows = p.M * p.n_heads;
-  if (f32)
-    attn_combine_kernel<float><<<rows, 128, 0, st>>>(p);
-  else
-    attn_combine_kernel<__nv_bfloat16><<<rows, 128, 0, st>>>(p);
-  return cudaGetLastError();
-}
 
 }  // namespace fd

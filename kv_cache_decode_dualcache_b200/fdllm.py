@@ -101,7 +101,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                      i32, P(ctypes.c_float), P(ctypes.c_float),
                                      P(ctypes.c_int32), P(ctypes.c_uint8)]
     lib.fdllm_read_kv.argtypes = [vp, i32, i32, i32, P(ctypes.c_float), P(ctypes.c_float)]
-    lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32]
+    lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32]
     lib.fdllm_attention.argtypes = [vp, vp, vp, i32, i32, i32]
     lib.fdllm_gemm_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
     lib.fdllm_profile_enable.argtypes = [vp, i32]
@@ -252,8 +252,8 @@ def _pair_rows(m: int) -> int:
     return 2 * ((m + 31) // 32) * 32
 
 
-def fdllm_gemm(ctx, w_dev, x_dev, y_dev, splits: int = 0) -> None:
-    """y_dev[M, N] (float32 CUDA tensor) = x @ w_dev[N, K]^T.
+def fdllm_gemm(ctx, w_dev, x_dev, y_dev, splits: int = 0, accumulate: bool = False) -> None:
+    """y_dev[M, N] (float32 CUDA tensor) = x @ w_dev[N, K]^T (+= when accumulate).
 
     M is y_dev's row count.  x_dev is [M, K] float32 (fp32 model) or the
     two-term bf16 pair-row layout with 2*ceil(M/32)*32 rows (bf16 model)."""
@@ -265,7 +265,7 @@ def fdllm_gemm(ctx, w_dev, x_dev, y_dev, splits: int = 0) -> None:
     if x_dev.shape[0] < need or x_dev.shape[1] != K or not x_dev.is_contiguous():
         raise ValueError(f"x_dev must be a contiguous [{need}, {K}] tensor")
     _check(load_library().fdllm_gemm(ctx, w_dev.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(), N,
-                                     M, K, splits), ctx)
+                                     M, K, splits, int(accumulate)), ctx)
 
 
 def fdllm_gemm_noalloc(w_dev, x_dev, y_dev, splits: int = 0, stream=None) -> None:

@@ -46,3 +46,35 @@ def test_attention_matches_oracle(setup, M, L, qscale):
     err = np.abs(got - ref).max()
     tol = 1e-4 * max(1.0, np.abs(ref).max())
     assert err <= tol, (err, tol)
+
+
+@pytest.fixture(scope="module", params=["small-bf16", "small-gqa-bf16"])
+def long_setup(request):
+    require_gpu()
+    shape = synth.SHAPES[request.param]
+    dec = make_decoder(shape, synth.make_weights(shape, device="cpu"), 1024)
+    prompt = synth.make_prompt(shape, 700).numpy()
+    x = np.concatenate([prompt, np.full(60, shape.mask_id)])
+    dec.step_debug(x, x, 700, 32, 0.9, "dual", logits=False)   # caches 760 positions
+    return shape, dec
+
+
+@pytest.mark.parametrize("M,L", [(32, 760), (7, 700), (64, 760), (16, 577)])
+def test_attention_long_keys_split_path(long_setup, M, L):
+    shape, dec = long_setup
+    H, hd = shape.n_heads, shape.head_dim
+    g = torch.Generator(device="cuda").manual_seed(M + L)
+    q = torch.randn(M, H, hd, generator=g, device="cuda") * 4.0
+    qh, ql = split(q)
+    qd = torch.stack([qh, ql]).contiguous()
+    rows = 2 * ((M + 31) // 32) * 32
+    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.bfloat16)
+    for _ in range(2):  # the split counters reset themselves between calls
+        fdllm.fdllm_attention(dec.ctx, qd, o, 1, L)
+        torch.cuda.synchronize()
+        k, v = dec.read_kv(1, 0, L)
+        qx = (qh.double() + ql.double()).cpu().numpy()
+        ref = attention(qx, k.astype(np.float64), v.astype(np.float64)).reshape(M, H * hd)
+        got = from_pair_rows(o, M).double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())

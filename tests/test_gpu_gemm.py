@@ -51,3 +51,16 @@ def test_gemm_split_results_are_deterministic(dec):
         fdllm.fdllm_gemm(dec.ctx, w, x, y, 8)
         outs.append(y.cpu())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_gemm_accumulate_adds_into_y(dec):
+    g = torch.Generator(device="cuda").manual_seed(9)
+    w = (torch.randn(640, 1024, generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    x = torch.randn(48, 1024, generator=g, device="cuda")
+    y0 = torch.randn(48, 640, generator=g, device="cuda")
+    for splits in (1, 4):
+        y = y0.clone()
+        fdllm.fdllm_gemm(dec.ctx, w, pair_rows(x), y, splits, accumulate=True)
+        torch.cuda.synchronize()
+        ref = y0.double().cpu().numpy() + x.double().cpu().numpy() @ w.double().cpu().numpy().T
+        assert np.abs(y.cpu().numpy() - ref).max() <= 2e-5 * np.sqrt(1024) * 0.3 * 5
