@@ -74,9 +74,12 @@ typedef enum {
 
 typedef enum {
   FDLLM_DTYPE_F32 = 0,     /* float32 weights and activations, CUDA cores */
-  FDLLM_DTYPE_BF16 = 1     /* bfloat16 weights on tensor cores; activations, q and the
-                              K/V cache stored as two terms (hi + lo, ~16 significant
-                              bits), float32 accumulation and residual stream */
+  FDLLM_DTYPE_BF16 = 1     /* bfloat16 weights, run on tensor cores: the GEMM weights
+                              are held as fp16 on the device (exact for every bf16
+                              value of magnitude in [2^-17, 65504]); activations, q,
+                              the K/V cache and the softmax weights stored as two fp16
+                              terms (hi + lo, ~22 significant bits); float32
+                              accumulation and residual stream */
 } fdllm_dtype;
 
 /* Model shape and numerics.  Requirements (FDLLM_ERR_ARG otherwise):
@@ -197,7 +200,8 @@ FDLLM_API int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k
 
 /* Kernel-level check of the GEMM the decoder runs (tcgen05 on the bf16
  * model, CUDA cores on the fp32 one): y = x W^T with a plain float output.
- * w_dev [N, K] is a device pointer in the ctx dtype (row-major).  x_dev
+ * w_dev [N, K] is a device pointer in the ctx dtype (row-major); the bf16
+ * model's decoder runs the same tcgen05 kernel on fp16 operands.  x_dev
  * holds the M x K activations as the decoder stores them: fp32 model, plain
  * [M, K] float rows; bf16 model, two-term bf16 rows (x = hi + lo with
  * hi = bf16(x), lo = bf16(x - hi)) grouped by 32 tokens: group j occupies
@@ -215,9 +219,9 @@ FDLLM_API int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, f
  * o = softmax(q K^T / sqrt(head_dim)) V with keys [0, L) of layer `layer`
  * (as left by the last forward), no mask.  fp32 model: q_dev [M, n_heads,
  * head_dim] and o_dev [M, n_heads * head_dim] float.  bf16 model: q_dev is
- * two planes of bf16 [M, n_heads, head_dim] (hi terms, then lo terms) and
- * o_dev receives two-term bf16 rows of n_heads * head_dim in the 32-token
- * grouping described for fdllm_gemm.  The same kernel choice (and key split
+ * two planes of fp16 [M, n_heads, head_dim] (hi terms, then lo terms) and
+ * o_dev receives two-term fp16 rows of n_heads * head_dim in the 32-token
+ * grouping described for fdllm_gemm (the decoder's storage format).  The same kernel choice (and key split
  * for M <= 64) as a decode step.  Errors: ARG, STATE, CUDA. */
 FDLLM_API int fdllm_attention(fdllm_ctx* ctx, const void* q_dev, void* o_dev, int layer, int M,
                               int L);

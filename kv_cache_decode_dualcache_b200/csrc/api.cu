@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
@@ -245,13 +246,16 @@ void dfree_all(fdllm_ctx* ctx) {
   ctx->allocations.clear();
 }
 
+// 2-byte row-major [rows, cols] operand, boxes of box_rows x 64 elements with
+// the 128-byte swizzle.  f16: fp16 (the decoder's storage), else bf16.
 bool make_map(fdllm_ctx* ctx, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool f16 = true) {
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = ctx->encode(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                           2, const_cast<void*>(base), dims,
                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -320,6 +324,7 @@ int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* 
              const EpiParams& ep_in, int* n_part_out = nullptr) {
   const bool lm = ep_in.kind == EPI_LMHEAD;
   GemmShape gs = plan_gemm(ctx, N, M, K, !lm);
+  gs.f16 = ctx->tc ? 1 : 0;  // fp16 weights and two-term fp16 activations
   EpiParams ep = ep_in;
   ep.N = N;
   ep.M = M;
@@ -727,6 +732,14 @@ GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_
   g.splits = best_s;
   g.units = base_units * best_s;
   g.grid = std::min(g.units, num_sms);
+  // K blocks per TMEM accumulation chain.  The tensor core's float32
+  // accumulation rounds toward zero: measured on B200, every K block of 64
+  // added to a running TMEM accumulator biases it by about -5e-8 relative
+  // (-3.8e-6 after K = 4096, -1.2e-5 after K = 12288).  Chains of 8 blocks
+  // keep that near -4e-7, the level of a plain float32 dot product; the
+  // epilogue warps sum the chains with round-to-nearest float32 adds.
+  g.kc = nt == 256 ? 16 : 8;
+  if (const char* kc = std::getenv("FDLLM_KC_EXPERIMENT")) g.kc = std::atoi(kc);
   return g;
 }
 
@@ -973,6 +986,15 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
   ctx->final_norm = (float*)take(sizeof(float) * d);
   CK(copy_to(ctx->embed, "embed", (size_t)V * d * es));
   CK(copy_to(ctx->lm_head, "lm_head", (size_t)V * d * es));
+  // The GEMM weights of the bf16 model are held as fp16 (exact for every
+  // bf16 value of magnitude in [2^-17, 65504]; below 2^-17 the fp16 grid
+  // spacing 2^-24 applies), so that the tensor-core products with the
+  // two-term fp16 activations keep 22 significant bits.  The embedding
+  // table stays bf16 (read directly into the float32 residual stream).
+  auto to_f16 = [&](void* p, size_t n) -> cudaError_t {
+    return ctx->tc ? launch_bf16_to_f16(p, n, ctx->err_dev, nullptr) : cudaSuccess;
+  };
+  CK(to_f16(ctx->lm_head, (size_t)V * d));
   CK(norm_to(ctx->final_norm, "final_norm"));
   ctx->layers.assign(c.n_layers, LayerW());
   for (int l = 0; l < c.n_layers; ++l) {
@@ -998,6 +1020,10 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
                     cudaMemcpyDefault));
     CK(norm_to(lw.attn_norm, p + "attn_norm"));
     CK(norm_to(lw.ffn_norm, p + "ffn_norm"));
+    CK(to_f16(lw.wqkv, (size_t)(hq + 2 * hkv) * d));
+    CK(to_f16(lw.wo, (size_t)d * hq));
+    CK(to_f16(lw.wgu, 2ull * F * d));
+    CK(to_f16(lw.wd, (size_t)d * F));
     if (ctx->tc) {
       if (!make_map(ctx, &lw.m_qkv, lw.wqkv, hq + 2 * hkv, d, 128) ||
           !make_map(ctx, &lw.m_o, lw.wo, d, hq, 128) ||
@@ -1009,6 +1035,16 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
   if (ctx->tc && !make_map(ctx, &ctx->m_head, ctx->lm_head, V, d, 128))
     return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for lm_head");
   CK(cudaDeviceSynchronize());
+  {
+    int e = 0;
+    CK(cudaMemcpy(&e, ctx->err_dev, sizeof(int), cudaMemcpyDeviceToHost));
+    if (e) {
+      const int zero = 0;
+      cudaMemcpy(ctx->err_dev, &zero, sizeof(int), cudaMemcpyHostToDevice);
+      return fail(ctx, FDLLM_ERR_SHAPE,
+                  "a GEMM weight is NaN or outside the fp16 range (|w| > 65504)");
+    }
+  }
   ctx->weights = arena;
   ctx->weights_loaded = true;
   return FDLLM_OK;
@@ -1126,12 +1162,7 @@ int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k_out, floa
       }
       uint16_t raw;
       std::memcpy(&raw, page.data() + e * 2, 2);
-      if (plane < 2) {  // bf16 K terms
-        uint32_t u = (uint32_t)raw << 16;
-        std::memcpy(&val, &u, 4);
-        return val;
-      }
-      __half_raw hr;  // fp16 V terms
+      __half_raw hr;  // fp16 K and V terms
       hr.x = raw;
       return __half2float(__half(hr));
     };
@@ -1186,8 +1217,9 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
                  2.0 * (ctx->tc ? 2 : 1) * M * N * K);
     if (ctx->tc) {
       CUtensorMap wm, xm;
-      if (!make_map(ctx, &wm, w_dev, N, K, 128) ||
-          !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt))
+      gs.f16 = 0;  // bf16 operands (see the header)
+      if (!make_map(ctx, &wm, w_dev, N, K, 128, false) ||
+          !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt, false))
         return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
       GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
                      ctx->n_counters};

@@ -16,13 +16,12 @@
 // idling, and merge their online-softmax states through shared memory at
 // the end.
 //
-// Every operand is two-term (hi + lo): q and K as bf16 pairs, V as fp16
-// pairs, and the softmax weights P are split the same way into fp16 pairs.
-// Each product takes the three significant cross terms:
-//   S  = q_hi K_hi + q_hi K_lo + q_lo K_hi        (bf16 MMAs, f32 accumulate)
-//   PV = P_hi V_hi + P_hi V_lo + P_lo V_hi        (fp16 MMAs, f32 accumulate)
-// so the attention output carries ~16 significant bits like every other
-// stored activation of the bf16 model (see split_bf16).  Online softmax in
+// Every operand is two-term (hi + lo fp16 pairs): q, K, V and the softmax
+// weights P.  Each product takes the three significant cross terms:
+//   S  = q_hi K_hi + q_hi K_lo + q_lo K_hi        (fp16 MMAs, f32 accumulate)
+//   PV = P_hi V_hi + P_hi V_lo + P_lo V_hi
+// so the attention output carries ~22 significant bits like every other
+// stored activation of the bf16 model (see split_f16).  Online softmax in
 // f32, exp2 domain.
 //
 // With n_split > 1 (long sequences) each split writes unnormalised partial
@@ -58,13 +57,6 @@ FD_DEV void ldsm_x4_t(uint32_t addr, uint32_t* r) {
                : "r"(addr));
 }
 
-FD_DEV void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 FD_DEV void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -101,7 +93,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   const int key_hi = min(p.L, key_lo + p.keys_per_split);
   const int n_kt = (key_hi - key_lo + 63) / 64;
 
-  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q);
+  const __half* qg = reinterpret_cast<const __half*>(p.q);
   const uint16_t* pool = reinterpret_cast<const uint16_t*>(p.kv_pool);
   pdl_trigger();
   pdl_wait();
@@ -112,7 +104,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     const int r = row0 + i;
     const bool ok = r < rows_total;
     const int m = ok ? r / rep : 0, jj = ok ? r % rep : 0;
-    const __nv_bfloat16* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
+    const __half* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
     cp_async16(q_s + swz<HD>(i, ch), src, ok ? 16 : 0);
     cp_async16(q_s + TILE + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
   }
@@ -165,12 +157,12 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
           const uint32_t ka = swz<HD>(key, 2 * kk + ((lane >> 3) & 1));
           ldsm_x4(kv_s(buf, 0) + ka, kh);
           ldsm_x4(kv_s(buf, 1) + ka, kl);
-          mma_bf16(s[2 * np], qh, kh[0], kh[1]);
-          mma_bf16(s[2 * np + 1], qh, kh[2], kh[3]);
-          mma_bf16(s[2 * np], qh, kl[0], kl[1]);
-          mma_bf16(s[2 * np + 1], qh, kl[2], kl[3]);
-          mma_bf16(s[2 * np], ql, kh[0], kh[1]);
-          mma_bf16(s[2 * np + 1], ql, kh[2], kh[3]);
+          mma_f16(s[2 * np], qh, kh[0], kh[1]);
+          mma_f16(s[2 * np + 1], qh, kh[2], kh[3]);
+          mma_f16(s[2 * np], qh, kl[0], kl[1]);
+          mma_f16(s[2 * np + 1], qh, kl[2], kl[3]);
+          mma_f16(s[2 * np], ql, kh[0], kh[1]);
+          mma_f16(s[2 * np + 1], ql, kh[2], kh[3]);
         }
       }
       // ---- online softmax (rows lane/4 and lane/4 + 8)
@@ -300,17 +292,17 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     const size_t orow = (size_t)m * H + head;
     if (p.n_split == 1) {
       const float inv = 1.0f / lrow[r];
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
+      __half* o = reinterpret_cast<__half*>(p.o);
       const size_t hi_off = (size_t)pair_row(m) * hq + (size_t)head * HD;
       const size_t lo_off = hi_off + (size_t)PAIR_LO * hq;
 #pragma unroll
       for (int j = 0; j < HD / 8; ++j) {
         const int d = j * 8 + 2 * (lane & 3);
-        __nv_bfloat16 h0, l0, h1, l1;
-        split_bf16(oacc[j][2 * r] * inv, h0, l0);
-        split_bf16(oacc[j][2 * r + 1] * inv, h1, l1);
-        *reinterpret_cast<__nv_bfloat162*>(o + hi_off + d) = __halves2bfloat162(h0, h1);
-        *reinterpret_cast<__nv_bfloat162*>(o + lo_off + d) = __halves2bfloat162(l0, l1);
+        __half h0, l0, h1, l1;
+        split_f16(oacc[j][2 * r] * inv, h0, l0);
+        split_f16(oacc[j][2 * r + 1] * inv, h1, l1);
+        *reinterpret_cast<__half2*>(o + hi_off + d) = __halves2half2(h0, h1);
+        *reinterpret_cast<__half2*>(o + lo_off + d) = __halves2half2(l0, l1);
       }
     } else {
       float* po = p.part_o + ((size_t)blockIdx.z * rows_all + orow) * HD;
@@ -364,7 +356,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     s_inv[tid] = 1.0f / den;
   }
   __syncthreads();
-  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.o);
+  __half* o = reinterpret_cast<__half*>(p.o);
   // 8 outputs per thread per pass, every partial load issued before any store
   for (int base = 0; base < n_rows * HD; base += 128 * 8) {
     float acc[8];
@@ -389,8 +381,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
         const int i = idx / HD, d = idx % HD;
         const int rr = row0 + i;
         const int m = rr / rep, head = g * rep + rr % rep;
-        __nv_bfloat16 hi, lo;
-        split_bf16(acc[e] * s_inv[i], hi, lo);
+        __half hi, lo;
+        split_f16(acc[e] * s_inv[i], hi, lo);
         const size_t off = (size_t)pair_row(m) * hq + (size_t)head * HD + d;
         o[off] = hi;
         o[off + (size_t)PAIR_LO * hq] = lo;

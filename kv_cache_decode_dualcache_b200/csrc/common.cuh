@@ -19,6 +19,7 @@ enum : int {
   DEV_ERR_TIMEOUT = 1,   // a bounded wait gave up
   DEV_ERR_TOKEN = 2,     // a token id outside [0, vocab) or a mask id in the prompt
   DEV_ERR_SHAPE = 4,     // a kernel was launched with a shape it cannot handle
+  DEV_ERR_RANGE = 8,     // a weight outside the fp16 range
 };
 
 constexpr int KV_PAGE = 64;             // positions per KV-cache page
@@ -36,12 +37,15 @@ template <> FD_DEV __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float
 template <> FD_DEV __half from_f<__half>(float v) { return __float2half_rn(v); }
 
 // Two-term storage of the bf16 model's activations and K/V: x = hi + lo with
-// hi = round(x) and lo = round(x - hi) in the storage type (bf16: 16
-// significant bits together; fp16: 22).  A single bf16 term (8 bits) put a
-// rounding flip of ~1/256 relative into the logits for every stored element
-// whose float32 and float64 values straddle a rounding boundary; on this
-// workload (logits x30) one such flip in the final hidden state alone moves
-// a logit by ~0.03.
+// hi = round(x) and lo = round(x - hi) in the storage type.  The decoder
+// stores fp16 pairs (22 significant bits together; the GEMM weights are
+// converted to fp16 at load, exactly for every bf16 weight of magnitude
+// >= 2^-17).  A single 16-bit term puts a rounding flip of 2^-9 (bf16) or
+// 2^-12 (fp16) relative into every stored element whose float32 and float64
+// values straddle a rounding boundary, and 32 layers of a random-weight
+// network amplify those flips into logit errors far above 3e-2; bf16 pairs
+// (16 bits) still left confidence errors of ~1.3e-3 at the LLaDA-8B shape.
+// split_bf16 serves the bf16 operands of the stand-alone GEMM entry points.
 FD_DEV void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
@@ -255,17 +259,17 @@ FD_DEV uint64_t smem_desc_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: D f32, A and B bf16, both K-major,
-// M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
-  return (1u << 4)                      // D format f32
-         | (1u << 7)                    // A format bf16
-         | (1u << 10)                   // B format bf16
-         | ((uint32_t)(n >> 3) << 17)   // N >> 3
-         | ((uint32_t)(128 >> 4) << 24);  // M >> 4
+// Instruction descriptor, kind::f16: D f32, A and B both fp16 (f16 = true)
+// or both bf16, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int n, bool f16) {
+  return (1u << 4)                          // D format f32
+         | ((f16 ? 0u : 1u) << 7)           // A format: 0 fp16, 1 bf16
+         | ((f16 ? 0u : 1u) << 10)          // B format: the same as A
+         | ((uint32_t)(n >> 3) << 17)       // N >> 3
+         | ((uint32_t)(128 >> 4) << 24);    // M >> 4
 }
 
-FD_DEV void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+FD_DEV void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                         uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -303,6 +307,56 @@ FD_DEV void tmem_ld32(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Load 64 consecutive TMEM columns of this warp's 32 lanes into v[0..63]
+// (one instruction, one wait).
+FD_DEV void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+        "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+        "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+        "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Store v[0..31] into 32 consecutive TMEM columns of this warp's 32 lanes
+// and wait for the store to complete.
+FD_DEV void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Named barrier among `count` threads (a multiple of 32).

@@ -7,7 +7,7 @@
 // call epi_chunk with e = their feature index.  Control flow is uniform
 // within each warp (the LM-head reduction uses warp shuffles).
 //
-// Stores of the bf16 model are two-term (hi + lo, see split_bf16): the q
+// Stores of the bf16 model are two-term fp16 (hi + lo, see split_f16): the q
 // planes, the K/V cache planes and the SwiGLU output in pair rows.
 #pragma once
 
@@ -81,9 +81,9 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
             if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f))
               reinterpret_cast<float*>(ep.f_out)[i] = y;
           } else {
-            __nv_bfloat16 hi, lo;
-            split_bf16(y, hi, lo);
-            __nv_bfloat16* f = reinterpret_cast<__nv_bfloat16*>(ep.f_out);
+            __half hi, lo;
+            split_f16(y, hi, lo);
+            __half* f = reinterpret_cast<__half*>(ep.f_out);
             const size_t r = (size_t)pair_row(tok);
             const size_t i = (r + PAIR_LO) * F + j;
             if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f)) {
@@ -147,18 +147,18 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
             if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
           }
         } else if (is_q) {
-          __nv_bfloat16 hi, lo;
-          split_bf16(y, hi, lo);
-          __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(ep.q_out);
+          __half hi, lo;
+          split_f16(y, hi, lo);
+          __half* q = reinterpret_cast<__half*>(ep.q_out);
           const size_t i = (size_t)tok * hq + n;
           if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
             q[i] = hi;
             q[ep.q_plane + i] = lo;
           }
         } else if (!is_v) {
-          __nv_bfloat16 hi, lo;
-          split_bf16(y, hi, lo);
-          __nv_bfloat16* k = reinterpret_cast<__nv_bfloat16*>(ep.kv_pool);
+          __half hi, lo;
+          split_f16(y, hi, lo);
+          __half* k = reinterpret_cast<__half*>(ep.kv_pool);
           const int head = (n - hq) / hd;
           const size_t i0 = kv_offset_pg(ep, page, pos, 0, head, dh);
           const size_t i1 = kv_offset_pg(ep, page, pos, 1, head, dh);

@@ -1,4 +1,5 @@
-// Persistent tcgen05 GEMM for the bfloat16 model: Y[t, n] = sum_k X[t, k] W[n, k].
+// Persistent tcgen05 GEMM: Y[t, n] = sum_k X[t, k] W[n, k], W and X both fp16
+// (the decoder's storage) or both bf16 (the stand-alone GEMM entry points).
 //
 // The weight matrix is the 128-row A operand (the "swap-AB" arrangement: the
 // model's output features fill the MMA's M = 128; the few block tokens are
@@ -36,6 +37,7 @@ namespace {
 constexpr int BK = 64;                    // K elements per stage (128 bytes of bf16)
 constexpr int A_STAGE_BYTES = 128 * BK * 2;
 constexpr int LM_MAX_ROWS = 256;          // largest M for the LM-head epilogue
+
 
 template <int NT> struct TcCfg;
 template <> struct TcCfg<64> { static constexpr int STAGES = 8; };
@@ -82,9 +84,11 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int TOK = NT / 2;  // tokens per token tile
   using Lay = TcLayout<NT>;
   constexpr int STAGES = Lay::STAGES;
-  constexpr uint32_t IDESC = idesc_bf16_f32(NT);
+  // operand type: fp16 (the decoder's weights and two-term activations) or bf16
+  const uint32_t idesc = gs.f16 ? idesc_f32acc(NT, true) : idesc_f32acc(NT, false);
   constexpr uint32_t TMEM_COLS = 2 * NT;
   constexpr uint32_t STAGE_TX = A_STAGE_BYTES + Lay::B_STAGE_BYTES;
+  const int KC = gs.kc;  // K blocks per TMEM accumulation chain (see plan_gemm_tc)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -186,28 +190,37 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      uint32_t it = 0, local = 0;
+      // Each unit's K range is accumulated in TMEM in chains of at most KC
+      // K blocks (one accumulator buffer per chain, alternating); the
+      // epilogue warps add the chains up in float32 registers.
+      uint32_t it = 0, chain = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x, ++local) {
+      for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x) {
         const UnitCoord c = decode_unit(gs, u);
-        const uint32_t buf = local & 1u;
-        if (!mbar_wait(&acc_empty[buf], ((local >> 1) & 1u) ^ 1u, sc.err, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d = tmem + buf * NT;
-        for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1u, sc.err, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(a_st + s * A_STAGE_BYTES);
-          const uint32_t b0 = smem_u32(b_st + s * Lay::B_STAGE_BYTES);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            tc_mma_bf16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), IDESC,
-                        (kb > c.kb_lo || k > 0) ? 1u : 0u);
+        for (int k0 = c.kb_lo; k0 < c.kb_hi && ok; k0 += KC, ++chain) {
+          const uint32_t buf = chain & 1u;
+          if (!mbar_wait(&acc_empty[buf], ((chain >> 1) & 1u) ^ 1u, sc.err, abort_flag)) {
+            ok = false;
+            break;
           }
-          tc_commit(&empty[s]);
+          tc_fence_after();
+          const uint32_t d = tmem + buf * NT;
+          const int k1 = min(k0 + KC, c.kb_hi);
+          for (int kb = k0; kb < k1; ++kb, ++it) {
+            const int s = it % STAGES;
+            if (!mbar_wait(&full[s], (it / STAGES) & 1u, sc.err, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(a_st + s * A_STAGE_BYTES);
+            const uint32_t b0 = smem_u32(b_st + s * Lay::B_STAGE_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              tc_mma(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
+                     (kb > k0 || k > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[s]);
+          }
+          tc_commit(&acc_full[buf]);
         }
-        tc_commit(&acc_full[buf]);
       }
     }
   } else {
@@ -215,24 +228,46 @@ __global__ void __launch_bounds__(192, 1)
     const int quad = warp & 3;
     const int e = quad * 32 + lane;  // feature row = TMEM lane
     pdl_wait();                      // reads / writes of the previous kernel's data follow
-    uint32_t local = 0;
-    for (int u = blockIdx.x; u < gs.units; u += gridDim.x, ++local) {
+    uint32_t chain = 0;
+    for (int u = blockIdx.x; u < gs.units; u += gridDim.x) {
       const UnitCoord c = decode_unit(gs, u);
-      const uint32_t buf = local & 1u;
-      const bool got = mbar_wait(&acc_full[buf], (local >> 1) & 1u, sc.err, abort_flag);
-      tc_fence_after();
+      // acc[t] = this lane's feature for token t of the tile: the sum over the
+      // unit's accumulation chains of the hi- and lo-term columns (columns
+      // [64g, 64g+32) of a chain buffer hold the hi term of tokens 32g..,
+      // the next 32 their lo term).  The sums are written back into the
+      // first TOK columns of the last chain's buffer, which the epilogue
+      // keeps until the unit is done, and read back 32 tokens at a time.
+      float acc[TOK];
+#pragma unroll
+      for (int t = 0; t < TOK; ++t) acc[t] = 0.0f;
+      bool got = true;
+      uint32_t col = 0, last_buf = 0;
+      for (int k0 = c.kb_lo; k0 < c.kb_hi; k0 += KC, ++chain) {
+        const uint32_t buf = chain & 1u;
+        got = mbar_wait(&acc_full[buf], (chain >> 1) & 1u, sc.err, abort_flag) && got;
+        tc_fence_after();
+        col = tmem + ((uint32_t)(quad * 32) << 16) + buf * NT;
+#pragma unroll
+        for (int g = 0; g < TOK / 32; ++g) {
+          float v[64];
+          tmem_ld64(col + g * 64, v);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) acc[g * 32 + t] += v[t] + v[t + 32];
+        }
+        last_buf = buf;
+        if (k0 + KC < c.kb_hi) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < TOK / 32; ++g) tmem_st32(col + g * 32, acc + g * 32);
       const int n0 = c.tile * 128;
       const int tile_id = c.tile * gs.n_tt + c.tt;
       float* ws_unit = sc.ws + ((size_t)tile_id * gs.splits + c.split) * (TOK * 128);
       for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
-        // columns [64ch, 64ch+32) hold the hi term, [64ch+32, 64ch+64) the lo term
-        float v[32], vl[32];
-        FD_CHECK(buf * NT + ch * 64 + 64 <= TMEM_COLS, ep.check, 21, buf * NT + ch * 64, TMEM_COLS);
-        const uint32_t col = tmem + ((uint32_t)(quad * 32) << 16) + buf * NT + ch * 64;
-        tmem_ld32(col, v);
-        tmem_ld32(col + 32, vl);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] += vl[t];
+        float v[32];
+        tmem_ld32(col + ch * 32, v);
         if (gs.splits == 1) {
           named_bar(1, EPI_THREADS);  // previous chunk's epilogue is done with `tile`
 #pragma unroll
@@ -248,7 +283,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
+      mbar_arrive(&acc_empty[last_buf]);
       if (gs.splits > 1) {
         __threadfence();
         named_bar(1, EPI_THREADS);
@@ -263,19 +298,19 @@ __global__ void __launch_bounds__(192, 1)
           __threadfence();
           const float* ws_tile = sc.ws + (size_t)tile_id * gs.splits * (TOK * 128);
           for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
-            float acc[32];
+            float racc[32];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) acc[t] = 0.0f;
+            for (int t = 0; t < 32; ++t) racc[t] = 0.0f;
             for (int sp = 0; sp < gs.splits; ++sp) {
               const float* p = ws_tile + (size_t)sp * (TOK * 128) + ch * CHUNK_T * 128 + e;
               const size_t wi = (size_t)(p - sc.ws) + 31 * 128;
               if (!FD_CHECK(wi < sc.ws_elems, ep.check, 24, wi, sc.ws_elems)) continue;
 #pragma unroll
-              for (int t = 0; t < 32; ++t) acc[t] += __ldcg(p + t * 128);
+              for (int t = 0; t < 32; ++t) racc[t] += __ldcg(p + t * 128);
             }
             named_bar(1, EPI_THREADS);
 #pragma unroll
-            for (int t = 0; t < 32; ++t) tile[t * 128 + e] = acc[t];
+            for (int t = 0; t < 32; ++t) tile[t * 128 + e] = racc[t];
             named_bar(1, EPI_THREADS);
             if (got) epi_chunk<false>(ep, tile, n0, c.tt * TOK + ch * CHUNK_T, e, lm);
           }

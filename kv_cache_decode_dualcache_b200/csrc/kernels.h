@@ -34,15 +34,15 @@ struct EpiParams {
   int kind;
   int N;             // output features (rows of the weight matrix)
   int M;             // valid token rows
-  int act_f32;       // 1: activations / outputs are float (fp32 model); 0: bf16
+  int act_f32;       // 1: activations / outputs are float (fp32 model); 0: two-term fp16
   // EPI_STORE
   float* out;
   int ld_out;
   // EPI_QKV
-  void* q_out;       // fp32: [M, H*hd]; bf16: hi plane then lo plane, each [rows, H*hd]
-  size_t q_plane;    // elements per q plane (bf16)
+  void* q_out;       // fp32: [M, H*hd]; bf16 model: fp16 hi plane then lo plane, each [rows, H*hd]
+  size_t q_plane;    // elements per q plane (bf16 model)
   void* kv_pool;     // [layers][pages][planes][Hkv][KV_PAGE][hd]; planes: fp32 K,V;
-                     // bf16 K hi, K lo (bf16), V hi, V lo (fp16)
+                     // bf16 model: K hi, K lo, V hi, V lo (all fp16)
   int kv_planes;
   const int* page_table;
   int n_pages;
@@ -53,7 +53,7 @@ struct EpiParams {
   // EPI_RESID
   float* h;          // [M, N]
   // EPI_SWIGLU
-  void* f_out;       // [M, N/2] (fp32) or two-term pair rows (bf16)
+  void* f_out;       // [M, N/2] (fp32) or two-term fp16 pair rows (bf16 model)
   // EPI_LMHEAD
   float logit_scale;
   int mask_id;
@@ -77,6 +77,8 @@ struct GemmShape {
   int kb_total;      // ceil(K / 64)
   int units;         // n_tiles * n_tt * splits
   int grid;          // CTAs launched
+  int f16;           // tcgen05 operands: 1 = fp16 (the decoder), 0 = bf16
+  int kc;            // K blocks per TMEM accumulation chain (tcgen05 GEMM)
 };
 
 struct GemmScratch {
@@ -115,7 +117,8 @@ cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, si
 cudaError_t init_kernel_attributes();
 
 // Launchers (return cudaError_t of the launch).
-// bf16 model: activations in two-term pair rows, token tiles of nt/2 tokens.
+// bf16 model: activations in two-term pair rows, token tiles of nt/2 tokens;
+// operand type fp16 or bf16 by gs.f16.
 cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
                            const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
                            cudaStream_t st, bool pdl = false);
@@ -126,9 +129,9 @@ cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int
 int gemm_tc_smem_bytes(int nt);
 
 struct AttnParams {
-  const void* q;       // [M, H, hd] (fp32) or hi/lo planes of [M, H, hd] (bf16)
-  size_t q_plane;      // elements per q plane (bf16)
-  void* o;             // [M, H*hd] (fp32) or two-term pair rows (bf16)
+  const void* q;       // [M, H, hd] (fp32) or fp16 hi/lo planes of [M, H, hd] (bf16 model)
+  size_t q_plane;      // elements per q plane (bf16 model)
+  void* o;             // [M, H*hd] (fp32) or two-term fp16 pair rows (bf16 model)
   const void* kv_pool;
   int kv_planes;
   const int* page_table;
@@ -149,12 +152,13 @@ int attn_rows_per_cta(int M, int n_heads, int n_kv_heads);
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl = false);
 
 // h[i] = embed[x[r0+i]]; a[i] = RMSNorm(h[i]) * g, i in [0, M).  With sp,
-// r0 = sp->r0.
+// r0 = sp->r0.  bf16 model: bf16 embedding rows, a in two-term fp16 pair rows.
 cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
                                  int vocab, const float* g, float eps, float* h, void* a,
                                  int f32, int* err, const StepParams* sp, cudaStream_t st,
                                  bool pdl = false);
-// a[i] = RMSNorm(h[h_row0 + i]) * g, i in [0, M).  bf16: two-term pair rows.
+// a[i] = RMSNorm(h[h_row0 + i]) * g, i in [0, M).  bf16 model: two-term fp16
+// pair rows.
 // With sp and rows_from_lm0, h_row0 = sp->lm0.
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
                            void* a, int f32, const StepParams* sp, bool rows_from_lm0,
@@ -179,5 +183,8 @@ cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream
                                bool pdl = false);
 cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
                                 cudaStream_t st, bool pdl = false);
+// In place: n bf16 values -> fp16 (round to nearest even).  A value outside
+// the fp16 range sets DEV_ERR_RANGE in *err.
+cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, cudaStream_t st);
 
 }  // namespace fd

@@ -1,6 +1,7 @@
 // CUDA-core kernels: embedding + RMSNorm, RMSNorm, the LM-head partial
 // merge fused with the threshold/unmask/scatter step, and the float32 GEMM
 // and attention of the fp32 model.
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -39,14 +40,14 @@ FD_DEV float block_max(float v, float* red) {
 // ------------------------------------------------------------------ RMSNorm
 // a[row] = h[h_row0 + row] / sqrt(mean(h^2) + eps) * g; one CTA per row.  With
 // `x` given, h[row] is first gathered from the embedding table at token
-// x[r0 + row].  fp32 model: a is [M, d] float; bf16 model: a is two-term in
-// pair rows.
+// x[r0 + row].  fp32 model: a is [M, d] float; bf16 model (bf16 embedding
+// rows): a is two-term fp16 in pair rows.
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x, int r0,
                                                       const T* __restrict__ embed, int vocab,
                                                       float* __restrict__ h, int h_row0, int d,
                                                       const float* __restrict__ g, float eps,
-                                                      T* __restrict__ a, int* err,
+                                                      void* __restrict__ a, int* err,
                                                       const StepParams* sp, int rows_from_lm0) {
   // The row stays in registers (d <= 256 * RMS_VPT): every load is issued
   // before any store.
@@ -94,17 +95,17 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x,
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int j = threadIdx.x + k * 256;
-      if (j < d) a[(size_t)row * d + j] = from_f<T>(v[k] * inv * __ldg(&g[j]));
+      if (j < d) reinterpret_cast<float*>(a)[(size_t)row * d + j] = v[k] * inv * __ldg(&g[j]);
     }
   } else {
-    __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(a);
+    __half* ab = reinterpret_cast<__half*>(a);
     const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int j = threadIdx.x + k * 256;
       if (j < d) {
-        __nv_bfloat16 hi, lo;
-        split_bf16(v[k] * inv * __ldg(&g[j]), hi, lo);
+        __half hi, lo;
+        split_f16(v[k] * inv * __ldg(&g[j]), hi, lo);
         ab[r_hi + j] = hi;
         ab[r_lo + j] = lo;
       }
@@ -169,6 +170,15 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
     state->remaining = n_left;
     state->unmasked = n_un;
     state->steps += 1;
+  }
+}
+
+__global__ void bf16_to_f16_kernel(uint16_t* p, size_t n, int* err) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = __uint_as_float((uint32_t)p[i] << 16);
+    if (!(fabsf(v) <= 65504.0f)) atomicOr(err, DEV_ERR_RANGE);  // also NaN
+    p[i] = __half_as_ushort(__float2half_rn(v));
   }
 }
 
@@ -303,10 +313,9 @@ cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed,
   if (M <= 0) return cudaSuccess;
   if (f32)
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, x, r0,
-                    (const float*)embed, vocab, h, 0, d, g, eps, (float*)a, err, sp, 0);
+                    (const float*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, x, r0,
-                  (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, (__nv_bfloat16*)a, err, sp,
-                  0);
+                  (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
 }
 
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
@@ -316,11 +325,11 @@ cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float
   const int* nx = nullptr;
   if (f32)
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, nx, 0,
-                    (const float*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, (float*)a,
+                    (const float*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
                     (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
-                  (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps,
-                  (__nv_bfloat16*)a, (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+                  (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
+                  (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
 }
 
 cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,
@@ -331,6 +340,13 @@ cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x,
   return launch_k(pdl, merge_select_kernel, dim3(1), dim3(256), 0, st,
                   reinterpret_cast<const SoftmaxState*>(lm_part), n_part, n, x, s, mask_id, tau,
                   select, conf, tok, unmask, state, sp);
+}
+
+cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const size_t blocks = std::min<size_t>((n + 255) / 256, 4096);
+  bf16_to_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint16_t*>(p), n, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st, bool pdl) {

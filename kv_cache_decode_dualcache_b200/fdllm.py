@@ -289,8 +289,8 @@ def fdllm_attention(ctx, q_dev, o_dev, layer: int, L: int) -> None:
     """Attention of M queries over cached keys [0, L) of ``layer``.
 
     fp32 model: q_dev [M, H, hd], o_dev [M, H*hd] float32.  bf16 model:
-    q_dev [2, M, H, hd] (hi plane, lo plane), o_dev two-term pair rows
-    [2*ceil(M/32)*32, H*hd] bf16."""
+    q_dev [2, M, H, hd] fp16 (hi plane, lo plane), o_dev two-term fp16 pair
+    rows [2*ceil(M/32)*32, H*hd]."""
     two_term = q_dev.dim() == 4
     M = int(q_dev.shape[1] if two_term else q_dev.shape[0])
     need = _pair_rows(M) if two_term else M

@@ -1,11 +1,12 @@
-"""Builders for the two-term (hi + lo) bf16 layouts the bf16 decoder uses,
-written with plain torch ops for the GPU kernel tests."""
+"""Builders for the two-term (hi + lo) layouts of the bf16 model, written
+with plain torch ops for the GPU kernel tests: bf16 pairs for the stand-alone
+GEMM entry points, fp16 pairs for the decoder's own storage."""
 import torch
 
 
-def split(x: torch.Tensor):
-    hi = x.to(torch.bfloat16)
-    lo = (x - hi.float()).to(torch.bfloat16)
+def split(x: torch.Tensor, dtype=torch.bfloat16):
+    hi = x.to(dtype)
+    lo = (x - hi.float()).to(dtype)
     return hi, lo
 
 

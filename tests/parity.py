@@ -1,8 +1,8 @@
 """Shared helpers for the GPU parity tests (teacher-forced per-step compare).
 
 The acceptance rule: per step, logits max-abs within ``z_tol`` (1e-4 for the
-float32 model, 3e-2 for bfloat16 against the oracle's bf16 storage
-emulation), confidences within 1e-3, and token ids / unmask sets identical
+float32 model, 3e-2 for the bf16 model, both against the exact float64
+oracle), confidences within 1e-3, and token ids / unmask sets identical
 except at positions where the oracle's top-2 logit margin or |conf - tau| is
 below 1e-3; those positions are counted and returned.
 """

@@ -32,10 +32,10 @@ def test_attention_matches_oracle(setup, M, L, qscale):
     H, hd = shape.n_heads, shape.head_dim
     g = torch.Generator(device="cuda").manual_seed(M * 1000 + L)
     q = torch.randn(M, H, hd, generator=g, device="cuda") * qscale
-    qh, ql = split(q)
+    qh, ql = split(q, torch.float16)
     qd = torch.stack([qh, ql]).contiguous()
     rows = 2 * ((M + 31) // 32) * 32
-    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.bfloat16)
+    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.float16)
     fdllm.fdllm_attention(dec.ctx, qd, o, 0, L)
     torch.cuda.synchronize()
     k, v = dec.read_kv(0, 0, L)
@@ -65,10 +65,10 @@ def test_attention_long_keys_split_path(long_setup, M, L):
     H, hd = shape.n_heads, shape.head_dim
     g = torch.Generator(device="cuda").manual_seed(M + L)
     q = torch.randn(M, H, hd, generator=g, device="cuda") * 4.0
-    qh, ql = split(q)
+    qh, ql = split(q, torch.float16)
     qd = torch.stack([qh, ql]).contiguous()
     rows = 2 * ((M + 31) // 32) * 32
-    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.bfloat16)
+    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.float16)
     for _ in range(2):  # the split counters reset themselves between calls
         fdllm.fdllm_attention(dec.ctx, qd, o, 1, L)
         torch.cuda.synchronize()
