@@ -35,7 +35,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 const int kNtChoices[3] = {64, 128, 256};   // token-tile rows (two-term: rows/2 tokens)
 constexpr size_t kWorkspaceBytes = 64ull << 20;
 constexpr int kMaxLmRows = 256;
-constexpr int kMaxAttnSplit = 16;
+constexpr int kMaxAttnSplit = 8;   // key splits = CTAs of one thread-block cluster
 constexpr int kAttnSplitMaxM = 64;
 constexpr int kSpRing = 8;
 
@@ -100,9 +100,6 @@ struct fdllm_ctx {
   float* ws = nullptr;
   int* counters = nullptr;
   int n_counters = 0;
-  float* attn_po = nullptr;
-  float* attn_ml = nullptr;
-  int* attn_cnt = nullptr;      // split-merge counters of the attention kernel
   float* lm_part = nullptr;
   size_t lm_part_cap = 0;   // SoftmaxState entries
   float* conf = nullptr;
@@ -279,6 +276,8 @@ int check_config(const fdllm_config* c, std::string* why) {
   if (!(c->dtype == FDLLM_DTYPE_F32 || c->dtype == FDLLM_DTYPE_BF16)) return bad("unknown dtype");
   if (c->dtype == FDLLM_DTYPE_BF16 && c->head_dim == 32)
     return bad("the bf16 attention kernel needs head_dim 64 or 128");
+  if (c->dtype == FDLLM_DTYPE_BF16 && (c->n_kv_heads * c->head_dim) % 64)
+    return bad("n_kv_heads * head_dim must be a multiple of 64");
   if (c->max_batch != 1) return bad("max_batch must be 1");
   if (c->max_seq < 1 || c->max_seq > (1 << 20)) return bad("max_seq out of range");
   if (!(c->rms_eps >= 0.0f) || !std::isfinite(c->rope_theta) || !(c->rope_theta > 0.0f) ||
@@ -292,8 +291,8 @@ int check_config(const fdllm_config* c, std::string* why) {
 // token tile of nt rows (nt/2 tokens, two-term), the K split chosen to
 // balance the per-CTA K blocks over the persistent grid (deterministic
 // reduction of the splits).  Plans are memoised per shape.
-GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split) {
-  if (ctx->tc) return plan_gemm_tc(ctx->num_sms, N, M, K, allow_split, kWorkspaceBytes);
+GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split, bool lm) {
+  if (ctx->tc) return plan_gemm_tc(ctx->num_sms, N, M, K, allow_split, kWorkspaceBytes, lm ? 128 : 256);
   GemmShape g{};
   g.N = N;
   g.M = M;
@@ -308,11 +307,11 @@ GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split)
   return g;
 }
 
-GemmShape plan_gemm(fdllm_ctx* ctx, int N, int M, int K, bool allow_split) {
-  const auto key = std::make_tuple(N, M, K, allow_split ? 1 : 0);
+GemmShape plan_gemm(fdllm_ctx* ctx, int N, int M, int K, bool allow_split, bool lm = false) {
+  const auto key = std::make_tuple(N, M, K, (allow_split ? 1 : 0) + (lm ? 2 : 0));
   auto it = ctx->plans.find(key);
   if (it != ctx->plans.end()) return it->second;
-  GemmShape g = make_plan(ctx, N, M, K, allow_split);
+  GemmShape g = make_plan(ctx, N, M, K, allow_split, lm);
   ctx->plans[key] = g;
   return g;
 }
@@ -323,7 +322,7 @@ int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* 
              const void* act, CUtensorMap* amaps, int act_row0, int N, int M, int K,
              const EpiParams& ep_in, int* n_part_out = nullptr) {
   const bool lm = ep_in.kind == EPI_LMHEAD;
-  GemmShape gs = plan_gemm(ctx, N, M, K, !lm);
+  GemmShape gs = plan_gemm(ctx, N, M, K, !lm, lm);
   gs.f16 = ctx->tc ? 1 : 0;  // fp16 weights and two-term fp16 activations
   EpiParams ep = ep_in;
   ep.N = N;
@@ -398,9 +397,6 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   ap.n_heads = c.n_heads;
   ap.n_kv_heads = c.n_kv_heads;
   ap.head_dim = c.head_dim;
-  ap.part_o = ctx->attn_po;
-  ap.part_ml = ctx->attn_ml;
-  ap.counters = ctx->attn_cnt;
   ap.n_split = 1;
   ap.keys_per_split = ((L + 63) / 64) * 64;
   const double es = (double)ctx->esz;
@@ -413,16 +409,15 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
     KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
     return FDLLM_OK;
   }
-  // Key splits only when one CTA would stream many key tiles (long
-  // sequences, few query rows): enough CTAs to cover the SMs twice, at least
-  // 4 key tiles per split.
+  // Few query rows (block steps): split the keys so that the (row tile, KV
+  // head, split) CTAs fill the SMs once, at least 2 key tiles per split.
   const int rep = c.n_heads / c.n_kv_heads;
   const int rows_per_cta = attn_rows_per_cta(M, c.n_heads, c.n_kv_heads);
   const int ctas = ((M * rep + rows_per_cta - 1) / rows_per_cta) * c.n_kv_heads;
   const int key_tiles = (L + 63) / 64;
-  if (M <= kAttnSplitMaxM && key_tiles > 8) {
-    int want = std::max(1, (2 * ctx->num_sms) / std::max(1, ctas));
-    want = std::min(want, std::min(kMaxAttnSplit, key_tiles / 4));
+  if (M <= kAttnSplitMaxM && key_tiles >= 4) {
+    int want = std::max(1, ctx->num_sms / std::max(1, ctas));
+    want = std::min(want, std::min(kMaxAttnSplit, key_tiles / 2));
     if (want > 1) {
       const int tiles_per = (key_tiles + want - 1) / want;
       ap.keys_per_split = tiles_per * 64;
@@ -430,8 +425,7 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
     }
   }
   {
-    const double part = ap.n_split > 1 ? (double)ap.n_split * M * c.n_heads * c.head_dim * 4.0 : 0;
-    ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes + part, att_flops);
+    ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
     KL(launch_attn_mma(ap, ctx->stream, ctx->pdl));
   }
   return FDLLM_OK;
@@ -691,7 +685,8 @@ namespace fd {
 // Error message for calls without a ctx (fdllm_last_error(NULL)).
 void set_thread_error(const std::string& msg) { g_create_error = msg; }
 
-GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes) {
+GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes,
+                       int max_nt) {
   GemmShape g{};
   g.N = N;
   g.M = M;
@@ -699,7 +694,7 @@ GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_
   g.n_tiles = (N + 127) / 128;
   g.kb_total = (K + 63) / 64;
   int nt = 64;
-  while (nt / 2 < M && nt < 256) nt *= 2;
+  while (nt / 2 < M && nt < max_nt) nt *= 2;
   g.nt = nt;
   g.n_tt = (M + nt / 2 - 1) / (nt / 2);
   const int base_units = g.n_tiles * g.n_tt;
@@ -830,12 +825,6 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->n_counters = ((max_n + 127) / 128) * ((S + 31) / 32);
   ctx->counters = (int*)dalloc(ctx, sizeof(int) * ctx->n_counters);
   if (ctx->tc) ctx->ws = (float*)dalloc(ctx, kWorkspaceBytes);
-  const size_t attn_rows = (size_t)kAttnSplitMaxM * c.n_heads;
-  ctx->attn_po = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * c.head_dim);
-  ctx->attn_ml = (float*)dalloc(ctx, sizeof(float) * kMaxAttnSplit * attn_rows * 2);
-  // one counter per (query row tile of >= 16 rows, KV head) of a split launch (M <= 64)
-  const int attn_cnt_n = ((kAttnSplitMaxM * (c.n_heads / c.n_kv_heads) + 15) / 16) * c.n_kv_heads;
-  ctx->attn_cnt = (int*)dalloc(ctx, sizeof(int) * attn_cnt_n);
   const size_t max_parts = std::max<size_t>((size_t)ctx->num_sms,
                                             (size_t)((c.vocab + 127) / 128) * ((kMaxLmRows + 31) / 32));
   ctx->lm_part_cap = max_parts * kMaxLmRows;
@@ -853,10 +842,9 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->cap_f = arows * c.ffn_dim;
   for (void* p : {(void*)ctx->kv_pool, (void*)ctx->page_table, (void*)ctx->rope, (void*)ctx->x,
                   (void*)ctx->h, ctx->a, ctx->q, ctx->o, ctx->f, (void*)ctx->counters,
-                  (void*)ctx->attn_po, (void*)ctx->attn_ml, (void*)ctx->lm_part,
+                  (void*)ctx->lm_part,
                   (void*)ctx->conf, (void*)ctx->tok, (void*)ctx->unmask, (void*)ctx->state,
-                  (void*)ctx->err_dev, (void*)ctx->check, (void*)ctx->sp,
-                  (void*)ctx->attn_cnt})
+                  (void*)ctx->err_dev, (void*)ctx->check, (void*)ctx->sp})
     if (!p) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (ctx->tc && !ctx->ws) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (cudaMallocHost(&ctx->state_host, sizeof(DecodeState)) != cudaSuccess ||
@@ -883,7 +871,6 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
             cudaMemset(ctx->counters, 0, sizeof(int) * ctx->n_counters) == cudaSuccess &&
             cudaMemset(ctx->err_dev, 0, sizeof(int)) == cudaSuccess &&
             cudaMemset(ctx->check, 0, 4 * sizeof(int)) == cudaSuccess &&
-            cudaMemset(ctx->attn_cnt, 0, sizeof(int) * attn_cnt_n) == cudaSuccess &&
             cudaMemset(ctx->kv_pool, 0, kv_elems * ctx->esz) == cudaSuccess &&
             cudaMemset(ctx->a, 0, ctx->esz * arows * c.d_model) == cudaSuccess &&
             cudaMemset(ctx->o, 0, ctx->esz * arows * hq) == cudaSuccess &&
@@ -1007,17 +994,43 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
     lw.attn_norm = (float*)take(sizeof(float) * d);
     lw.ffn_norm = (float*)take(sizeof(float) * d);
     uint8_t* qkv = (uint8_t*)lw.wqkv;
-    CK(copy_to(qkv, p + "wq", (size_t)hq * d * es));
-    CK(copy_to(qkv + (size_t)hq * d * es, p + "wk", (size_t)hkv * d * es));
-    CK(copy_to(qkv + (size_t)(hq + hkv) * d * es, p + "wv", (size_t)hkv * d * es));
+    const size_t row = (size_t)d * es;  // bytes per weight row
+    if (ctx->tc) {
+      // q and k heads: within each head, slab s (32 rows) holds dims
+      // 16s .. 16s+15 then their rotate-half partners dims + hd/2 (the
+      // epilogue's rope_slab_dim); 2-D copies over the heads.
+      auto put_heads = [&](uint8_t* dst, const std::string& n, int heads) -> cudaError_t {
+        const uint8_t* src = (const uint8_t*)find(n)->data;
+        for (int sl = 0; sl < hd / 32; ++sl)
+          for (int half = 0; half < 2; ++half) {
+            cudaError_t e = cudaMemcpy2D(dst + (32 * sl + 16 * half) * row, hd * row,
+                                         src + (16 * sl + half * (hd / 2)) * row, hd * row,
+                                         16 * row, heads, cudaMemcpyDefault);
+            if (e != cudaSuccess) return e;
+          }
+        return cudaSuccess;
+      };
+      CK(put_heads(qkv, p + "wq", c.n_heads));
+      CK(put_heads(qkv + (size_t)hq * row, p + "wk", c.n_kv_heads));
+      CK(copy_to(qkv + (size_t)(hq + hkv) * row, p + "wv", (size_t)hkv * row));
+      // gate / up: slab s holds gate rows 16s .. 16s+15 then the matching up rows
+      CK(cudaMemcpy2D(lw.wgu, 32 * row, find(p + "w_gate")->data, 16 * row, 16 * row, F / 16,
+                      cudaMemcpyDefault));
+      CK(cudaMemcpy2D((uint8_t*)lw.wgu + 16 * row, 32 * row, find(p + "w_up")->data, 16 * row,
+                      16 * row, F / 16, cudaMemcpyDefault));
+    } else {
+      CK(copy_to(qkv, p + "wq", (size_t)hq * row));
+      CK(copy_to(qkv + (size_t)hq * row, p + "wk", (size_t)hkv * row));
+      CK(copy_to(qkv + (size_t)(hq + hkv) * row, p + "wv", (size_t)hkv * row));
+      // gate/up interleaved in groups of 64 rows: [g0..g63, u0..u63, g64..g127, ...]
+      const size_t grp = 64 * row;
+      CK(cudaMemcpy2D(lw.wgu, 2 * grp, find(p + "w_gate")->data, grp, grp, F / 64,
+                      cudaMemcpyDefault));
+      CK(cudaMemcpy2D((uint8_t*)lw.wgu + grp, 2 * grp, find(p + "w_up")->data, grp, grp, F / 64,
+                      cudaMemcpyDefault));
+    }
     CK(copy_to(lw.wo, p + "wo", (size_t)d * hq * es));
     CK(copy_to(lw.wd, p + "w_down", (size_t)d * F * es));
-    // gate/up interleaved in groups of 64 rows: [g0..g63, u0..u63, g64..g127, ...]
-    const size_t grp = 64ull * d * es;
-    CK(cudaMemcpy2D(lw.wgu, 2 * grp, find(p + "w_gate")->data, grp, grp, F / 64,
-                    cudaMemcpyDefault));
-    CK(cudaMemcpy2D((uint8_t*)lw.wgu + grp, 2 * grp, find(p + "w_up")->data, grp, grp, F / 64,
-                    cudaMemcpyDefault));
     CK(norm_to(lw.attn_norm, p + "attn_norm"));
     CK(norm_to(lw.ffn_norm, p + "ffn_norm"));
     CK(to_f16(lw.wqkv, (size_t)(hq + 2 * hkv) * d));

@@ -24,10 +24,11 @@
 // stored activation of the bf16 model (see split_f16).  Online softmax in
 // f32, exp2 domain.
 //
-// With n_split > 1 (long sequences) each split writes unnormalised partial
-// outputs and its (max, sum) per row; the last split CTA of a (row tile, KV
-// head) to arrive (a self-resetting counter) merges all splits in split
-// order and writes o, so the result does not depend on arrival order.
+// With n_split > 1 (block steps: few query rows, so the keys are split to
+// fill the SMs) the n_split CTAs of a (row tile, KV head) run as one
+// thread-block cluster; each keeps its unnormalised partial output and
+// (max, sum) per row in shared memory and cluster rank 0 merges them in
+// split order over distributed shared memory and writes o.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -35,7 +36,7 @@ namespace fd {
 
 namespace {
 
-constexpr int kMaxSplit = 16;
+constexpr int kMaxSplit = 8;  // portable thread-block cluster size
 
 FD_DEV void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
@@ -276,12 +277,57 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   }
   const bool writer = warp_active && kg == 0;
 
+  // ---- merge the key splits of this (row tile, KV head): the n_split CTAs
+  // form one thread-block cluster (cluster rank = split index); rank 0 folds
+  // ranks 1, 2, ... in order through distributed shared memory, so the
+  // result does not depend on timing.
+  if (p.n_split > 1) {
+    constexpr int PER_LANE = HD / 2 + 4;
+    float* xch = reinterpret_cast<float*>(sm + 2 * TILE);
+    float* mine = xch + (size_t)(warp * 32 + lane) * PER_LANE;
+    __syncthreads();  // the key-group merge above is done with xch
+    if (writer) {
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mine[j * 4 + c] = oacc[j][c];
+      mine[HD / 2] = mrow[0];
+      mine[HD / 2 + 1] = mrow[1];
+      mine[HD / 2 + 2] = lrow[0];
+      mine[HD / 2 + 3] = lrow[1];
+    }
+    cluster_sync();  // every split's state is in its shared memory
+    if (cluster_rank() == 0 && writer) {
+      for (int k = 1; k < p.n_split; ++k) {
+        const uint32_t rem = cluster_map(smem_u32(mine), k);
+        float other[PER_LANE];
+#pragma unroll
+        for (int i = 0; i < PER_LANE; i += 4) ld_cluster_v4(rem + 4 * i, other + i);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float mo = other[HD / 2 + r], lo_ = other[HD / 2 + 2 + r];
+          const float mn = fmaxf(mrow[r], mo);
+          const float a = (mrow[r] == -INFINITY) ? 0.0f : exp2f(mrow[r] - mn);
+          const float b = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+#pragma unroll
+          for (int j = 0; j < HD / 8; ++j) {
+            oacc[j][2 * r] = oacc[j][2 * r] * a + other[j * 4 + 2 * r] * b;
+            oacc[j][2 * r + 1] = oacc[j][2 * r + 1] * a + other[j * 4 + 2 * r + 1] * b;
+          }
+          lrow[r] = lrow[r] * a + lo_ * b;
+          mrow[r] = mn;
+        }
+      }
+    }
+    cluster_sync();  // ranks 1.. keep their shared memory until rank 0 has read it
+    if (cluster_rank() != 0) return;
+  }
+
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
     lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
   }
-  const int rows_all = p.M * H;
   const int hq = H * HD;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -289,107 +335,20 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     const int rr = row0 + rg * 16 + (lane >> 2) + 8 * r;
     if (rr >= rows_total) continue;
     const int m = rr / rep, head = g * rep + rr % rep;
-    const size_t orow = (size_t)m * H + head;
-    if (p.n_split == 1) {
-      const float inv = 1.0f / lrow[r];
-      __half* o = reinterpret_cast<__half*>(p.o);
-      const size_t hi_off = (size_t)pair_row(m) * hq + (size_t)head * HD;
-      const size_t lo_off = hi_off + (size_t)PAIR_LO * hq;
+    const float inv = 1.0f / lrow[r];
+    __half* o = reinterpret_cast<__half*>(p.o);
+    const size_t hi_off = (size_t)pair_row(m) * hq + (size_t)head * HD;
+    const size_t lo_off = hi_off + (size_t)PAIR_LO * hq;
 #pragma unroll
-      for (int j = 0; j < HD / 8; ++j) {
-        const int d = j * 8 + 2 * (lane & 3);
-        __half h0, l0, h1, l1;
-        split_f16(oacc[j][2 * r] * inv, h0, l0);
-        split_f16(oacc[j][2 * r + 1] * inv, h1, l1);
-        *reinterpret_cast<__half2*>(o + hi_off + d) = __halves2half2(h0, h1);
-        *reinterpret_cast<__half2*>(o + lo_off + d) = __halves2half2(l0, l1);
-      }
-    } else {
-      float* po = p.part_o + ((size_t)blockIdx.z * rows_all + orow) * HD;
-#pragma unroll
-      for (int j = 0; j < HD / 8; ++j) {
-        const int d = j * 8 + 2 * (lane & 3);
-        *reinterpret_cast<float2*>(po + d) = make_float2(oacc[j][2 * r], oacc[j][2 * r + 1]);
-      }
-      if ((lane & 3) == 0) {
-        float* ml = p.part_ml + ((size_t)blockIdx.z * rows_all + orow) * 2;
-        ml[0] = mrow[r];
-        ml[1] = lrow[r];
-      }
+    for (int j = 0; j < HD / 8; ++j) {
+      const int d = j * 8 + 2 * (lane & 3);
+      __half h0, l0, h1, l1;
+      split_f16(oacc[j][2 * r] * inv, h0, l0);
+      split_f16(oacc[j][2 * r + 1] * inv, h1, l1);
+      *reinterpret_cast<__half2*>(o + hi_off + d) = __halves2half2(h0, h1);
+      *reinterpret_cast<__half2*>(o + lo_off + d) = __halves2half2(l0, l1);
     }
   }
-  if (p.n_split == 1) return;
-
-  // ---- split merge by the last split CTA of this (row tile, KV head)
-  __shared__ int s_last;
-  __shared__ float s_w[64][kMaxSplit];
-  __shared__ float s_inv[64];
-  __threadfence();
-  __syncthreads();
-  int* cnt = p.counters + blockIdx.y * gridDim.x + blockIdx.x;
-  if (tid == 0) {
-    const int prev = atomicAdd(cnt, 1);
-    s_last = (prev == p.n_split - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int n_rows = min(16 * NRG, rows_total - row0);
-  if (tid < n_rows) {  // per-row split weights
-    const int rr = row0 + tid;
-    const size_t orow = (size_t)(rr / rep) * H + g * rep + rr % rep;
-    float mc[kMaxSplit], lc[kMaxSplit];
-    float mstar = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kMaxSplit; ++c) {
-      mc[c] = c < p.n_split ? __ldcg(p.part_ml + ((size_t)c * rows_all + orow) * 2) : -INFINITY;
-      lc[c] = c < p.n_split ? __ldcg(p.part_ml + ((size_t)c * rows_all + orow) * 2 + 1) : 0.0f;
-      mstar = fmaxf(mstar, mc[c]);
-    }
-    float den = 0.0f;
-#pragma unroll
-    for (int c = 0; c < kMaxSplit; ++c) {
-      const float w = mc[c] == -INFINITY ? 0.0f : exp2f(mc[c] - mstar);
-      s_w[tid][c] = w;
-      den += w * lc[c];
-    }
-    s_inv[tid] = 1.0f / den;
-  }
-  __syncthreads();
-  __half* o = reinterpret_cast<__half*>(p.o);
-  // 8 outputs per thread per pass, every partial load issued before any store
-  for (int base = 0; base < n_rows * HD; base += 128 * 8) {
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-    for (int c = 0; c < p.n_split; ++c) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int idx = base + e * 128 + tid;
-        if (idx < n_rows * HD) {
-          const int i = idx / HD, d = idx % HD;
-          const int rr = row0 + i;
-          const size_t orow = (size_t)(rr / rep) * H + g * rep + rr % rep;
-          acc[e] += s_w[i][c] * __ldcg(p.part_o + ((size_t)c * rows_all + orow) * HD + d);
-        }
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int idx = base + e * 128 + tid;
-      if (idx < n_rows * HD) {
-        const int i = idx / HD, d = idx % HD;
-        const int rr = row0 + i;
-        const int m = rr / rep, head = g * rep + rr % rep;
-        __half hi, lo;
-        split_f16(acc[e] * s_inv[i], hi, lo);
-        const size_t off = (size_t)pair_row(m) * hq + (size_t)head * HD + d;
-        o[off] = hi;
-        o[off + (size_t)PAIR_LO * hq] = lo;
-      }
-    }
-  }
-  if (tid == 0) *cnt = 0;
 }
 
 template <int HD, int NKG>
@@ -409,8 +368,28 @@ cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
   }
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
   const int rows_per_cta = 16 * (4 / NKG);
-  dim3 grid((rows + rows_per_cta - 1) / rows_per_cta, p.n_kv_heads, p.n_split);
-  return launch_k(pdl, attn_mma_kernel<HD, NKG>, grid, dim3(128), (size_t)smem, st, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + rows_per_cta - 1) / rows_per_cta, p.n_kv_heads, p.n_split);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute la[2];
+  int na = 0;
+  if (pdl) {
+    la[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (p.n_split > 1) {  // the splits of a (row tile, KV head) form one cluster
+    la[na].id = cudaLaunchAttributeClusterDimension;
+    la[na].val.clusterDim.x = 1;
+    la[na].val.clusterDim.y = 1;
+    la[na].val.clusterDim.z = p.n_split;
+    ++na;
+  }
+  cfg.attrs = la;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<HD, NKG>, p);
 }
 
 template <int HD>

@@ -1,14 +1,18 @@
-// GEMM epilogues shared by the tcgen05 GEMM (bf16 model) and the CUDA-core
-// GEMM (fp32 model).
+// GEMM epilogues.
 //
-// Both GEMMs hand the epilogue output tiles of 128 features x 32 tokens,
-// staged in shared memory as float tile[t * 128 + e] (t = token row in the
-// chunk, e = feature within the 128-feature tile).  The 128 epilogue threads
-// call epi_chunk with e = their feature index.  Control flow is uniform
-// within each warp (the LM-head reduction uses warp shuffles).
+// epi_chunk: output tiles of 128 features x 32 tokens staged in shared
+// memory as float tile[t * 128 + e] (t = token row in the chunk, e = feature
+// within the 128-feature tile); the 128 epilogue threads call it with e =
+// their feature index.  It serves every epilogue of the CUDA-core GEMM (fp32
+// model, natural weight-row order) and the LM-head reduction of the tcgen05
+// GEMM.  Control flow is uniform within each warp (the LM-head reduction
+// uses warp shuffles).
 //
-// Stores of the bf16 model are two-term fp16 (hi + lo, see split_f16): the q
-// planes, the K/V cache planes and the SwiGLU output in pair rows.
+// epi_regs: the other epilogues of the tcgen05 GEMM (bf16 model), straight
+// from the registers the accumulator was read into, on the permuted weight
+// rows described at rope_slab_dim.  Its stores are two-term fp16 (hi + lo,
+// see split_f16): the q planes, the K/V cache planes and the SwiGLU output
+// in pair rows.
 #pragma once
 
 #include "common.cuh"
@@ -32,15 +36,13 @@ FD_DEV size_t kv_offset_pg(const EpiParams& ep, int page, int pos, int plane, in
 //   tile: [32][128] float in shared memory, fully written before the call.
 //   n0:   first feature of the tile; t0: token row of tile row 0.
 //   lm:   per-token softmax states of this CTA (EPI_LMHEAD only).
-template <bool F32>
 FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, int e,
                       SoftmaxState* lm) {
   const int n = n0 + e;
   switch (ep.kind) {
     case EPI_STORE: {
       if (n < ep.N)
-        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t)
-        {
+        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
           const size_t i = (size_t)(t0 + t) * ep.ld_out + n;
           if (FD_CHECK(i < ep.cap_out, ep.check, 1, i, ep.cap_out)) ep.out[i] = tile[t * 128 + e];
         }
@@ -66,35 +68,22 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
       break;
     }
     case EPI_SWIGLU: {
-      // Rows [128j, 128j+64) of the fused weight are gate rows [64j, 64j+64),
-      // rows [128j+64, 128j+128) the matching up rows.
+      // fp32 model: rows [128j, 128j+64) of the fused weight are gate rows
+      // [64j, 64j+64), rows [128j+64, 128j+128) the matching up rows.
       const int F = ep.N / 2;
       const int j = (n0 / 128) * 64 + e;
       if (e < 64 && j < F)
         for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
           const float g = tile[t * 128 + e];
           const float u = tile[t * 128 + e + 64];
-          const float y = silu_f(g) * u;
-          const int tok = t0 + t;
-          if (F32) {
-            const size_t i = (size_t)tok * F + j;
-            if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f))
-              reinterpret_cast<float*>(ep.f_out)[i] = y;
-          } else {
-            __half hi, lo;
-            split_f16(y, hi, lo);
-            __half* f = reinterpret_cast<__half*>(ep.f_out);
-            const size_t r = (size_t)pair_row(tok);
-            const size_t i = (r + PAIR_LO) * F + j;
-            if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f)) {
-              f[r * F + j] = hi;
-              f[i] = lo;
-            }
-          }
+          const size_t i = (size_t)(t0 + t) * F + j;
+          if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f))
+            reinterpret_cast<float*>(ep.f_out)[i] = silu_f(g) * u;
         }
       break;
     }
     case EPI_QKV: {
+      // fp32 model: natural row order, RoPE partners through the tile
       if (n >= ep.N) break;
       const int hd = ep.head_dim, half = hd / 2;
       const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
@@ -119,6 +108,7 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
         page0 = __ldg(&ep.page_table[pidx0]);
         page1 = __ldg(&ep.page_table[(pos0 + t0 + nt - 1) / KV_PAGE]);
       }
+      float* kv = reinterpret_cast<float*>(ep.kv_pool);
 #pragma unroll
       for (int t = 0; t < CHUNK_T; ++t) {
         if (t >= nt) break;
@@ -135,48 +125,14 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
           }
         }
         const int page = (pos / KV_PAGE == pidx0) ? page0 : page1;
-        if (F32) {
-          float* kv = reinterpret_cast<float*>(ep.kv_pool);
-          if (is_q) {
-            const size_t i = (size_t)tok * hq + n;
-            if (FD_CHECK(i < ep.cap_q, ep.check, 4, i, ep.cap_q))
-              reinterpret_cast<float*>(ep.q_out)[i] = y;
-          } else {
-            const size_t i = is_v ? kv_offset_pg(ep, page, pos, 1, (n - hq - hk) / hd, dh)
-                                  : kv_offset_pg(ep, page, pos, 0, (n - hq) / hd, dh);
-            if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
-          }
-        } else if (is_q) {
-          __half hi, lo;
-          split_f16(y, hi, lo);
-          __half* q = reinterpret_cast<__half*>(ep.q_out);
+        if (is_q) {
           const size_t i = (size_t)tok * hq + n;
-          if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
-            q[i] = hi;
-            q[ep.q_plane + i] = lo;
-          }
-        } else if (!is_v) {
-          __half hi, lo;
-          split_f16(y, hi, lo);
-          __half* k = reinterpret_cast<__half*>(ep.kv_pool);
-          const int head = (n - hq) / hd;
-          const size_t i0 = kv_offset_pg(ep, page, pos, 0, head, dh);
-          const size_t i1 = kv_offset_pg(ep, page, pos, 1, head, dh);
-          if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
-            k[i0] = hi;
-            k[i1] = lo;
-          }
+          if (FD_CHECK(i < ep.cap_q, ep.check, 4, i, ep.cap_q))
+            reinterpret_cast<float*>(ep.q_out)[i] = y;
         } else {
-          __half hi, lo;
-          split_f16(y, hi, lo);
-          __half* v = reinterpret_cast<__half*>(ep.kv_pool);
-          const int head = (n - hq - hk) / hd;
-          const size_t i0 = kv_offset_pg(ep, page, pos, 2, head, dh);
-          const size_t i1 = kv_offset_pg(ep, page, pos, 3, head, dh);
-          if (FD_CHECK(i1 < ep.cap_kv, ep.check, 6, i1, ep.cap_kv)) {
-            v[i0] = hi;
-            v[i1] = lo;
-          }
+          const size_t i = is_v ? kv_offset_pg(ep, page, pos, 1, (n - hq - hk) / hd, dh)
+                                : kv_offset_pg(ep, page, pos, 0, (n - hq) / hd, dh);
+          if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
         }
       }
       break;
@@ -210,6 +166,146 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
         }
         s = warp_sum(s);
         if (lane == 0) lm[tok] = sm_merge(lm[tok], SoftmaxState{mx, s, arg});
+      }
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+// Weight-row order of the tensor-core path inside every 32-row slab (one
+// warp's TMEM lanes), so that the two rows an epilogue output needs sit 16
+// lanes apart in the same warp and meet through one shuffle:
+//   q / k heads: slab s of a head (rows 32s .. 32s+31) holds dims
+//                16s .. 16s+15 in lanes 0..15 and their rotate-half partners
+//                (dim + hd/2) in lanes 16..31; rope_slab_dim maps the row
+//                r within the head to its dim;
+//   gate / up:   slab s of the fused matrix holds gate features
+//                16s .. 16s+15 in lanes 0..15 and the matching up features
+//                in lanes 16..31.
+// The V rows and every other weight keep their natural order.
+FD_DEV __host__ int rope_slab_dim(int r, int hd) {
+  return 16 * (r >> 5) + (r & 15) + ((r >> 4) & 1) * (hd / 2);
+}
+
+// Epilogue of one 32-token chunk held in registers by the 128 threads of an
+// epilogue warpgroup: v[t] = output feature n0 + e of token row t0 + t.
+// e = tile row = 32 * (warp % 4) + lane.  Shuffles stay within a warp and
+// control flow is warp-uniform (N and the q / k / v region boundaries are
+// multiples of 64 for the QKV and SwiGLU layouts).  EPI_LMHEAD is not
+// handled here: it needs all 128 features of a token (epi_chunk).
+FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0, int e) {
+  const int lane = e & 31;
+  const int n = n0 + e;
+  const int nt = min(CHUNK_T, ep.M - t0);
+  if (nt <= 0) return;
+  switch (ep.kind) {
+    case EPI_STORE: {
+      if (n >= ep.N) break;
+#pragma unroll
+      for (int t = 0; t < CHUNK_T; ++t) {
+        if (t >= nt) break;
+        const size_t i = (size_t)(t0 + t) * ep.ld_out + n;
+        if (FD_CHECK(i < ep.cap_out, ep.check, 1, i, ep.cap_out)) ep.out[i] = v[t];
+      }
+      break;
+    }
+    case EPI_RESID: {
+      // all loads of h before any store (see epi_chunk)
+      if (n >= ep.N) break;
+      float hv[CHUNK_T];
+#pragma unroll
+      for (int t = 0; t < CHUNK_T; ++t)
+        hv[t] = (t < nt) ? ep.h[(size_t)(t0 + t) * ep.N + n] : 0.0f;
+#pragma unroll
+      for (int t = 0; t < CHUNK_T; ++t) {
+        if (t >= nt) break;
+        const size_t i = (size_t)(t0 + t) * ep.N + n;
+        if (FD_CHECK(i < ep.cap_h, ep.check, 2, i, ep.cap_h)) ep.h[i] = hv[t] + v[t];
+      }
+      break;
+    }
+    case EPI_SWIGLU: {
+      if (n >= ep.N) break;  // warp-uniform
+      const int F = ep.N / 2;
+      const int j = 16 * (n >> 5) + (lane & 15);  // FFN feature of this lane pair
+      const bool up = lane >= 16;
+      __half* f = reinterpret_cast<__half*>(ep.f_out);
+#pragma unroll
+      for (int t = 0; t < CHUNK_T; ++t) {
+        if (t >= nt) break;
+        const float p = __shfl_xor_sync(0xffffffffu, v[t], 16);
+        const float g = up ? p : v[t];
+        const float u = up ? v[t] : p;
+        __half hi, lo;
+        split_f16(silu_f(g) * u, hi, lo);
+        // lanes 0..15 store the hi term, lanes 16..31 the lo term
+        const size_t i = ((size_t)pair_row(t0 + t) + (up ? PAIR_LO : 0)) * F + j;
+        if (FD_CHECK(i < ep.cap_f, ep.check, 3, i, ep.cap_f)) f[i] = up ? lo : hi;
+      }
+      break;
+    }
+    case EPI_QKV: {
+      if (n >= ep.N) break;  // warp-uniform
+      const int hd = ep.head_dim, half = hd / 2;
+      const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
+      const int region = n < hq ? 0 : (n < hq + hk ? 1 : 2);  // q, k, v (uniform per warp)
+      const int rn = n - (region == 0 ? 0 : (region == 1 ? hq : hq + hk));
+      const int head = rn / hd;
+      const int r = rn - head * hd;
+      const int dim = region < 2 ? rope_slab_dim(r, hd) : r;
+      const int pos0 = (ep.sp ? ep.sp->r0 : ep.pos0) + t0;
+      const bool second = lane >= 16;  // holds dim + hd/2 of the rotate-half pair
+      int page0 = 0, page1 = 0;
+      if (region > 0) {
+        page0 = __ldg(&ep.page_table[pos0 / KV_PAGE]);
+        page1 = __ldg(&ep.page_table[(pos0 + nt - 1) / KV_PAGE]);
+      }
+      // 16 tokens at a time: the RoPE table loads of a half are issued
+      // before its stores (see EPI_RESID), in fewer registers than 32.
+#pragma unroll
+      for (int h16 = 0; h16 < CHUNK_T; h16 += 16) {
+        if (h16 >= nt) break;
+        float2 cs[16];
+        if (region < 2) {
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            cs[t] = (h16 + t < nt)
+                        ? __ldg(&ep.rope[(size_t)(pos0 + h16 + t) * half + (dim % half)])
+                        : make_float2(1.0f, 0.0f);
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          if (h16 + t >= nt) break;
+          float y = v[h16 + t];
+          if (region < 2) {
+            const float p = __shfl_xor_sync(0xffffffffu, y, 16);
+            y = second ? (y * cs[t].x + p * cs[t].y) : (y * cs[t].x - p * cs[t].y);
+          }
+          __half hi, lo;
+          split_f16(y, hi, lo);
+          const int tok = t0 + h16 + t;
+          const int pos = pos0 + h16 + t;
+          if (region == 0) {
+            __half* q = reinterpret_cast<__half*>(ep.q_out);
+            const size_t i = (size_t)tok * hq + head * hd + dim;
+            if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
+              q[i] = hi;
+              q[ep.q_plane + i] = lo;
+            }
+          } else {
+            const int page = (pos / KV_PAGE == pos0 / KV_PAGE) ? page0 : page1;
+            const int plane = region == 1 ? 0 : 2;
+            __half* kv = reinterpret_cast<__half*>(ep.kv_pool);
+            const size_t i0 = kv_offset_pg(ep, page, pos, plane, head, dim);
+            const size_t i1 = kv_offset_pg(ep, page, pos, plane + 1, head, dim);
+            if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
+              kv[i0] = hi;
+              kv[i1] = lo;
+            }
+          }
+        }
       }
       break;
     }

@@ -5,16 +5,19 @@
 // model's output features fill the MMA's M = 128; the few block tokens are
 // the MMA's N), so a block step with 32 tokens still issues full 128-row
 // MMAs while it streams the weights once from HBM.  The activations are
-// two-term (hi + lo bf16) in pair rows: every 64 rows hold the hi and the lo
-// term of 32 tokens, so a token tile of NT rows covers NT/2 tokens and the
-// lo term costs tensor work only (the weights are read once).  Both operands
-// are K-major, staged by TMA with the 128-byte swizzle into a STAGES-deep
-// ring of shared-memory buffers; one thread issues tcgen05.mma into a
-// double-buffered TMEM accumulator (128 lanes x NT columns each), and four
-// epilogue warps drain the accumulator with tcgen05.ld, 64 columns (hi and
-// lo of 32 tokens, summed) at a time, through the shared epilogue (RoPE +
-// KV-cache write, residual add, SwiGLU, or the fused LM-head
-// max/argmax/sum-exp).
+// two-term (hi + lo) in pair rows: every 64 rows hold the hi and the lo term
+// of 32 tokens, so a token tile of NT rows covers NT/2 tokens and the lo term
+// costs tensor work only (the weights are read once).  Both operands are
+// K-major, staged by TMA with the 128-byte swizzle into a STAGES-deep ring of
+// shared-memory buffers; one thread issues tcgen05.mma into a ring of NBUF
+// TMEM accumulators (128 lanes x NT columns each), one per accumulation chain
+// of at most KC K blocks.  The epilogue warps read each chain with
+// tcgen05.ld (64 columns: hi and lo of 32 tokens, summed), add the chains up
+// in float32 registers and hand the buffer back at once, so the next unit's
+// MMAs overlap the epilogue's global-memory work.  The epilogue itself
+// (RoPE + KV-cache write, residual add, SwiGLU) runs from registers on the
+// permuted weight rows of epi_regs; the fused LM-head max/argmax/sum-exp
+// goes through a shared tile (epi_chunk).
 //
 // Work units are (feature tile, token tile, K split).  CTAs loop over units
 // with a stride of gridDim.x.  With more than one split, each split writes
@@ -22,8 +25,11 @@
 // atomic counter per tile, reset by that CTA) sums the partials in split
 // order, so results do not depend on arrival order.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
-// MMA issuer, warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
+// Warp roles: warp 0 = TMA producer, warp 1 = TMEM owner and MMA issuer,
+// warps 2.. = EG epilogue warpgroups (TMEM lane quadrant = warp % 4; group g
+// takes tokens [g * TOK / EG, (g + 1) * TOK / EG) of each tile).  NT = 256
+// runs two epilogue warpgroups (320 threads) to hold its 128 tokens of
+// accumulators in registers.
 #include <type_traits>
 
 #include "common.cuh"
@@ -40,25 +46,30 @@ constexpr int LM_MAX_ROWS = 256;          // largest M for the LM-head epilogue
 
 
 template <int NT> struct TcCfg;
-template <> struct TcCfg<64> { static constexpr int STAGES = 8; };
-template <> struct TcCfg<128> { static constexpr int STAGES = 6; };
-template <> struct TcCfg<256> { static constexpr int STAGES = 4; };
+template <> struct TcCfg<64> { static constexpr int STAGES = 8, NBUF = 4, EG = 1; };
+template <> struct TcCfg<128> { static constexpr int STAGES = 6, NBUF = 4, EG = 1; };
+template <> struct TcCfg<256> { static constexpr int STAGES = 4, NBUF = 2, EG = 2; };
 
 template <int NT>
 struct TcLayout {
   static constexpr int STAGES = TcCfg<NT>::STAGES;
+  static constexpr int NBUF = TcCfg<NT>::NBUF;   // TMEM accumulator buffers
+  static constexpr int EG = TcCfg<NT>::EG;       // epilogue warpgroups
+  static constexpr bool LM = EG == 1;            // LM-head epilogue available
+  static constexpr int THREADS = 64 + 128 * EG;
   static constexpr int B_STAGE_BYTES = NT * BK * 2;
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + STAGES * A_STAGE_BYTES;
   static constexpr int TILE_OFF = B_OFF + STAGES * B_STAGE_BYTES;
-  static constexpr int BAR_OFF = TILE_OFF + CHUNK_T * 128 * 4;
-  static constexpr int N_BARS = 2 * STAGES + 4;
+  static constexpr int BAR_OFF = TILE_OFF + (LM ? CHUNK_T * 128 * 4 : 0);
+  static constexpr int N_BARS = 2 * STAGES + 2 * NBUF;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int LM_OFF = MISC_OFF + 16;
-  static constexpr int END = LM_OFF + LM_MAX_ROWS * (int)sizeof(SoftmaxState);
+  static constexpr int END = LM_OFF + (LM ? LM_MAX_ROWS * (int)sizeof(SoftmaxState) : 0);
   static constexpr int SMEM = END + 1024;  // slack for 1024-byte alignment
   static_assert(B_STAGE_BYTES % 1024 == 0, "B stages must stay 1024-byte aligned");
   static_assert(SMEM <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
+  static_assert(NBUF * NT <= 512, "TMEM holds 512 columns");
 };
 
 struct UnitCoord {
@@ -77,16 +88,19 @@ FD_DEV UnitCoord decode_unit(const GemmShape& gs, int u) {
 }
 
 template <int NT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap,
                    const __grid_constant__ CUtensorMap amap, GemmShape gs, EpiParams ep,
                    GemmScratch sc) {
   constexpr int TOK = NT / 2;  // tokens per token tile
   using Lay = TcLayout<NT>;
   constexpr int STAGES = Lay::STAGES;
+  constexpr int NBUF = Lay::NBUF;
+  constexpr int EPI_ALL = 128 * Lay::EG;   // epilogue threads
+  constexpr int GT = TOK / Lay::EG;        // tokens per epilogue warpgroup
   // operand type: fp16 (the decoder's weights and two-term activations) or bf16
   const uint32_t idesc = gs.f16 ? idesc_f32acc(NT, true) : idesc_f32acc(NT, false);
-  constexpr uint32_t TMEM_COLS = 2 * NT;
+  constexpr uint32_t TMEM_COLS = NBUF * NT;
   constexpr uint32_t STAGE_TX = A_STAGE_BYTES + Lay::B_STAGE_BYTES;
   const int KC = gs.kc;  // K blocks per TMEM accumulation chain (see plan_gemm_tc)
 
@@ -100,7 +114,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
-  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint64_t* acc_empty = bars + 2 * STAGES + NBUF;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 2);
@@ -108,16 +122,16 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool lmhead = ep.kind == EPI_LMHEAD;
+  const bool lmhead = Lay::LM && ep.kind == EPI_LMHEAD;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NBUF; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], EPI_THREADS);
+      mbar_init(&acc_empty[i], EPI_ALL);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 1) tmem_alloc(misc, TMEM_COLS);
   if (lmhead && warp >= 2) {
-    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_THREADS)
+    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_ALL)
       lm[t] = sm_empty();
   }
   tc_fence_before();
@@ -191,15 +205,16 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       // Each unit's K range is accumulated in TMEM in chains of at most KC
-      // K blocks (one accumulator buffer per chain, alternating); the
-      // epilogue warps add the chains up in float32 registers.
+      // K blocks (one accumulator buffer per chain, NBUF buffers in
+      // rotation); the epilogue warps add the chains up in float32 registers
+      // and release each buffer as soon as they have read it.
       uint32_t it = 0, chain = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < gs.units && ok; u += gridDim.x) {
         const UnitCoord c = decode_unit(gs, u);
         for (int k0 = c.kb_lo; k0 < c.kb_hi && ok; k0 += KC, ++chain) {
-          const uint32_t buf = chain & 1u;
-          if (!mbar_wait(&acc_empty[buf], ((chain >> 1) & 1u) ^ 1u, sc.err, abort_flag)) {
+          const uint32_t buf = chain % NBUF;
+          if (!mbar_wait(&acc_empty[buf], ((chain / NBUF) & 1u) ^ 1u, sc.err, abort_flag)) {
             ok = false;
             break;
           }
@@ -225,106 +240,103 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    // Warpgroup grp handles tokens [grp * GT, (grp + 1) * GT) of each token
+    // tile; its warps read TMEM lane quadrant warp % 4 (feature rows).
+    const int grp = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int e = quad * 32 + lane;  // feature row = TMEM lane
+    const bool leader = warp == 2 && lane == 0;
     pdl_wait();                      // reads / writes of the previous kernel's data follow
     uint32_t chain = 0;
     for (int u = blockIdx.x; u < gs.units; u += gridDim.x) {
       const UnitCoord c = decode_unit(gs, u);
-      // acc[t] = this lane's feature for token t of the tile: the sum over the
-      // unit's accumulation chains of the hi- and lo-term columns (columns
-      // [64g, 64g+32) of a chain buffer hold the hi term of tokens 32g..,
-      // the next 32 their lo term).  The sums are written back into the
-      // first TOK columns of the last chain's buffer, which the epilogue
-      // keeps until the unit is done, and read back 32 tokens at a time.
-      float acc[TOK];
+      // acc[t] = this lane's feature for token grp * GT + t of the tile: the
+      // sum over the unit's accumulation chains of the hi- and lo-term
+      // columns (columns [64g, 64g+32) of a chain buffer hold the hi term of
+      // tokens 32g.., the next 32 their lo term).
+      float acc[GT];
 #pragma unroll
-      for (int t = 0; t < TOK; ++t) acc[t] = 0.0f;
+      for (int t = 0; t < GT; ++t) acc[t] = 0.0f;
       bool got = true;
-      uint32_t col = 0, last_buf = 0;
       for (int k0 = c.kb_lo; k0 < c.kb_hi; k0 += KC, ++chain) {
-        const uint32_t buf = chain & 1u;
-        got = mbar_wait(&acc_full[buf], (chain >> 1) & 1u, sc.err, abort_flag) && got;
+        const uint32_t buf = chain % NBUF;
+        got = mbar_wait(&acc_full[buf], (chain / NBUF) & 1u, sc.err, abort_flag) && got;
         tc_fence_after();
-        col = tmem + ((uint32_t)(quad * 32) << 16) + buf * NT;
+        const uint32_t col = tmem + ((uint32_t)(quad * 32) << 16) + buf * NT + grp * 2 * GT;
 #pragma unroll
-        for (int g = 0; g < TOK / 32; ++g) {
+        for (int g = 0; g < GT / 32; ++g) {
           float v[64];
           tmem_ld64(col + g * 64, v);
 #pragma unroll
           for (int t = 0; t < 32; ++t) acc[g * 32 + t] += v[t] + v[t + 32];
         }
-        last_buf = buf;
-        if (k0 + KC < c.kb_hi) {
-          tc_fence_before();
-          mbar_arrive(&acc_empty[buf]);
-        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
       }
-#pragma unroll
-      for (int g = 0; g < TOK / 32; ++g) tmem_st32(col + g * 32, acc + g * 32);
       const int n0 = c.tile * 128;
       const int tile_id = c.tile * gs.n_tt + c.tt;
-      float* ws_unit = sc.ws + ((size_t)tile_id * gs.splits + c.split) * (TOK * 128);
-      for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
-        float v[32];
-        tmem_ld32(col + ch * 32, v);
-        if (gs.splits == 1) {
-          named_bar(1, EPI_THREADS);  // previous chunk's epilogue is done with `tile`
-#pragma unroll
-          for (int t = 0; t < 32; ++t) tile[t * 128 + e] = v[t];
-          named_bar(1, EPI_THREADS);
-          if (got) epi_chunk<false>(ep, tile, n0, c.tt * TOK + ch * CHUNK_T, e, lm);
-        } else {
-          const size_t wi = (size_t)(ws_unit - sc.ws) + (ch * CHUNK_T + 31) * 128 + e;
-          if (FD_CHECK(wi < sc.ws_elems, ep.check, 22, wi, sc.ws_elems)) {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) ws_unit[(ch * CHUNK_T + t) * 128 + e] = v[t];
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[last_buf]);
+      const int tg0 = c.tt * TOK + grp * GT;  // first token row of this warpgroup
+      bool run_epi = gs.splits == 1;
       if (gs.splits > 1) {
+        // float partial tile [TOK][128] of this split; the last split to
+        // arrive sums all of them in split order and runs the epilogue.
+        float* ws_unit = sc.ws + ((size_t)tile_id * gs.splits + c.split) * (TOK * 128);
+        const size_t wi = (size_t)(ws_unit - sc.ws) + (size_t)(grp * GT + GT - 1) * 128 + e;
+        if (FD_CHECK(wi < sc.ws_elems, ep.check, 22, wi, sc.ws_elems)) {
+#pragma unroll
+          for (int t = 0; t < GT; ++t) ws_unit[(grp * GT + t) * 128 + e] = acc[t];
+        }
         __threadfence();
-        named_bar(1, EPI_THREADS);
-        if (e == 0) {
+        named_bar(1, EPI_ALL);
+        if (leader) {
           int prev = -1;
           if (FD_CHECK(tile_id < sc.n_counters, ep.check, 23, tile_id, sc.n_counters))
             prev = atomicAdd(&sc.counters[tile_id], 1);
           *last_flag = (prev == gs.splits - 1);
         }
-        named_bar(1, EPI_THREADS);
-        if (*last_flag) {
+        named_bar(1, EPI_ALL);
+        run_epi = *last_flag;
+        if (run_epi) {
           __threadfence();
           const float* ws_tile = sc.ws + (size_t)tile_id * gs.splits * (TOK * 128);
-          for (int ch = 0; ch < TOK / CHUNK_T; ++ch) {
-            float racc[32];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) racc[t] = 0.0f;
-            for (int sp = 0; sp < gs.splits; ++sp) {
-              const float* p = ws_tile + (size_t)sp * (TOK * 128) + ch * CHUNK_T * 128 + e;
-              const size_t wi = (size_t)(p - sc.ws) + 31 * 128;
-              if (!FD_CHECK(wi < sc.ws_elems, ep.check, 24, wi, sc.ws_elems)) continue;
+          for (int t = 0; t < GT; ++t) acc[t] = 0.0f;
+          for (int sp = 0; sp < gs.splits; ++sp) {
+            const float* p = ws_tile + (size_t)sp * (TOK * 128) + (size_t)grp * GT * 128 + e;
+            const size_t pi = (size_t)(p - sc.ws) + (size_t)(GT - 1) * 128;
+            if (!FD_CHECK(pi < sc.ws_elems, ep.check, 24, pi, sc.ws_elems)) continue;
 #pragma unroll
-              for (int t = 0; t < 32; ++t) racc[t] += __ldcg(p + t * 128);
-            }
-            named_bar(1, EPI_THREADS);
-#pragma unroll
-            for (int t = 0; t < 32; ++t) tile[t * 128 + e] = racc[t];
-            named_bar(1, EPI_THREADS);
-            if (got) epi_chunk<false>(ep, tile, n0, c.tt * TOK + ch * CHUNK_T, e, lm);
+            for (int t = 0; t < GT; ++t) acc[t] += __ldcg(p + t * 128);
           }
-          if (e == 0) sc.counters[tile_id] = 0;
+          if (leader) sc.counters[tile_id] = 0;
         }
-        named_bar(1, EPI_THREADS);
       }
+      if (run_epi && got) {
+#pragma unroll
+        for (int ch = 0; ch < GT / CHUNK_T; ++ch) {
+          float v[CHUNK_T];
+#pragma unroll
+          for (int t = 0; t < CHUNK_T; ++t) v[t] = acc[ch * CHUNK_T + t];
+          if (lmhead) {
+            // all 128 features of a token meet in the shared tile
+            named_bar(1, EPI_ALL);  // previous chunk's reduction is done with `tile`
+#pragma unroll
+            for (int t = 0; t < CHUNK_T; ++t) tile[t * 128 + e] = v[t];
+            named_bar(1, EPI_ALL);
+            epi_chunk(ep, tile, n0, tg0 + ch * CHUNK_T, e, lm);
+          } else {
+            epi_regs(ep, v, n0, tg0 + ch * CHUNK_T, e);
+          }
+        }
+      }
+      if (gs.splits > 1) named_bar(1, EPI_ALL);  // last_flag is read before the next unit
     }
   }
 
   __syncthreads();
   if (lmhead && warp >= 2) {
     SoftmaxState* out = reinterpret_cast<SoftmaxState*>(ep.lm_part) + (size_t)blockIdx.x * gs.M;
-    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_THREADS) {
+    for (int t = threadIdx.x - 64; t < gs.M && t < LM_MAX_ROWS; t += EPI_ALL) {
       const size_t i = (size_t)blockIdx.x * gs.M + t;
       if (FD_CHECK(i < ep.cap_lm, ep.check, 25, i, ep.cap_lm)) out[t] = lm[t];
     }
@@ -351,7 +363,8 @@ cudaError_t launch_nt(const CUtensorMap* w_map, const CUtensorMap* act_map, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_k(pdl, gemm_tc_kernel<NT>, dim3(gs.grid), dim3(192), (size_t)TcLayout<NT>::SMEM,
+  return launch_k(pdl, gemm_tc_kernel<NT>, dim3(gs.grid), dim3(TcLayout<NT>::THREADS),
+                  (size_t)TcLayout<NT>::SMEM,
                   st, *w_map, *act_map, gs, ep, sc);
 }
 
@@ -369,7 +382,7 @@ int gemm_tc_smem_bytes(int nt) {
 cudaError_t launch_gemm_tc(const CUtensorMap* w_map, const CUtensorMap* act_map,
                            const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
                            cudaStream_t st, bool pdl) {
-  if (ep.kind == EPI_LMHEAD && gs.M > LM_MAX_ROWS) return cudaErrorInvalidValue;
+  if (ep.kind == EPI_LMHEAD && (gs.M > LM_MAX_ROWS || gs.nt > 128)) return cudaErrorInvalidValue;
   switch (gs.nt) {
     case 64: return launch_nt<64>(w_map, act_map, gs, ep, sc, st, pdl);
     case 128: return launch_nt<128>(w_map, act_map, gs, ep, sc, st, pdl);

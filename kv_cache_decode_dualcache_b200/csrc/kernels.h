@@ -90,10 +90,12 @@ struct GemmScratch {
 };
 
 // Tile / split plan of the tcgen05 GEMM for N output features, M tokens and
-// reduction length K on a GPU with num_sms SMs: token tile of nt rows (nt/2
-// tokens of two-term activations), K split chosen to balance the per-CTA K
-// blocks over the persistent grid, within ws_bytes of split-K workspace.
-GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes);
+// reduction length K on a GPU with num_sms SMs: token tile of nt <= max_nt
+// rows (nt/2 tokens of two-term activations), K split chosen to balance the
+// per-CTA K blocks over the persistent grid, within ws_bytes of split-K
+// workspace.  The LM-head epilogue needs max_nt <= 128.
+GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_t ws_bytes,
+                       int max_nt = 256);
 
 // Launch with the programmatic stream-serialization attribute (when pdl).
 template <typename... KArgs, typename... Args>
@@ -139,11 +141,8 @@ struct AttnParams {
   int M;               // query positions
   int L;               // keys [0, L)
   int n_heads, n_kv_heads, head_dim;
-  int n_split;         // key splits (1 = write o directly)
+  int n_split;         // key splits, <= 8: one thread-block cluster per (row tile, KV head)
   int keys_per_split;  // multiple of 64
-  float* part_o;       // [n_split][M*H][hd]
-  float* part_ml;      // [n_split][M*H][2]
-  int* counters;       // [row tiles * Hkv] arrival counters of the splits (self-resetting)
 };
 
 cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl = false);

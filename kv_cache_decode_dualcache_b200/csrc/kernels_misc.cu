@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(128)
   SoftmaxState* lmp = lm - t0;  // index by absolute token row
   if (ep.kind == EPI_LMHEAD && e < 32) lm[e] = sm_empty();
   __syncthreads();
-  epi_chunk<true>(ep, tile, n0, t0, e, lmp);
+  epi_chunk(ep, tile, n0, t0, e, lmp);
   __syncthreads();
   if (ep.kind == EPI_LMHEAD) {
     SoftmaxState* out = reinterpret_cast<SoftmaxState*>(ep.lm_part) + (size_t)blockIdx.x * gs.M;
