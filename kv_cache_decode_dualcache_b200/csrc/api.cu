@@ -127,6 +127,18 @@ struct fdllm_ctx {
     int launches;
   };
   std::map<std::tuple<int, int, int>, StepGraph> step_graphs;
+  // DualCache block steps of at most 32 tokens (bf16 model) run as one
+  // attention launch plus one chain-kernel launch per layer (chain.cu).
+  bool use_chain = true;
+  int* chain_sync = nullptr;        // per-phase done counters of one step, then the abort word
+  int chain_sync_cap = 0;
+  struct ChainProg {
+    std::vector<ChainArgs> launches;           // kernel arguments per launch
+    std::vector<int> first;                    // index of each launch's first phase in the step
+    std::vector<double> bytes, flops;          // algorithmic bytes / flops per launch
+    int n_phases = 0;
+  };
+  std::map<std::tuple<int, int, uintptr_t>, ChainProg> chain_progs;
   // per-kernel-class timing (fdllm_profile_enable)
   struct ProfPending {
     cudaEvent_t a, b;
@@ -486,6 +498,202 @@ int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg,
                   d, ep, n_part);
 }
 
+// ----------------------------------------------------- block-step chains
+bool chain_applicable(const fdllm_ctx* ctx, int M, int lm0, int n_lm) {
+  return ctx->tc && ctx->use_chain && ctx->weights_loaded && M >= 1 && M <= 32 && lm0 == 0 &&
+         n_lm == M && ctx->cfg.d_model % 512 == 0 && ctx->cfg.d_model <= CHAIN_NORM_GROUPS * 512;
+}
+
+// The phases of one block step over M rows with keys [0, L): launch 0 =
+// [EMBED_NORM, QKV_0]; launch l + 1 = [O_l, NORM, gate/up_l, down_l, NORM,
+// QKV_{l+1} or LM head].  The attention of layer l runs between launches l
+// and l + 1.
+int build_chain(fdllm_ctx* ctx, int M, int L, float* dbg, fdllm_ctx::ChainProg* out) {
+  const fdllm_config& c = ctx->cfg;
+  const int d = c.d_model, hq = c.n_heads * c.head_dim, hkv = c.n_kv_heads * c.head_dim;
+  const int nl = c.n_layers;
+  const CUtensorMap& amap_a = ctx->m_a[0];   // 64-row token tiles
+  const CUtensorMap& amap_o = ctx->m_o[0];
+  const CUtensorMap& amap_f = ctx->m_f[0];
+  const int G = ctx->num_sms;
+  const double es = 2.0;
+  std::vector<ChainPhase> ph;
+  fdllm_ctx::ChainProg pr;
+  int rot = 0;
+  double bytes = 0, flops = 0;
+  std::vector<std::pair<int, int>> chains;   // (first phase, phase count)
+  auto begin_chain = [&]() {
+    chains.push_back({(int)ph.size(), 0});
+    rot = 0;
+    bytes = flops = 0;
+  };
+  auto end_chain = [&]() {
+    chains.back().second = (int)ph.size() - chains.back().first;
+    pr.bytes.push_back(bytes);
+    pr.flops.push_back(flops);
+  };
+  auto norm = [&](int type, const float* gain) {
+    ChainPhase P{};
+    P.type = type;
+    P.gain = gain;
+    if (!ph.empty() && ph.back().type == CH_GEMM && ph.back().ep.kind == EPI_RESID)
+      P.resid_splits = ph.back().splits;
+    ph.push_back(P);
+    bytes += (double)M * d * (4.0 + 4.0 + 2.0 * es);
+  };
+  auto gemm = [&](const CUtensorMap& wmap, const CUtensorMap& amap, int N, int K, EpiParams ep,
+                  bool lm) -> bool {
+    // Split count: inside one launch a phase ends with its slowest CTA, so
+    // balance comes first: the largest per-CTA share of K blocks (units go
+    // round robin), plus a small charge per split for the partial tiles
+    // (residual GEMMs: read by the next norm) or for the last-arriver
+    // reduction (the other epilogues).
+    const int T = (N + 127) / 128, KB = (K + 63) / 64;
+    int best_s = 1;
+    double best = 1e300;
+    for (int sp = 1; sp <= (lm ? 1 : 16) && sp <= KB; ++sp) {
+      const long long units = (long long)T * sp;
+      if ((size_t)units * 32 * 128 * sizeof(float) > kWorkspaceBytes) break;
+      const double load = (double)((units + G - 1) / G) * ((KB + sp - 1) / sp);
+      const double cost = load + (ep.kind == EPI_RESID ? 0.25 * sp : (sp > 1 ? 4.0 : 0.0) + 0.5 * sp);
+      if (cost < best) {
+        best = cost;
+        best_s = sp;
+      }
+    }
+    if (T > ctx->n_counters) return false;
+    ChainPhase P{};
+    P.type = CH_GEMM;
+    P.N = N;
+    P.K = K;
+    P.kb_total = KB;
+    P.n_tiles = T;
+    P.splits = best_s;
+    P.units = T * best_s;
+    P.kc = 8;
+    P.rot = rot;
+    rot = (rot + P.units) % G;
+    P.wmap = wmap;
+    P.amap = amap;
+    ep.N = N;
+    ep.M = M;
+    ep.act_f32 = 0;
+    P.ep = ep;
+    ph.push_back(P);
+
+    double out_b = 0;
+    switch (ep.kind) {
+      case EPI_QKV: out_b = (double)M * N * es * 2; break;
+      case EPI_RESID: out_b = 2.0 * M * N * 4.0; break;
+      case EPI_SWIGLU: out_b = (double)M * (N / 2) * es * 2; break;
+      default: break;
+    }
+    bytes += (double)N * K * es + 2.0 * M * K * es + out_b;
+    flops += 2.0 * M * N * K;
+    return true;
+  };
+  auto qkv = [&](int l) {
+    EpiParams ep = epi_base(ctx, EPI_QKV);
+    ep.q_out = ctx->q;
+    ep.layer = l;
+    return gemm(ctx->layers[l].m_qkv, amap_a, hq + 2 * hkv, d, ep, false);
+  };
+  bool ok = true;
+  begin_chain();
+  norm(CH_EMBED_NORM, ctx->layers[0].attn_norm);
+  ok = ok && qkv(0);
+  end_chain();
+  for (int l = 0; l < nl && ok; ++l) {
+    LayerW& lw = ctx->layers[l];
+    begin_chain();
+    EpiParams ep = epi_base(ctx, EPI_RESID);
+    ep.h = ctx->h;
+    ok = ok && gemm(lw.m_o, amap_o, d, hq, ep, false);
+    norm(CH_NORM, lw.ffn_norm);
+    ep = epi_base(ctx, EPI_SWIGLU);
+    ep.f_out = ctx->f;
+    ok = ok && gemm(lw.m_gu, amap_a, 2 * c.ffn_dim, d, ep, false);
+    ep = epi_base(ctx, EPI_RESID);
+    ep.h = ctx->h;
+    ok = ok && gemm(lw.m_d, amap_f, d, c.ffn_dim, ep, false);
+    if (l + 1 < nl) {
+      norm(CH_NORM, ctx->layers[l + 1].attn_norm);
+      ok = ok && qkv(l + 1);
+    } else {
+      norm(CH_NORM, ctx->final_norm);
+      ep = epi_base(ctx, EPI_LMHEAD);
+      ep.lm_part = ctx->lm_part;
+      ep.dbg_logits = dbg;
+      ok = ok && gemm(ctx->m_head, amap_a, c.vocab, d, ep, true);
+    }
+    end_chain();
+  }
+  if (!ok) return fail(ctx, FDLLM_ERR_CUDA, "block-step chain: unexpected GEMM plan");
+  if ((size_t)G * M > ctx->lm_part_cap)
+    return fail(ctx, FDLLM_ERR_CUDA, "LM-head partial buffer too small");
+  pr.n_phases = (int)ph.size();
+  for (const auto& ch : chains) {
+    if (ch.second > CHAIN_MAX_PHASES) return fail(ctx, FDLLM_ERR_CUDA, "chain too long");
+    ChainArgs A{};
+    for (int i = 0; i < ch.second; ++i) A.ph[i] = ph[ch.first + i];
+    A.n_phases = ch.second;
+    A.M = M;
+    A.d = c.d_model;
+    A.vocab = c.vocab;
+    A.eps = c.rms_eps;
+    A.x = ctx->x;
+    A.embed = ctx->embed;
+    A.h = ctx->h;
+    A.a = ctx->a;
+    A.sp = ctx->sp;
+    A.sc = GemmScratch{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
+                       ctx->n_counters};
+    pr.launches.push_back(A);
+    pr.first.push_back(ch.first);
+  }
+  const int n_sync = (pr.n_phases + 1) * CHAIN_DONE_STRIDE;
+  if (n_sync > ctx->chain_sync_cap) {
+    ctx->chain_sync = (int*)dalloc(ctx, sizeof(int) * n_sync);
+    if (!ctx->chain_sync) return fail(ctx, FDLLM_ERR_OOM, "chain counter allocation failed");
+    ctx->chain_sync_cap = n_sync;
+  }
+  *out = pr;
+  return FDLLM_OK;
+}
+
+// One block step (rows [sp->r0, sp->r0 + M), keys [0, L)) through the chain
+// kernel: n_layers + 1 chain launches with the attention launches between
+// them.  The LM partials come from every CTA of the grid.
+int forward_chain(fdllm_ctx* ctx, int M, int L, float* dbg, int* n_part) {
+  const auto key = std::make_tuple(M, L, (uintptr_t)dbg);
+  auto it = ctx->chain_progs.find(key);
+  if (it == ctx->chain_progs.end()) {
+    fdllm_ctx::ChainProg pr;
+    int rc = build_chain(ctx, M, L, dbg, &pr);
+    if (rc) return rc;
+    it = ctx->chain_progs.emplace(key, pr).first;
+  }
+  const fdllm_ctx::ChainProg& pr = it->second;
+  const fdllm_config& c = ctx->cfg;
+  CK(cudaMemsetAsync(ctx->chain_sync, 0, sizeof(int) * (pr.n_phases + 1) * CHAIN_DONE_STRIDE,
+                     ctx->stream));
+  for (size_t ci = 0; ci < pr.launches.size(); ++ci) {
+    ChainArgs A = pr.launches[ci];
+    A.done = ctx->chain_sync + pr.first[ci] * CHAIN_DONE_STRIDE;
+    A.gabort = ctx->chain_sync + pr.n_phases * CHAIN_DONE_STRIDE;
+    {
+      ProfScope ps(ctx, "chain.step", pr.bytes[ci], pr.flops[ci]);
+      KL(launch_chain(A, ctx->num_sms, ctx->stream));
+    }
+    if ((int)ci < c.n_layers) {
+      int rc = run_attention(ctx, (int)ci, M, L);
+      if (rc) return rc;
+    }
+  }
+  *n_part = ctx->num_sms;
+  return FDLLM_OK;
+}
+
 int sync_state(fdllm_ctx* ctx) {
   CK(cudaMemcpyAsync(ctx->state_host, ctx->state, sizeof(DecodeState), cudaMemcpyDeviceToHost,
                      ctx->stream));
@@ -535,7 +743,8 @@ int set_step_params(fdllm_ctx* ctx, int r0, int lm0, int s, float tau) {
 // from the step scalars) and the merge/select kernel.
 int enqueue_step(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int B, float tau, float* dbg,
                  int* n_part) {
-  int rc = forward(ctx, r0, M, L, lm0, B, dbg, n_part);
+  int rc = chain_applicable(ctx, M, lm0, B) ? forward_chain(ctx, M, L, dbg, n_part)
+                                            : forward(ctx, r0, M, L, lm0, B, dbg, n_part);
   if (rc) return rc;
   ProfScope ps(ctx, "merge_select", (double)*n_part * B * 12.0, 0.0);
   KL(launch_merge_select(ctx->lm_part, *n_part, B, ctx->x, 0, ctx->cfg.mask_id, tau, 1, ctx->conf,
@@ -765,6 +974,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
     ctx->custom_alloc = true;
   }
   ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
+  if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {
@@ -1047,6 +1257,7 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
   }
   if (ctx->tc && !make_map(ctx, &ctx->m_head, ctx->lm_head, V, d, 128))
     return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for lm_head");
+
   CK(cudaDeviceSynchronize());
   {
     int e = 0;

@@ -426,6 +426,7 @@ cudaError_t init_kernel_attributes() {
   if (e == cudaSuccess) e = set_attr<128, 2>();
   if (e == cudaSuccess) e = set_attr<128, 4>();
   if (e == cudaSuccess) e = gemm_tc_init_attributes();
+  if (e == cudaSuccess) e = chain_init_attributes();
   return e;
 }
 

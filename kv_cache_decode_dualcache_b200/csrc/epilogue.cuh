@@ -212,12 +212,13 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
       break;
     }
     case EPI_RESID: {
-      // all loads of h before any store (see epi_chunk)
+      // all loads of h before any store (see epi_chunk); through L2, since
+      // in the chain kernel other SMs wrote h earlier in the same launch
       if (n >= ep.N) break;
       float hv[CHUNK_T];
 #pragma unroll
       for (int t = 0; t < CHUNK_T; ++t)
-        hv[t] = (t < nt) ? ep.h[(size_t)(t0 + t) * ep.N + n] : 0.0f;
+        hv[t] = (t < nt) ? __ldcg(ep.h + (size_t)(t0 + t) * ep.N + n) : 0.0f;
 #pragma unroll
       for (int t = 0; t < CHUNK_T; ++t) {
         if (t >= nt) break;
@@ -312,6 +313,125 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
     default:
       break;
   }
+}
+
+}  // namespace fd
+
+namespace fd {
+
+// epi_regs for the QKV and SwiGLU epilogues, with the two-term fp16 output
+// staged in shared memory and written back as 16-byte stores: a thread
+// stores 8 chunks of 16 bytes per tile instead of 64 scattered 2-byte
+// values, and those narrow stores are what limits an SM's epilogue (each
+// store instruction waits for write credits toward L2).  Called by the 128
+// threads of one warpgroup, which sync on named barrier `bar`; st is 16 KB
+// of shared memory that the caller does not use until the call returns.
+// v[t] = output feature n0 + e of token row t0 + t (see epi_regs).
+FD_DEV void epi_staged_f16(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0, int e,
+                           __half* st, int bar) {
+  const int lane = e & 31;
+  const int n = n0 + e;
+  const int nt = min(CHUNK_T, ep.M - t0);
+  if (nt <= 0) return;
+  __half* st_hi = st;                 // [32 tokens][128 features]
+  __half* st_lo = st + CHUNK_T * 128;
+  if (ep.kind == EPI_SWIGLU) {
+    // 64 outputs per tile: feature j0 + f, f = 16 * (e / 32) + lane % 16
+    const int F = ep.N / 2;
+    const bool up = lane >= 16;
+    const int f = 16 * (e >> 5) + (lane & 15);
+#pragma unroll
+    for (int t = 0; t < CHUNK_T; ++t) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[t], 16);
+      const float g = up ? p : v[t];
+      const float u = up ? v[t] : p;
+      __half hi, lo;
+      split_f16(silu_f(g) * u, hi, lo);
+      if (!up) st_hi[t * 128 + f] = hi;
+      else st_lo[t * 128 + f] = lo;
+    }
+    named_bar(bar, EPI_THREADS);
+    // rows: 32 tokens x {hi, lo}; 64 features = 8 chunks of 8 per row
+    const int j0 = n0 / 2;  // 64 FFN features per 128-row tile
+    __half* fo = reinterpret_cast<__half*>(ep.f_out);
+    for (int c = e; c < CHUNK_T * 2 * 8; c += EPI_THREADS) {
+      const int t = c >> 4, term = (c >> 3) & 1, ch = c & 7;
+      if (t >= nt || n0 >= ep.N) continue;
+      const __half* src = (term ? st_lo : st_hi) + t * 128 + ch * 8;
+      const size_t i = ((size_t)pair_row(t0 + t) + (term ? PAIR_LO : 0)) * F + j0 + ch * 8;
+      if (FD_CHECK(i + 7 < ep.cap_f, ep.check, 3, i, ep.cap_f))
+        *reinterpret_cast<uint4*>(fo + i) = *reinterpret_cast<const uint4*>(src);
+    }
+    named_bar(bar, EPI_THREADS);
+    return;
+  }
+  // EPI_QKV: the tile is 128 / hd heads of one region (q, k or v); N and the
+  // region bounds are multiples of 64, so a warp is wholly inside or outside
+  const int hd = ep.head_dim, half = hd / 2;
+  const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
+  const bool valid = n < ep.N;
+  const int region = n0 < hq ? 0 : (n0 < hq + hk ? 1 : 2);
+  const int rbase = region == 0 ? 0 : (region == 1 ? hq : hq + hk);
+  const int rn = n - rbase;
+  const int head = rn / hd;
+  const int r = rn - head * hd;
+  const int dim = region < 2 ? rope_slab_dim(r, hd) : r;
+  const int col = (head - (n0 - rbase) / hd) * hd + dim;  // natural column within the tile
+  const int pos0 = (ep.sp ? ep.sp->r0 : ep.pos0) + t0;
+  const bool second = lane >= 16;
+  if (valid) {
+#pragma unroll
+    for (int h16 = 0; h16 < CHUNK_T; h16 += 16) {
+      float2 cs[16];
+      if (region < 2) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          cs[t] = (h16 + t < nt) ? __ldg(&ep.rope[(size_t)(pos0 + h16 + t) * half + (dim % half)])
+                                 : make_float2(1.0f, 0.0f);
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        float y = v[h16 + t];
+        if (region < 2) {
+          const float p = __shfl_xor_sync(0xffffffffu, y, 16);
+          y = second ? (y * cs[t].x + p * cs[t].y) : (y * cs[t].x - p * cs[t].y);
+        }
+        __half hi, lo;
+        split_f16(y, hi, lo);
+        st_hi[(h16 + t) * 128 + col] = hi;
+        st_lo[(h16 + t) * 128 + col] = lo;
+      }
+    }
+  }
+  named_bar(bar, EPI_THREADS);
+  {
+    const int head0 = (n0 - rbase) / hd;  // first head of the tile
+    const int pg0 = region > 0 ? __ldg(&ep.page_table[pos0 / KV_PAGE]) : 0;
+    const int pg1 = region > 0 ? __ldg(&ep.page_table[(pos0 + nt - 1) / KV_PAGE]) : 0;
+    // 32 tokens x 2 terms x 16 chunks of 8 features
+    for (int c = e; c < CHUNK_T * 2 * 16; c += EPI_THREADS) {
+      const int t = c >> 5, term = (c >> 4) & 1, ch = c & 15;
+      if (t >= nt || n0 + ch * 8 >= ep.N) continue;
+      const uint4 val = *reinterpret_cast<const uint4*>((term ? st_lo : st_hi) + t * 128 + ch * 8);
+      const int cf = ch * 8;                 // natural column within the tile
+      const int hh = head0 + cf / hd, dd = cf % hd;
+      if (region == 0) {
+        __half* q = reinterpret_cast<__half*>(ep.q_out);
+        const size_t i = (size_t)(t0 + t) * hq + (size_t)hh * hd + dd + (term ? ep.q_plane : 0);
+        if (FD_CHECK(i + 7 < ep.cap_q, ep.check, 4, i, ep.cap_q))
+          *reinterpret_cast<uint4*>(q + i) = val;
+      } else {
+        const int pos = pos0 + t;
+        const int page = (pos / KV_PAGE == pos0 / KV_PAGE) ? pg0 : pg1;
+        const int plane = (region == 1 ? 0 : 2) + term;
+        __half* kv = reinterpret_cast<__half*>(ep.kv_pool);
+        const size_t i = kv_offset_pg(ep, page, pos, plane, hh, dd);
+        if (FD_CHECK(i + 7 < ep.cap_kv, ep.check, 5, i, ep.cap_kv))
+          *reinterpret_cast<uint4*>(kv + i) = val;
+      }
+    }
+  }
+  named_bar(bar, EPI_THREADS);
 }
 
 }  // namespace fd

@@ -276,6 +276,16 @@ __global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
       const int n0 = c.tile * 128;
       const int tile_id = c.tile * gs.n_tt + c.tt;
       const int tg0 = c.tt * TOK + grp * GT;  // first token row of this warpgroup
+      if (lmhead || gs.splits > 1) {
+        // the paths below have named barriers: agree on `got` first (one
+        // thread samples the flags), so a failed wait in one thread cannot
+        // leave the others at a barrier
+        if (!got) *abort_flag = 1;
+        named_bar(1, EPI_ALL);
+        if (threadIdx.x == 64) misc[3] = *abort_flag == 0;
+        named_bar(1, EPI_ALL);
+        got = misc[3] != 0;
+      }
       bool run_epi = gs.splits == 1;
       if (gs.splits > 1) {
         // float partial tile [TOK][128] of this split; the last split to

@@ -163,6 +163,56 @@ cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float
                            void* a, int f32, const StepParams* sp, bool rows_from_lm0,
                            cudaStream_t st, bool pdl = false);
 
+// ------------------------------------------------ block-step chain kernel
+// One launch runs a program of phases of the DualCache block step (bf16
+// model, at most 32 block tokens), see chain.cu.
+enum ChainPhaseType : int {
+  CH_GEMM = 0,        // tcgen05 GEMM, one token tile, fused epilogue ep
+  CH_NORM = 1,        // a = RMSNorm(h) * gain over the block rows
+  CH_EMBED_NORM = 2,  // h = E[x[r0 + row]], then as CH_NORM
+};
+constexpr int CHAIN_NORM_GROUPS = 8;  // d_model: a multiple of 512, at most 8 * 512
+constexpr int CHAIN_DONE_STRIDE = 32;  // ints between phase counters (one 128-byte line each)
+
+constexpr int CHAIN_MAX_PHASES = 6;
+
+struct ChainPhase {
+  CUtensorMap wmap;         // weight map (GEMM)
+  CUtensorMap amap;         // activation map, 64-row token tile (GEMM)
+  int type;
+  int N, K, kb_total, n_tiles, splits, units, rot, kc;
+  const float* gain;        // norm gains (NORM, EMBED_NORM)
+  int resid_splits;         // NORM: split partials of the preceding residual GEMM to add
+                            // into h first (its EPI_RESID epilogue only stores partials)
+  EpiParams ep;             // GEMM epilogue (ep.M = block rows)
+};
+
+// Passed by value (kernel parameter space: read-only, so the compiler never
+// has to re-read a phase field after the kernel's own global stores); larger
+// than the classic 4 KB parameter limit, which CUDA 12.1+ lifts to 32 KB.
+struct ChainArgs {
+  ChainPhase ph[CHAIN_MAX_PHASES];
+  int n_phases;
+  int* done;                // CTAs finished per phase, phase p at done[p * CHAIN_DONE_STRIDE];
+                            // zero at launch
+  int* gabort;              // grid-wide abort word; zero at launch
+  int M;                    // block rows (<= 32)
+  int d, vocab;
+  float eps;
+  const int* x;             // token ids (EMBED_NORM: rows x[sp->r0 + row])
+  const void* embed;        // bf16 [vocab, d]
+  float* h;                 // residual stream [M, d]
+  void* a;                  // normed activations, two-term fp16 pair rows
+  const StepParams* sp;
+  GemmScratch sc;           // split-K partials and per-tile counters
+};
+static_assert(sizeof(ChainArgs) <= 32764, "kernel parameters are limited to 32 KB");
+
+// Cooperative launch of grid CTAs (one per SM).
+cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st);
+cudaError_t chain_init_attributes();
+int chain_smem_bytes();
+
 struct DecodeState {
   int remaining;     // masked positions left in the block after the step
   int unmasked;      // positions unmasked by the step
