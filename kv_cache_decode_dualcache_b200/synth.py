@@ -105,6 +105,16 @@ WORKLOADS = {
 }
 
 
+def step_weight_params(shape: ModelShape) -> int:
+    """Weights a DualCache block step reads: every layer's QKV, O, gate, up
+    and down matrices and the LM head (the embedding only for the block's
+    rows, negligible)."""
+    d, hd = shape.d_model, shape.head_dim
+    per_layer = (d * (shape.n_heads + 2 * shape.n_kv_heads) * hd + shape.n_heads * hd * d
+                 + 3 * d * shape.ffn_dim)
+    return shape.n_layers * per_layer + shape.vocab * d
+
+
 def weight_names(shape: ModelShape) -> List[str]:
     names = ["embed"]
     for i in range(shape.n_layers):
