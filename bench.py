@@ -30,6 +30,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "gen tokens/s (LLaDA-8B shape, DualCache, tau=0.9)"
+
+
+def metric_name(wl):
+    if wl.name == WORKLOAD and wl.tau == 0.9 and wl.cache_mode == "dual":
+        return METRIC
+    return f"gen tokens/s ({wl.name}, {wl.cache_mode}, tau={wl.tau})"
 WORKLOAD = "llada8b-p256-g256"
 
 
@@ -47,7 +53,7 @@ def _config(wl, n):
     return {"workload": wl.name, "model_shape": wl.shape.name, "prompt_len": wl.prompt_len,
             "gen_len": wl.gen_len, "block_size": wl.block_size, "tau": wl.tau,
             "cache_mode": wl.cache_mode, "batch_per_gpu": 1, "global_batch": n,
-            "weights": "random N(0,0.02) bf16, seed 1",
+            "weights": f"random N(0,0.02) bf16, seed {wl.shape.seed}",
             "l2": "no flush needed: each step streams ~16 GB of weights (> 126 MB L2)",
             "parallelism": "replicas" if n > 1 else "single"}
 
@@ -233,7 +239,7 @@ def run_reference(args, wl):
         if i >= args.warmup:
             vals.append(r)
     v = sum(r["tok_s"] for r in vals) / len(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+    line = {"impl": "reference", "metric": metric_name(wl), "value": v, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * wl.gen_len / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -366,7 +372,7 @@ def run_fdllm(args, wl):
                "t_refresh_s": round(r["t_refresh_s"], 3), "t_step_s": round(r["t_step_s"], 3)}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -376,8 +382,9 @@ def run_fdllm(args, wl):
                            "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
                            "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3),
                            "tokens_checksum": int(np.asarray(tokens, dtype=np.int64).sum())},
-                "block_step_roofline": block_step_roofline(
-                    wl, timing.cached_ms / max(1, timing.cached_steps), hbm),
+                "block_step_roofline": (block_step_roofline(
+                    wl, timing.cached_ms / timing.cached_steps, hbm)
+                    if timing.cached_steps else None),   # cache off: every step is a refresh
                 "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches,
@@ -397,13 +404,22 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fdllm", choices=["fdllm", "reference"])
-    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="another configuration of the same decoder (synth.WORKLOADS), "
+                         "e.g. llada8b-p1024-g1024, dream7b-p512-g512")
+    ap.add_argument("--tau", type=float, default=None, help="override the workload's tau")
+    ap.add_argument("--cache-mode", default=None, choices=["none", "prefix", "dual"],
+                    help="override the workload's cache mode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-cached-steps", type=int, default=18,
                     help="cached steps per generation assumed by the reference arm")
     args = ap.parse_args()
     from kv_cache_decode_dualcache_b200 import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.tau is not None or args.cache_mode is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, tau=wl.tau if args.tau is None else args.tau,
+                                 cache_mode=args.cache_mode or wl.cache_mode)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_fdllm(args, wl)

@@ -91,6 +91,8 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", TINY, 32, 64, 16, 0.9, "dual"),
     "llada8b-p256-g256": Workload("llada8b-p256-g256", LLADA_8B, 256, 256, 32, 0.9, "dual"),
+    "llada8b-p1024-g256": Workload("llada8b-p1024-g256", LLADA_8B, 1024, 256, 32, 0.9, "dual"),
+    "llada8b-p1024-g512": Workload("llada8b-p1024-g512", LLADA_8B, 1024, 512, 32, 0.9, "dual"),
     "llada8b-p1024-g1024": Workload("llada8b-p1024-g1024", LLADA_8B, 1024, 1024, 32, 0.9, "dual"),
     "dream7b-p512-g512": Workload("dream7b-p512-g512", DREAM_7B, 512, 512, 32, 0.9, "dual"),
     "llada8b-batch16": Workload("llada8b-batch16", LLADA_8B, 0, 256, 32, 0.9, "dual", batch=16),
