@@ -132,6 +132,7 @@ struct fdllm_ctx {
   bool use_chain = true;
   int* chain_sync = nullptr;        // per-phase done counters of one step, then the abort word
   int chain_sync_cap = 0;
+  float* norm_ss = nullptr;         // chain NORM phases: partial sums of squares [32][8]
   struct ChainProg {
     std::vector<ChainArgs> launches;           // kernel arguments per launch
     std::vector<int> first;                    // index of each launch's first phase in the step
@@ -536,6 +537,8 @@ int build_chain(fdllm_ctx* ctx, int M, int L, float* dbg, fdllm_ctx::ChainProg* 
     ChainPhase P{};
     P.type = type;
     P.gain = gain;
+    P.rot = rot;
+    rot = (rot + M * (d / 512)) % G;
     if (!ph.empty() && ph.back().type == CH_GEMM && ph.back().ep.kind == EPI_RESID)
       P.resid_splits = ph.back().splits;
     ph.push_back(P);
@@ -651,11 +654,16 @@ int build_chain(fdllm_ctx* ctx, int M, int L, float* dbg, fdllm_ctx::ChainProg* 
     pr.launches.push_back(A);
     pr.first.push_back(ch.first);
   }
-  const int n_sync = (pr.n_phases + 1) * CHAIN_DONE_STRIDE;
+  const int n_sync = (pr.n_phases + 1) * CHAIN_DONE_STRIDE + pr.n_phases * 32 +
+                     pr.n_phases * CHAIN_DONE_STRIDE;
   if (n_sync > ctx->chain_sync_cap) {
     ctx->chain_sync = (int*)dalloc(ctx, sizeof(int) * n_sync);
     if (!ctx->chain_sync) return fail(ctx, FDLLM_ERR_OOM, "chain counter allocation failed");
     ctx->chain_sync_cap = n_sync;
+  }
+  if (!ctx->norm_ss) {
+    ctx->norm_ss = (float*)dalloc(ctx, sizeof(float) * 32 * CHAIN_NORM_GROUPS);
+    if (!ctx->norm_ss) return fail(ctx, FDLLM_ERR_OOM, "chain norm scratch allocation failed");
   }
   *out = pr;
   return FDLLM_OK;
@@ -675,12 +683,18 @@ int forward_chain(fdllm_ctx* ctx, int M, int L, float* dbg, int* n_part) {
   }
   const fdllm_ctx::ChainProg& pr = it->second;
   const fdllm_config& c = ctx->cfg;
-  CK(cudaMemsetAsync(ctx->chain_sync, 0, sizeof(int) * (pr.n_phases + 1) * CHAIN_DONE_STRIDE,
-                     ctx->stream));
+  // counters of one step: [done per phase, abort word][NORM row counters][unit claims]
+  const int rowcnt0 = (pr.n_phases + 1) * CHAIN_DONE_STRIDE;
+  const int next0 = rowcnt0 + pr.n_phases * 32;
+  CK(cudaMemsetAsync(ctx->chain_sync, 0,
+                     sizeof(int) * (next0 + pr.n_phases * CHAIN_DONE_STRIDE), ctx->stream));
   for (size_t ci = 0; ci < pr.launches.size(); ++ci) {
     ChainArgs A = pr.launches[ci];
     A.done = ctx->chain_sync + pr.first[ci] * CHAIN_DONE_STRIDE;
     A.gabort = ctx->chain_sync + pr.n_phases * CHAIN_DONE_STRIDE;
+    A.rowcnt = ctx->chain_sync + rowcnt0 + pr.first[ci] * 32;
+    A.norm_ss = ctx->norm_ss;
+    A.next = ctx->chain_sync + next0 + pr.first[ci] * CHAIN_DONE_STRIDE;
     {
       ProfScope ps(ctx, "chain.step", pr.bytes[ci], pr.flops[ci]);
       KL(launch_chain(A, ctx->num_sms, ctx->stream));

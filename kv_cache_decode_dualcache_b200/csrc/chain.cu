@@ -35,6 +35,8 @@
 // owner and MMA issuer, warp 2 = activation (B) producer, warps 3..6 =
 // workers (TMEM lane quadrant = warp % 4): accumulator drain and epilogue,
 // norms.
+#include <climits>
+
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -58,9 +60,11 @@ constexpr int TILE_OFF = B_OFF + STAGES * B_BYTES;       // [32][128] float (LM 
 constexpr int RED_OFF = TILE_OFF + CHUNK_T * 128 * 4;    // norm reduction (4 floats)
 constexpr int LM_OFF = RED_OFF + 64;                     // [TOK] softmax states
 constexpr int BAR_OFF = LM_OFF + TOK * (int)sizeof(SoftmaxState);
-constexpr int N_BARS = 3 * STAGES + 2 * NBUF + 1;
+constexpr int UQ = 16;                   // unit queue entries (weight producer -> other roles)
+constexpr int N_BARS = 3 * STAGES + 2 * NBUF + 1 + 2 * UQ;
 constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
-constexpr int PH_OFF = (MISC_OFF + 16 + 127) / 128 * 128;  // workers' copy of the current phase
+constexpr int UQ_OFF = MISC_OFF + 16;  // [UQ] unit ids, then the workers' broadcast word
+constexpr int PH_OFF = (UQ_OFF + (UQ + 1) * 4 + 127) / 128 * 128;  // workers' copy of the phase
 constexpr int SMEM = PH_OFF + (int)sizeof(ChainPhase) + 1024;
 static_assert(SMEM <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
 static_assert(BAR_OFF % 8 == 0, "mbarriers need 8-byte alignment");
@@ -138,95 +142,110 @@ FD_DEV void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// a[row] = RMSNorm(h[row]) * g as two-term fp16 pair rows; 128 threads, one
-// row, 4 consecutive features per thread and 512-feature group (d a
-// multiple of 512, at most CHAIN_NORM_GROUPS groups).  With EMBED_NORM,
-// h[row] is first gathered from the bf16 embedding table; with
-// resid_splits, the preceding residual GEMM's split partials are first
-// added into h (in split order) and the row stored back.  Every load of a
-// round is issued before its first use.
-FD_DEV void norm_row(const ChainArgs& A, const ChainPhase& P, int row, float* red, int wt) {
+// NORM / EMBED_NORM phase: a[row] = RMSNorm(h[row]) * g as two-term fp16
+// pair rows, spread over every CTA.  Work items are (row, 512-feature group)
+// pairs, item i on CTA (i + rot) % G; a worker thread owns 4 consecutive
+// features of an item.  First every item of the CTA loads its features
+// (EMBED_NORM: gathers them from the bf16 embedding table; NORM with
+// resid_splits: adds the preceding residual GEMM's split partials, in split
+// order, and stores h back), all loads of an item in flight at once, and
+// publishes its partial sum of squares (ss[row][group], then one arrival on
+// the row's counter).  Only then does any item wait for its row's other
+// groups, so no CTA can wait on an item that waits on it.  The row total
+// sums the groups in group order.
+constexpr int NORM_MAX_ITEMS = 4;   // per CTA: M * (d / 512) <= 4 * gridDim.x
+constexpr int NORM_MAX_SPLITS = 16;
+
+FD_DEV bool norm_phase(const ChainArgs& A, const ChainPhase& P, int p, int cta, int G, int wt,
+                       float* red, volatile int* flag, int* err) {
   const int d = A.d;
-  const int ng = d >> 9;  // 512-feature groups
-  float* hr = A.h + (size_t)row * d;
-  float4 v[CHAIN_NORM_GROUPS];
-  if (P.type == CH_EMBED_NORM) {
-    const int r0 = A.sp ? A.sp->r0 : 0;
-    int tok = A.x[r0 + row];
-    if (tok < 0 || tok >= A.vocab) {
-      if (wt == 0) atomicOr(A.sc.err, DEV_ERR_TOKEN);
-      tok = 0;
-    }
-    const __nv_bfloat16* er = reinterpret_cast<const __nv_bfloat16*>(A.embed) + (size_t)tok * d;
-    uint2 raw[CHAIN_NORM_GROUPS];
-#pragma unroll
-    for (int g = 0; g < CHAIN_NORM_GROUPS; ++g)
-      if (g < ng) raw[g] = __ldg(reinterpret_cast<const uint2*>(er + g * 512 + wt * 4));
-#pragma unroll
-    for (int g = 0; g < CHAIN_NORM_GROUPS; ++g) {
-      if (g >= ng) break;
-      const __nv_bfloat162 lo2 = *reinterpret_cast<const __nv_bfloat162*>(&raw[g].x);
-      const __nv_bfloat162 hi2 = *reinterpret_cast<const __nv_bfloat162*>(&raw[g].y);
-      v[g] = make_float4(__low2float(lo2), __high2float(lo2), __low2float(hi2), __high2float(hi2));
-      *reinterpret_cast<float4*>(hr + g * 512 + wt * 4) = v[g];
-    }
-  } else {
-#pragma unroll
-    for (int g = 0; g < CHAIN_NORM_GROUPS; ++g)
-      if (g < ng) v[g] = __ldcg(reinterpret_cast<const float4*>(hr + g * 512 + wt * 4));
-    const int S = P.resid_splits;
-    if (S > 0) {
+  const int ng = d >> 9;
+  const int n_items = A.M * ng;
+  const bool leader = wt == 0;
+  int* rowcnt = A.rowcnt + p * 32;
+  int first = (cta - P.rot) % G;
+  if (first < 0) first += G;
+  float4 v[NORM_MAX_ITEMS];
+  // ---- load, partial sum of squares, publish
+  int k = 0;
+  for (int item = first; item < n_items && k < NORM_MAX_ITEMS; item += G, ++k) {
+    const int row = item / ng, g = item - row * ng;
+    const int j = g * 512 + wt * 4;
+    float* hj = A.h + (size_t)row * d + j;
+    float4 x;
+    if (P.type == CH_EMBED_NORM) {
+      const int r0 = A.sp ? A.sp->r0 : 0;
+      int tok = A.x[r0 + row];
+      if (tok < 0 || tok >= A.vocab) {
+        if (leader) atomicOr(err, DEV_ERR_TOKEN);
+        tok = 0;
+      }
+      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+          reinterpret_cast<const __nv_bfloat16*>(A.embed) + (size_t)tok * d + j));
+      const __nv_bfloat162 lo2 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+      const __nv_bfloat162 hi2 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+      x = make_float4(__low2float(lo2), __high2float(lo2), __low2float(hi2), __high2float(hi2));
+      *reinterpret_cast<float4*>(hj) = x;
+    } else {
+      const int S = P.resid_splits;
       // partial tiles [tile][split][token][128]; feature j lies in tile j / 128
-      for (int sp = 0; sp < S; ++sp) {
-        float4 pv[CHAIN_NORM_GROUPS];
+      const float* pp = A.sc.ws + (((size_t)(j >> 7) * S) * TOK + row) * 128 + (j & 127);
+      float4 pv[NORM_MAX_SPLITS];
+      x = __ldcg(reinterpret_cast<const float4*>(hj));
 #pragma unroll
-        for (int g = 0; g < CHAIN_NORM_GROUPS; ++g) {
-          if (g >= ng) break;
-          const int j = g * 512 + wt * 4;
-          pv[g] = __ldcg(reinterpret_cast<const float4*>(
-              A.sc.ws + (((size_t)(j >> 7) * S + sp) * TOK + row) * 128 + (j & 127)));
-        }
+      for (int sp = 0; sp < NORM_MAX_SPLITS; ++sp)
+        if (sp < S) pv[sp] = __ldcg(reinterpret_cast<const float4*>(pp + (size_t)sp * TOK * 128));
 #pragma unroll
-        for (int g = 0; g < CHAIN_NORM_GROUPS; ++g) {
-          if (g >= ng) break;
-          v[g].x += pv[g].x;
-          v[g].y += pv[g].y;
-          v[g].z += pv[g].z;
-          v[g].w += pv[g].w;
+      for (int sp = 0; sp < NORM_MAX_SPLITS; ++sp) {
+        if (sp < S) {
+          x.x += pv[sp].x;
+          x.y += pv[sp].y;
+          x.z += pv[sp].z;
+          x.w += pv[sp].w;
         }
       }
-#pragma unroll
-      for (int g = 0; g < CHAIN_NORM_GROUPS; ++g)
-        if (g < ng) *reinterpret_cast<float4*>(hr + g * 512 + wt * 4) = v[g];
+      if (S > 0) *reinterpret_cast<float4*>(hj) = x;
+    }
+    v[k] = x;
+    float ss = warp_sum(x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w);
+    named_bar(2, WORKERS);  // red is free
+    if ((wt & 31) == 0) red[wt >> 5] = ss;
+    named_bar(2, WORKERS);
+    if (leader) {
+      A.norm_ss[row * CHAIN_NORM_GROUPS + g] = (red[0] + red[1]) + (red[2] + red[3]);
+      fence_acq_rel_gpu();
+      atomicAdd(rowcnt + row, 1);
     }
   }
-  float ss = 0.0f;
-#pragma unroll
-  for (int g = 0; g < CHAIN_NORM_GROUPS; ++g)
-    if (g < ng) ss += v[g].x * v[g].x + v[g].y * v[g].y + v[g].z * v[g].z + v[g].w * v[g].w;
-  ss = warp_sum(ss);
-  named_bar(2, WORKERS);  // red is free (previous row done with it)
-  if ((wt & 31) == 0) red[wt >> 5] = ss;
-  named_bar(2, WORKERS);
-  const float tot = (red[0] + red[1]) + (red[2] + red[3]);
-  const float inv = 1.0f / sqrtf(tot / (float)d + A.eps);
-  __half* ab = reinterpret_cast<__half*>(A.a);
-  const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
-#pragma unroll
-  for (int g = 0; g < CHAIN_NORM_GROUPS; ++g) {
-    if (g >= ng) break;
+  // ---- per item: wait for the row's groups, normalise, store
+  bool ok = true;
+  k = 0;
+  for (int item = first; item < n_items && k < NORM_MAX_ITEMS; item += G, ++k) {
+    const int row = item / ng, g = item - row * ng;
     const int j = g * 512 + wt * 4;
+    if (leader) *flag = grid_wait(rowcnt + row, ng, err, A.gabort) ? 1 : 0;
+    named_bar(2, WORKERS);
+    ok = *flag != 0;
+    named_bar(2, WORKERS);
+    if (!ok) break;
+    float tot = 0.0f;
+    for (int q = 0; q < ng; ++q) tot += __ldcg(A.norm_ss + row * CHAIN_NORM_GROUPS + q);
+    const float inv = 1.0f / sqrtf(tot / (float)d + A.eps);
     const float4 gn = __ldg(reinterpret_cast<const float4*>(P.gain + j));
+    const float4 x = v[k];
     __half h0, l0, h1, l1, h2, l2, h3, l3;
-    split_f16(v[g].x * inv * gn.x, h0, l0);
-    split_f16(v[g].y * inv * gn.y, h1, l1);
-    split_f16(v[g].z * inv * gn.z, h2, l2);
-    split_f16(v[g].w * inv * gn.w, h3, l3);
+    split_f16(x.x * inv * gn.x, h0, l0);
+    split_f16(x.y * inv * gn.y, h1, l1);
+    split_f16(x.z * inv * gn.z, h2, l2);
+    split_f16(x.w * inv * gn.w, h3, l3);
     __half2 hh[2] = {__halves2half2(h0, h1), __halves2half2(h2, h3)};
     __half2 ll[2] = {__halves2half2(l0, l1), __halves2half2(l2, l3)};
+    __half* ab = reinterpret_cast<__half*>(A.a);
+    const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
     *reinterpret_cast<uint2*>(ab + r_hi + j) = *reinterpret_cast<const uint2*>(hh);
     *reinterpret_cast<uint2*>(ab + r_lo + j) = *reinterpret_cast<const uint2*>(ll);
   }
+  return ok;
 }
 
 __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant__ ChainArgs A) {
@@ -245,6 +264,9 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
   uint64_t* acc_full = bars + 3 * STAGES;
   uint64_t* acc_empty = bars + 3 * STAGES + NBUF;
   uint64_t* mma_done = bars + 3 * STAGES + 2 * NBUF;
+  uint64_t* uq_full = mma_done + 1;
+  uint64_t* uq_empty = uq_full + UQ;
+  volatile int* uq = reinterpret_cast<volatile int*>(smem + UQ_OFF);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
   ChainPhase* sph = reinterpret_cast<ChainPhase*>(smem + PH_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -267,6 +289,10 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
       mbar_init(&acc_empty[i], WORKERS);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < UQ; ++i) {
+      mbar_init(&uq_full[i], 1);
+      mbar_init(&uq_empty[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -279,17 +305,37 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------- weight (A) producer
-      uint32_t it = 0;
+      // Also the unit scheduler: it claims each GEMM phase's units (from the
+      // phase's global counter, so CTAs that stream faster take more units;
+      // the LM head keeps its static round-robin assignment, since the
+      // merge of its per-CTA softmax states must not depend on timing) and
+      // queues each unit id, then -1 at the phase end, for the other roles.
+      uint32_t it = 0, qi = 0;
       bool ok = true;
       const uint64_t stream_once = make_policy_evict_first();
+      auto push = [&](int u) -> bool {
+        const int slot = qi % UQ;
+        if (!mbar_wait(&uq_empty[slot], ((qi / UQ) & 1u) ^ 1u, err, abort_flag)) return false;
+        uq[slot] = u;
+        mbar_arrive(&uq_full[slot]);  // release: the write above is visible to its waiters
+        ++qi;
+        return true;
+      };
       for (int p = 0; p < A.n_phases && ok; ++p) {
         const Geom P = geom_of(A.ph[p]);
         if (P.type != CH_GEMM) continue;
+        const bool dyn = A.ph[p].ep.kind != EPI_LMHEAD;
+        int* next = A.next + p * CHAIN_DONE_STRIDE;
         const CUtensorMap* wmap = &A.ph[p].wmap;
         tma_prefetch_desc(wmap);
-        for (int u = first_unit(P, cta, G); u < P.units && ok; u += G) {
+        int u = dyn ? atomicAdd(next, 1) : first_unit(P, cta, G);
+        while (u < P.units && ok) {
+          if (!push(u)) { ok = false; break; }
           const Unit c = unit_of(P, u);
+          int u_next = P.units;
           for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
+            // claim the next unit while this unit's last stages are in flight
+            if (kb == c.kb_hi - 1) u_next = dyn ? atomicAdd(next, 1) : u + G;
             const int s = it % STAGES;
             if (!mbar_wait(&empty[s], ((it / STAGES) & 1u) ^ 1u, err, abort_flag)) {
               ok = false;
@@ -299,7 +345,9 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
             tma_load_2d_hint(a_st + s * A_BYTES, wmap, &full_a[s], kb * BK, c.tile * 128,
                              stream_once);
           }
+          u = u_next;
         }
+        if (ok && !push(-1)) ok = false;  // end of this CTA's share of phase p
         if (*(volatile int*)A.gabort) ok = false;
       }
       if (!ok) {
@@ -314,20 +362,30 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
   } else if (warp == 2) {
     if (lane == 0) {
       // ---------------------------------------------- activation (B) producer
-      uint32_t it = 0;
+      uint32_t it = 0, qi = 0;
       bool ok = true;
       for (int p = 0; p < A.n_phases && ok; ++p) {
         const Geom P = geom_of(A.ph[p]);
         if (P.type != CH_GEMM) continue;
-        int u = first_unit(P, cta, G);
-        if (u >= P.units) continue;
         const CUtensorMap* amap = &A.ph[p].amap;
-        tma_prefetch_desc(amap);
-        if (p > 0) {
-          if (!grid_wait(A.done + (p - 1) * CHAIN_DONE_STRIDE, G, err, A.gabort)) { ok = false; break; }
-          fence_proxy_async_global();
-        }
-        for (; u < P.units && ok; u += G) {
+        bool ready = p == 0;
+        for (;;) {
+          const int slot = qi % UQ;
+          if (!mbar_wait(&uq_full[slot], (qi / UQ) & 1u, err, abort_flag)) { ok = false; break; }
+          const int u = uq[slot];
+          ++qi;
+          if (u < 0) break;
+          if (!ready) {
+            // the activations of phase p are complete once every CTA has
+            // finished phase p - 1
+            tma_prefetch_desc(amap);
+            if (!grid_wait(A.done + (p - 1) * CHAIN_DONE_STRIDE, G, err, A.gabort)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            ready = true;
+          }
           const Unit c = unit_of(P, u);
           for (int kb = c.kb_lo; kb < c.kb_hi; ++kb, ++it) {
             const int s = it % STAGES;
@@ -338,6 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
             mbar_arrive_expect_tx(&full_b[s], B_BYTES);
             tma_load_2d(b_st + s * B_BYTES, amap, &full_b[s], kb * BK, 0);
           }
+          if (!ok) break;
         }
       }
       if (!ok) {
@@ -353,12 +412,17 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
     if (lane == 0) {
       // ---------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_f32acc(NT, true);
-      uint32_t it = 0, chain = 0;
+      uint32_t it = 0, chain = 0, qi = 0;
       bool ok = true;
       for (int p = 0; p < A.n_phases && ok; ++p) {
         const Geom P = geom_of(A.ph[p]);
         if (P.type != CH_GEMM) continue;
-        for (int u = first_unit(P, cta, G); u < P.units && ok; u += G) {
+        for (;;) {
+          const int slot = qi % UQ;
+          if (!mbar_wait(&uq_full[slot], (qi / UQ) & 1u, err, abort_flag)) { ok = false; break; }
+          const int u = uq[slot];
+          ++qi;
+          if (u < 0) break;
           const Unit c = unit_of(P, u);
           for (int k0 = c.kb_lo; k0 < c.kb_hi && ok; k0 += P.kc, ++chain) {
             const uint32_t buf = chain % NBUF;
@@ -401,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
     const int quad = warp & 3;
     const int e = quad * 32 + lane;    // feature row = TMEM lane
     const bool leader = wt == 0;
-    uint32_t chain = 0;
+    uint32_t chain = 0, wq = 0;
     bool ok = true;
     for (int p = 0; p < A.n_phases; ++p) {
       // the epilogues and norms read the phase from shared memory: loads
@@ -420,7 +484,26 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
           for (int t = wt; t < TOK; t += WORKERS) lm[t] = sm_empty();
           named_bar(1, WORKERS);
         }
-        for (int u = first_unit(PG, cta, G); u < P.units; u += G) {
+        for (;;) {
+          // next unit from the weight producer's queue (the leader waits and
+          // broadcasts it, so every worker takes the same path)
+          const int slot = wq % UQ;
+          if (leader)
+            uq[UQ] = mbar_wait(&uq_full[slot], (wq / UQ) & 1u, err, abort_flag) ? uq[slot]
+                                                                                : INT_MIN;
+          named_bar(1, WORKERS);
+          const int u = uq[UQ];
+          if (u == INT_MIN) {
+            ok = false;
+            break;
+          }
+          if (u < 0) {  // end of this CTA's share of the phase
+            named_bar(1, WORKERS);
+            if (leader) mbar_arrive(&uq_empty[slot]);
+            ++wq;
+            break;
+          }
+          {
           const Unit c = unit_of(PG, u);
           float acc[TOK];
 #pragma unroll
@@ -456,7 +539,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
 #pragma unroll
               for (int t = 0; t < TOK; ++t) ws_unit[t * 128 + e] = acc[t];
             }
-            continue;
+            goto unit_done;
           }
           if (!lmh) {
             // QKV / SwiGLU: with splits, the last split to arrive at a tile
@@ -503,7 +586,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
             if (run_epi)
               epi_staged_f16(P.ep, acc, n0, 0, e, reinterpret_cast<__half*>(tile), 1);
             named_bar(1, WORKERS);  // last_flag / tile are free for the next unit
-            continue;
+            goto unit_done;
           }
           // LM head: no splits, reduced into this CTA's softmax states.  The
           // barriers run in every thread; a failed wait anywhere skips the work.
@@ -518,6 +601,11 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
           }
           named_bar(1, WORKERS);
           if (fine) epi_chunk(P.ep, tile, n0, 0, e, lm);
+                  }
+        unit_done:
+          named_bar(1, WORKERS);  // every worker is done with the entry and the unit
+          if (leader) mbar_arrive(&uq_empty[slot]);
+          ++wq;
         }
         if (lmh) {
           named_bar(1, WORKERS);
@@ -525,7 +613,10 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
           for (int t = wt; t < P.ep.M; t += WORKERS) out[t] = lm[t];
         }
       } else if (ok && (P.type == CH_NORM || P.type == CH_EMBED_NORM)) {
-        if (p > 0 && cta < A.M) {
+        int first = (cta - P.rot) % G;
+        if (first < 0) first += G;
+        const bool has_items = first < A.M * (A.d >> 9);
+        if (p > 0 && has_items) {
           // one poller per CTA (thousands of polling threads would queue
           // behind the arrivals at the counter's L2 slice)
           if (leader) *last_flag = grid_wait(A.done + (p - 1) * CHAIN_DONE_STRIDE, G, err, A.gabort) ? 1 : 0;
@@ -533,8 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
           ok = *last_flag != 0;
           named_bar(1, WORKERS);
         }
-        if (ok)
-          for (int row = cta; row < A.M; row += G) norm_row(A, P, row, red, wt);
+        if (ok && has_items) ok = norm_phase(A, P, p, cta, G, wt, red, last_flag, err);
       }
       // this CTA's share of phase p is complete: release it to the grid.
       // ok leaves here the same in every worker thread.
@@ -570,6 +660,7 @@ cudaError_t chain_init_attributes() {
 
 cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st) {
   if (args.M < 1 || args.M > TOK || args.d % 512 || args.d > CHAIN_NORM_GROUPS * 512 ||
+      args.M * (args.d / 512) > NORM_MAX_ITEMS * grid ||
       args.n_phases < 1 || args.n_phases > CHAIN_MAX_PHASES)
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};

@@ -205,6 +205,11 @@ struct ChainArgs {
   void* a;                  // normed activations, two-term fp16 pair rows
   const StepParams* sp;
   GemmScratch sc;           // split-K partials and per-tile counters
+  int* rowcnt;              // NORM phases: per-row group arrivals, phase p at rowcnt[p * 32];
+                            // zero at launch
+  float* norm_ss;           // NORM phases: partial sums of squares [32][CHAIN_NORM_GROUPS]
+  int* next;                // GEMM phases: unit claim counters, phase p at next[p *
+                            // CHAIN_DONE_STRIDE]; zero at launch
 };
 static_assert(sizeof(ChainArgs) <= 32764, "kernel parameters are limited to 32 KB");
 
