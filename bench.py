@@ -398,6 +398,89 @@ def run_fdllm(args, wl):
     return 0
 
 
+def run_fdllm_batch(args, wl):
+    """Variable-length batch (independent sequences, per-sequence block
+    schedules) through fdllm_generate_batch; value = generated tokens of the
+    whole batch per second of device time (host prompts in, tokens out: the
+    batched entry point is host-buffer only, so value and e2e time the same
+    call)."""
+    import numpy as np
+    import torch
+    from kv_cache_decode_dualcache_b200 import build, fdllm, synth
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    shape = wl.shape
+    G, B, tau = wl.gen_len, wl.block_size, wl.tau
+    lens = synth.make_batch_prompt_lengths(wl.batch)
+    prompts = [synth.make_prompt(shape, n, salt=rank * 1000 + i).numpy() for i, n in enumerate(lens)]
+    stream = torch.cuda.Stream()
+    dec = fdllm.Decoder(shape, max(lens) + G, device=local, stream=stream.cuda_stream)
+    w = synth.make_weights(shape, device="cuda")
+    dec.load_weights(w)
+    del w
+    torch.cuda.empty_cache()
+    for _ in range(args.warmup):
+        dec.generate_batch(prompts, G, B, tau, wl.cache_mode)
+    sampler = ClockSampler(local) if rank == 0 else None
+    dec.launch_count(reset=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    steps = None
+    for _ in range(args.steps):
+        out, steps, st = dec.generate_batch(prompts, G, B, tau, wl.cache_mode)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = dec.launch_count(reset=True)
+    clocks = sampler.stop() if sampler else None
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    value = world * args.steps * wl.batch * G / (ms * 1e-3)
+    timing = dec.generate_batch(prompts, G, B, tau, wl.cache_mode, timing=True)[2]
+    fdllm.fdllm_profile_enable(dec.ctx, True)
+    dec.generate_batch(prompts, G, B, tau, wl.cache_mode)
+    prof = fdllm.fdllm_profile_read(dec.ctx)
+    fdllm.fdllm_profile_enable(dec.ctx, False)
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, _traffic_record())
+    if rank == 0:
+        cfg = _config(wl, world)
+        cfg.update({"prompt_lens": lens, "batch_per_gpu": wl.batch,
+                    "global_batch": wl.batch * world,
+                    "batching": "sequences run in turn through the single-sequence path"})
+        line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": cfg,
+                "decode": {"denoising_steps_per_generation": int(np.asarray(steps).sum()),
+                           "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
+                           "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3)},
+                "e2e": {"value": round(value, 2), "unit": "tokens/s",
+                        "h2d_bytes_per_step": 4 * sum(lens), "d2h_bytes_per_step": 4 * wl.batch * G},
+                "gpu_launches": launches, "roofline": roof, "clocks": clocks, "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,6 +505,8 @@ def main():
                                  cache_mode=args.cache_mode or wl.cache_mode)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if wl.batch > 1:
+        return run_fdllm_batch(args, wl)
     return run_fdllm(args, wl)
 
 

@@ -152,7 +152,9 @@ FDLLM_API int fdllm_create(const fdllm_config* cfg, int device, void* cuda_strea
                  const fdllm_allocator* alloc, fdllm_ctx** out);
 
 /* Copy the model weights into ctx-owned device memory in the kernels' layout
- * (Wq/Wk/Wv fused, W_gate/W_up interleaved in 64-row groups).  Every tensor
+ * (Wq/Wk/Wv fused and W_gate/W_up interleaved, rows reordered within 32-row
+ * groups so that the rotate-half and gate/up partners meet in one warp; the
+ * bf16 model's GEMM weights stored as fp16, exact for |w| >= 2^-17).  Every tensor
  * named above must appear exactly once.  The caller keeps ownership of the
  * inputs.  Errors: SHAPE (unknown/missing/duplicate name, wrong numel or
  * dtype), OOM, CUDA. */
@@ -177,6 +179,25 @@ FDLLM_API int fdllm_generate(fdllm_ctx* ctx, const int32_t* prompt_ids, int prom
 FDLLM_API int fdllm_generate_device(fdllm_ctx* ctx, const int32_t* prompt_ids_dev, int prompt_len,
                           int gen_len, int block_size, float tau, int cache_mode,
                           int32_t* out_tokens_dev, int* out_steps, fdllm_stats* stats);
+
+/* Variable-length batch: `batch` independent sequences, prompts[i] (host)
+ * holding prompt_lens[i] ids, each generating gen_len tokens with the same
+ * block size, tau and cache mode on its own block schedule (its blocks start
+ * at its own prompt end).  out_tokens (host, caller-owned, batch * gen_len)
+ * receives sequence i's tokens at [i * gen_len, (i + 1) * gen_len);
+ * out_steps (host, batch) its step counts; stats (optional) the totals over
+ * the batch, with steps_per_block (when not NULL) holding batch * gen_len /
+ * block_size entries, sequence by sequence.  Results equal fdllm_generate on
+ * each sequence alone.  The sequences run one after another through the
+ * single-sequence path (each step streams the weights for one sequence):
+ * this entry point fixes the batched interface, not a kernel path that
+ * shares the weight stream across sequences.  Every sequence's arguments are
+ * checked before any work (errors as fdllm_generate; ARG for batch < 1 or
+ * NULL arrays). */
+FDLLM_API int fdllm_generate_batch(fdllm_ctx* ctx, int batch, const int32_t* const* prompts,
+                                   const int* prompt_lens, int gen_len, int block_size, float tau,
+                                   int cache_mode, int32_t* out_tokens, int* out_steps,
+                                   fdllm_stats* stats);
 
 /* Teacher-forced single step (parity checking).  Runs the block-start full
  * forward on snapshot_ids (host, L ids), which fills the K/V cache, then one

@@ -1304,6 +1304,49 @@ int fdllm_generate_device(fdllm_ctx* ctx, const int32_t* prompt_ids_dev, int pro
                        cache_mode, out_tokens_dev, true, out_steps, stats);
 }
 
+int fdllm_generate_batch(fdllm_ctx* ctx, int batch, const int32_t* const* prompts,
+                         const int* prompt_lens, int gen_len, int block_size, float tau,
+                         int cache_mode, int32_t* out_tokens, int* out_steps, fdllm_stats* stats) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (batch < 1 || !prompts || !prompt_lens || !out_tokens || !out_steps)
+    return fail(ctx, FDLLM_ERR_ARG, "batch < 1 or a NULL array");
+  // every sequence's arguments before any work
+  const fdllm_config& c = ctx->cfg;
+  for (int i = 0; i < batch; ++i) {
+    int rc = check_gen_args(ctx, prompt_lens[i], gen_len, block_size, tau, cache_mode);
+    if (rc) return rc;
+    if (prompt_lens[i] > 0 && !prompts[i]) return fail(ctx, FDLLM_ERR_ARG, "NULL prompt");
+    for (int j = 0; j < prompt_lens[i]; ++j)
+      if (prompts[i][j] < 0 || prompts[i][j] >= c.vocab || prompts[i][j] == c.mask_id)
+        return fail(ctx, FDLLM_ERR_ARG, "prompt id out of range or equal to the mask id");
+  }
+  const int n_blocks = gen_len / block_size;
+  fdllm_stats tot{};
+  if (stats) tot.collect_timing = stats->collect_timing;
+  for (int i = 0; i < batch; ++i) {
+    fdllm_stats one{};
+    one.collect_timing = stats ? stats->collect_timing : 0;
+    one.steps_per_block = (stats && stats->steps_per_block)
+                              ? stats->steps_per_block + (size_t)i * n_blocks : nullptr;
+    int rc = generate_impl(ctx, prompts[i], false, prompt_lens[i], gen_len, block_size, tau,
+                           cache_mode, out_tokens + (size_t)i * gen_len, false, &out_steps[i],
+                           stats ? &one : nullptr);
+    if (rc) return rc;
+    tot.steps += one.steps;
+    tot.refresh_steps += one.refresh_steps;
+    tot.cached_steps += one.cached_steps;
+    tot.n_blocks += one.n_blocks;
+    tot.refresh_ms += one.refresh_ms;
+    tot.cached_ms += one.cached_ms;
+  }
+  if (stats) {
+    int32_t* spb = stats->steps_per_block;
+    *stats = tot;
+    stats->steps_per_block = spb;
+  }
+  return FDLLM_OK;
+}
+
 int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, const int32_t* current_ids,
                      int L, int block_start, int block_size, float tau, int cache_mode,
                      float* logits, float* conf, int32_t* tok, uint8_t* unmask) {

@@ -28,6 +28,7 @@ CACHE_MODES = {"none": 0, "prefix": 1, "dual": 2}
 DTYPES = {"fp32": 0, "bf16": 1}
 
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
+            "fdllm_generate_batch",
             "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
             "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
@@ -97,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                    P(ctypes.c_int32), P(i32), P(FdllmStats)]
     lib.fdllm_generate_device.argtypes = [vp, vp, i32, i32, i32, f32, i32, vp, P(i32),
                                           P(FdllmStats)]
+    lib.fdllm_generate_batch.argtypes = [vp, i32, P(P(ctypes.c_int32)), P(i32), i32, i32, f32,
+                                         i32, P(ctypes.c_int32), P(i32), P(FdllmStats)]
     lib.fdllm_step_debug.argtypes = [vp, P(ctypes.c_int32), P(ctypes.c_int32), i32, i32, i32, f32,
                                      i32, P(ctypes.c_float), P(ctypes.c_float),
                                      P(ctypes.c_int32), P(ctypes.c_uint8)]
@@ -112,7 +115,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_launch_count.restype = ctypes.c_int64
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
-                 "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_generate_batch", "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
                  "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -204,6 +207,24 @@ def fdllm_generate(ctx, prompt, gen_len: int, block_size: int, tau: float, cache
                               _i32_ptr(out), ctypes.byref(steps),
                               ctypes.byref(stats) if stats is not None else None), ctx)
     return out, steps.value
+
+
+def fdllm_generate_batch(ctx, prompts, gen_len: int, block_size: int, tau: float, cache_mode,
+                         stats: Optional[FdllmStats] = None):
+    """prompts: a list of 1-D id arrays (any lengths).  Returns (tokens
+    [batch, gen_len] int32, steps [batch] int32)."""
+    lib = load_library()
+    ps = [np.ascontiguousarray(np.asarray(p, dtype=np.int32)) for p in prompts]
+    n = len(ps)
+    ptrs = (ctypes.POINTER(ctypes.c_int32) * max(1, n))(*[_i32_ptr(p) for p in ps])
+    lens = (ctypes.c_int * max(1, n))(*[int(p.size) for p in ps])
+    out = np.empty((n, gen_len), dtype=np.int32)
+    steps = np.empty(n, dtype=np.int32)
+    mode = CACHE_MODES[cache_mode] if isinstance(cache_mode, str) else int(cache_mode)
+    _check(lib.fdllm_generate_batch(ctx, n, ptrs, lens, gen_len, block_size, float(tau), mode,
+                                    _i32_ptr(out), steps.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                    ctypes.byref(stats) if stats is not None else None), ctx)
+    return out, steps
 
 
 def fdllm_generate_device(ctx, prompt_dev, gen_len: int, block_size: int, tau: float, cache_mode,
@@ -360,6 +381,20 @@ class Decoder:
         out, steps = fdllm_generate(self.ctx, prompt, gen_len, block_size, tau, cache_mode, st)
         return out, steps, GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
                                          list(spb)[:n_blocks], st.refresh_ms, st.cached_ms)
+
+    def generate_batch(self, prompts, gen_len: int, block_size: int, tau: float,
+                       cache_mode="dual", timing: bool = False):
+        """Variable-length batch: returns (tokens [batch, gen_len], steps [batch],
+        GenerateStats of the totals, steps_per_block sequence by sequence)."""
+        n_blocks = gen_len // block_size if block_size > 0 else 0
+        spb = (ctypes.c_int32 * max(1, n_blocks * len(prompts)))()
+        st = FdllmStats(0, 0, 0, 0, ctypes.cast(spb, ctypes.POINTER(ctypes.c_int32)), int(timing),
+                        0.0, 0.0)
+        out, steps = fdllm_generate_batch(self.ctx, prompts, gen_len, block_size, tau, cache_mode,
+                                          st)
+        return out, steps, GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
+                                         list(spb)[:n_blocks * len(prompts)], st.refresh_ms,
+                                         st.cached_ms)
 
     def generate_device(self, prompt_dev, gen_len: int, block_size: int, tau: float, out_dev,
                         cache_mode="dual") -> int:
