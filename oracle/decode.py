@@ -82,6 +82,22 @@ def select_unmask(masked: np.ndarray, conf: np.ndarray, tau: float) -> np.ndarra
     return u
 
 
+def select_top_k(masked: np.ndarray, conf: np.ndarray, k: int) -> np.ndarray:
+    """Unmask set of one step of the fixed-count strategy that the threshold
+    rule replaces (techwalker.com Fast-dLLM article, section
+    "解决并行解码的质量下降问题": earlier methods unmask a fixed number of
+    tokens per step): the k most confident masked positions, the lower
+    position first among equal confidences; every masked position when fewer
+    than k are masked."""
+    masked = np.asarray(masked, dtype=bool)
+    conf = np.asarray(conf, dtype=np.float64)
+    cand = [int(i) for i in np.flatnonzero(masked)]
+    cand.sort(key=lambda i: (-conf[i], i))
+    u = np.zeros(masked.shape, dtype=bool)
+    u[cand[:max(0, int(k))]] = True
+    return u
+
+
 @dataclass
 class StepRecord:
     block: int
@@ -101,8 +117,11 @@ class GenerateResult:
 
 
 def generate(model, prompt: Sequence[int], gen_len: int, block_size: int, tau: float,
-             cache_mode="dual", keep_logits: bool = False, on_refresh=None) -> GenerateResult:
-    """Block-wise generation (see module docstring).
+             cache_mode="dual", keep_logits: bool = False, on_refresh=None,
+             fixed_k: Optional[int] = None) -> GenerateResult:
+    """Block-wise generation (see module docstring).  With ``fixed_k`` every
+    step unmasks the fixed_k most confident masked positions of the block
+    (``select_top_k``) instead of applying the threshold rule; tau is unused.
 
     ``model`` is anything with ``spec.mask_id`` and
     ``forward(x, rows, cache=None, return_kv=False, head_rows=None)``; the
@@ -144,7 +163,7 @@ def generate(model, prompt: Sequence[int], gen_len: int, block_size: int, tau: f
             first = False
             conf, tok = confidence(z, mask_id)
             masked = x[s:e] == mask_id
-            u = select_unmask(masked, conf, tau)
+            u = select_top_k(masked, conf, fixed_k) if fixed_k else select_unmask(masked, conf, tau)
             x[s:e][u] = tok[u]
             n_steps += 1
             res.trace.append(StepRecord(b, kind, conf, tok, u, z if keep_logits else None))
