@@ -180,6 +180,18 @@ FDLLM_API int fdllm_generate_device(fdllm_ctx* ctx, const int32_t* prompt_ids_de
                           int gen_len, int block_size, float tau, int cache_mode,
                           int32_t* out_tokens_dev, int* out_steps, fdllm_stats* stats);
 
+/* Fixed-count decoding, the strategy that the confidence threshold replaces
+ * (techwalker.com Fast-dLLM article, section "解决并行解码的质量下降问题":
+ * earlier methods unmask a fixed number of tokens per step): as
+ * fdllm_generate, but every step unmasks the k most confident masked
+ * positions of the block (the lower position first among equal
+ * confidences; all remaining ones when fewer than k are masked), so a block
+ * of B positions takes ceil(B / k) steps.  Errors as fdllm_generate; ARG for
+ * k < 1. */
+FDLLM_API int fdllm_generate_fixed_k(fdllm_ctx* ctx, const int32_t* prompt_ids, int prompt_len,
+                                     int gen_len, int block_size, int k, int cache_mode,
+                                     int32_t* out_tokens, int* out_steps, fdllm_stats* stats);
+
 /* Variable-length batch: `batch` independent sequences, prompts[i] (host)
  * holding prompt_lens[i] ids, each generating gen_len tokens with the same
  * block size, tau and cache mode on its own block schedule (its blocks start

@@ -121,6 +121,7 @@ struct fdllm_ctx {
   StepParams* sp = nullptr;     // device step scalars (read by the kernels)
   StepParams* sp_host = nullptr;  // pinned ring of kSpRing slots: a pending async copy
   int sp_slot = 0;                // never reads a slot overwritten after it was queued
+  int fixed_k = 0;                // > 0 during fdllm_generate_fixed_k
   struct StepGraph {
     cudaGraphExec_t exec;
     int n_part;
@@ -748,7 +749,7 @@ int sync_state(fdllm_ctx* ctx) {
 int set_step_params(fdllm_ctx* ctx, int r0, int lm0, int s, float tau) {
   StepParams* slot = ctx->sp_host + ctx->sp_slot;
   ctx->sp_slot = (ctx->sp_slot + 1) % kSpRing;
-  *slot = StepParams{r0, lm0, s, tau};
+  *slot = StepParams{r0, lm0, s, tau, ctx->fixed_k};
   CK(cudaMemcpyAsync(ctx->sp, slot, sizeof(StepParams), cudaMemcpyHostToDevice, ctx->stream));
   return FDLLM_OK;
 }
@@ -1302,6 +1303,18 @@ int fdllm_generate_device(fdllm_ctx* ctx, const int32_t* prompt_ids_dev, int pro
   if (!ctx) return FDLLM_ERR_ARG;
   return generate_impl(ctx, prompt_ids_dev, true, prompt_len, gen_len, block_size, tau,
                        cache_mode, out_tokens_dev, true, out_steps, stats);
+}
+
+int fdllm_generate_fixed_k(fdllm_ctx* ctx, const int32_t* prompt_ids, int prompt_len,
+                           int gen_len, int block_size, int k, int cache_mode,
+                           int32_t* out_tokens, int* out_steps, fdllm_stats* stats) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (k < 1) return fail(ctx, FDLLM_ERR_ARG, "k must be >= 1");
+  ctx->fixed_k = k;
+  const int rc = generate_impl(ctx, prompt_ids, false, prompt_len, gen_len, block_size, 0.0f,
+                               cache_mode, out_tokens, false, out_steps, stats);
+  ctx->fixed_k = 0;
+  return rc;
 }
 
 int fdllm_generate_batch(fdllm_ctx* ctx, int batch, const int32_t* const* prompts,

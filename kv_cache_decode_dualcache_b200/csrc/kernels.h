@@ -26,6 +26,7 @@ struct StepParams {
   int lm0;           // first LM-head row within the forward
   int s;             // block start position (unmask target)
   float tau;         // confidence threshold
+  int fixed_k;       // > 0: unmask the fixed_k most confident masked positions instead
 };
 
 // Everything a GEMM epilogue needs.  Token index t is the row within the

@@ -122,9 +122,11 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
   __shared__ int s_best;
   pdl_trigger();
   pdl_wait();
+  int fixed_k = 0;
   if (sp) {
     s = sp->s;
     tau = sp->tau;
+    fixed_k = sp->fixed_k;
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int t = warp; t < n; t += blockDim.x >> 5) {
@@ -146,7 +148,19 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
   const bool valid = i < n;
   const bool masked = valid && x[s + i] == mask_id;
   const float ci = valid ? s_conf[i] : 0.0f;
-  const bool pass = masked && (ci >= tau);
+  bool pass = masked && (ci >= tau);
+  if (fixed_k > 0) {
+    // fixed-count strategy: the fixed_k most confident masked positions,
+    // the lower position first among equal confidences (NaN counts as -1)
+    const float mine = (ci == ci) ? ci : -1.0f;
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      if (j == i || x[s + j] != mask_id) continue;
+      const float cj = (s_conf[j] == s_conf[j]) ? s_conf[j] : -1.0f;
+      rank += (cj > mine || (cj == mine && j < i)) ? 1 : 0;
+    }
+    pass = masked && rank < fixed_k;
+  }
   const int n_pass = __syncthreads_count(pass);
   if (threadIdx.x == 0) {
     int best = -1;

@@ -28,7 +28,7 @@ CACHE_MODES = {"none": 0, "prefix": 1, "dual": 2}
 DTYPES = {"fp32": 0, "bf16": 1}
 
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
-            "fdllm_generate_batch",
+            "fdllm_generate_batch", "fdllm_generate_fixed_k",
             "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
             "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
@@ -98,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                    P(ctypes.c_int32), P(i32), P(FdllmStats)]
     lib.fdllm_generate_device.argtypes = [vp, vp, i32, i32, i32, f32, i32, vp, P(i32),
                                           P(FdllmStats)]
+    lib.fdllm_generate_fixed_k.argtypes = [vp, P(ctypes.c_int32), i32, i32, i32, i32, i32,
+                                           P(ctypes.c_int32), P(i32), P(FdllmStats)]
     lib.fdllm_generate_batch.argtypes = [vp, i32, P(P(ctypes.c_int32)), P(i32), i32, i32, f32,
                                          i32, P(ctypes.c_int32), P(i32), P(FdllmStats)]
     lib.fdllm_step_debug.argtypes = [vp, P(ctypes.c_int32), P(ctypes.c_int32), i32, i32, i32, f32,
@@ -115,7 +117,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_launch_count.restype = ctypes.c_int64
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
-                 "fdllm_generate_batch", "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
                  "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -206,6 +208,19 @@ def fdllm_generate(ctx, prompt, gen_len: int, block_size: int, tau: float, cache
     _check(lib.fdllm_generate(ctx, _i32_ptr(p), int(p.size), gen_len, block_size, float(tau), mode,
                               _i32_ptr(out), ctypes.byref(steps),
                               ctypes.byref(stats) if stats is not None else None), ctx)
+    return out, steps.value
+
+
+def fdllm_generate_fixed_k(ctx, prompt, gen_len: int, block_size: int, k: int, cache_mode,
+                           stats: Optional[FdllmStats] = None):
+    lib = load_library()
+    p = np.ascontiguousarray(np.asarray(prompt, dtype=np.int32))
+    out = np.empty(gen_len, dtype=np.int32)
+    steps = ctypes.c_int()
+    mode = CACHE_MODES[cache_mode] if isinstance(cache_mode, str) else int(cache_mode)
+    _check(lib.fdllm_generate_fixed_k(ctx, _i32_ptr(p), int(p.size), gen_len, block_size, int(k),
+                                      mode, _i32_ptr(out), ctypes.byref(steps),
+                                      ctypes.byref(stats) if stats is not None else None), ctx)
     return out, steps.value
 
 
@@ -373,12 +388,17 @@ class Decoder:
         fdllm_load_weights(self.ctx, weights, self.shape.dtype)
 
     def generate(self, prompt, gen_len: int, block_size: int, tau: float, cache_mode="dual",
-                 timing: bool = False):
+                 timing: bool = False, fixed_k: Optional[int] = None):
+        """Threshold decoding (tau), or with fixed_k the fixed-count strategy."""
         n_blocks = gen_len // block_size if block_size > 0 else 0
         spb = (ctypes.c_int32 * max(1, n_blocks))()
         st = FdllmStats(0, 0, 0, 0, ctypes.cast(spb, ctypes.POINTER(ctypes.c_int32)), int(timing),
                         0.0, 0.0)
-        out, steps = fdllm_generate(self.ctx, prompt, gen_len, block_size, tau, cache_mode, st)
+        if fixed_k is not None:
+            out, steps = fdllm_generate_fixed_k(self.ctx, prompt, gen_len, block_size, fixed_k,
+                                                cache_mode, st)
+        else:
+            out, steps = fdllm_generate(self.ctx, prompt, gen_len, block_size, tau, cache_mode, st)
         return out, steps, GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
                                          list(spb)[:n_blocks], st.refresh_ms, st.cached_ms)
 
