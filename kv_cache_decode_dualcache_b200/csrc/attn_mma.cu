@@ -10,9 +10,11 @@
 // is a (position, head-in-group) pair, so the query heads that share a KV
 // head in GQA share the K/V tiles.  K/V tiles of 64 keys (one cache page)
 // are double-buffered in shared memory with cp.async, in a 16-byte-chunk XOR
-// swizzle so ldmatrix is conflict-free.  The four warps are NKG key groups x
-// (4 / NKG) row groups of 16 rows: with few query rows (a 32-token block,
-// MHA: NKG = 2) the warps split every key tile between them instead of
+// swizzle so ldmatrix is conflict-free.  The NW warps (4, or 8 for full
+// forwards with many query rows, so that twice the warps share each K/V
+// tile) are NKG key groups x (NW / NKG) row groups of 16 rows: with few
+// query rows (a 32-token block, MHA: NKG = 2) the warps split every key
+// tile between them instead of
 // idling, and merge their online-softmax states through shared memory at
 // the end.
 //
@@ -72,17 +74,19 @@ FD_DEV uint32_t swz(int r, int ch) {
   return (uint32_t)(r * HD * 2 + ((ch ^ (r & 7)) << 4));
 }
 
-template <int HD, int NKG>
-__global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
+template <int HD, int NKG, int NW>
+__global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
+  constexpr int NT = NW * 32;        // threads
   constexpr int TILE = 64 * HD * 2;  // bytes of one [64][HD] 2-byte tile
   constexpr int CH = HD / 8;         // 16-byte chunks per row
-  constexpr int NRG = 4 / NKG;       // row groups of 16 rows
+  constexpr int NRG = NW / NKG;      // row groups of 16 rows
+  constexpr int QT = 16 * NRG * HD * 2;  // bytes of one Q plane
   constexpr int KEYS = 64 / NKG;     // keys of a tile per key group
   constexpr int NNT = KEYS / 8;      // 8-key n-tiles per key group
   extern __shared__ __align__(128) uint8_t sm[];
   // layout: Q hi, Q lo, then per buffer b: K hi, K lo, V hi, V lo
   const uint32_t q_s = smem_u32(sm);
-  auto kv_s = [&](int buf, int plane) { return q_s + (2 + buf * 4 + plane) * TILE; };
+  auto kv_s = [&](int buf, int plane) { return q_s + 2 * QT + (buf * 4 + plane) * TILE; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = warp % NRG, kg = warp / NRG;
@@ -100,21 +104,21 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   pdl_wait();
 
   // ---- Q tiles (hi and lo planes), 16 * NRG rows
-  for (int idx = tid; idx < 16 * NRG * CH; idx += 128) {
+  for (int idx = tid; idx < 16 * NRG * CH; idx += NT) {
     const int i = idx / CH, ch = idx % CH;
     const int r = row0 + i;
     const bool ok = r < rows_total;
     const int m = ok ? r / rep : 0, jj = ok ? r % rep : 0;
     const __half* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
     cp_async16(q_s + swz<HD>(i, ch), src, ok ? 16 : 0);
-    cp_async16(q_s + TILE + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
+    cp_async16(q_s + QT + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
   }
   auto load_kv = [&](int kt, int buf) {
     const int k0 = key_lo + kt * 64;
     const int page = p.page_table[k0 / KV_PAGE];
     const size_t plane = (size_t)Hkv * KV_PAGE * HD;
     const size_t base = ((size_t)p.layer * p.n_pages + page) * 4 * plane + (size_t)g * KV_PAGE * HD;
-    for (int idx = tid; idx < 64 * CH; idx += 128) {
+    for (int idx = tid; idx < 64 * CH; idx += NT) {
       const int i = idx / CH, ch = idx % CH;
       const bool ok = (k0 + i) < key_hi;
       const size_t e = base + (size_t)(ok ? i : 0) * HD + ch * 8;
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
         uint32_t qh[4], ql[4];
         const uint32_t qa = swz<HD>(rg * 16 + (lane & 15), 2 * kk + (lane >> 4));
         ldsm_x4(q_s + qa, qh);
-        ldsm_x4(q_s + TILE + qa, ql);
+        ldsm_x4(q_s + QT + qa, ql);
 #pragma unroll
         for (int np = 0; np < NNT / 2; ++np) {
           uint32_t kh[4], kl[4];
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
     // per warp: 32 lanes x (HD/2 accumulators + 2 max + 2 sums) floats,
     // placed over the (now unused) K/V buffers
     constexpr int PER_LANE = HD / 2 + 4;
-    float* xch = reinterpret_cast<float*>(sm + 2 * TILE);
+    float* xch = reinterpret_cast<float*>(sm + 2 * QT);
     float* mine = xch + (size_t)(warp * 32 + lane) * PER_LANE;
     if (kg > 0) {
 #pragma unroll
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   // result does not depend on timing.
   if (p.n_split > 1) {
     constexpr int PER_LANE = HD / 2 + 4;
-    float* xch = reinterpret_cast<float*>(sm + 2 * TILE);
+    float* xch = reinterpret_cast<float*>(sm + 2 * QT);
     float* mine = xch + (size_t)(warp * 32 + lane) * PER_LANE;
     __syncthreads();  // the key-group merge above is done with xch
     if (writer) {
@@ -351,26 +355,33 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(AttnParams p) {
   }
 }
 
-template <int HD, int NKG>
+// Shared memory: Q hi and lo planes of 16 * NW / NKG rows, then two buffers
+// of the four K/V planes of a 64-key tile.
+template <int HD, int NKG, int NW>
+constexpr int attn_smem() { return 2 * (16 * (NW / NKG) * HD * 2) + 8 * 64 * HD * 2; }
+
+template <int HD, int NKG, int NW>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(attn_mma_kernel<HD, NKG>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, 10 * 64 * HD * 2);
+  static_assert(attn_smem<HD, NKG, NW>() <= 232448, "exceeds the 227 KB shared memory limit");
+  return cudaFuncSetAttribute(attn_mma_kernel<HD, NKG, NW>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              attn_smem<HD, NKG, NW>());
 }
 
-template <int HD, int NKG>
+template <int HD, int NKG, int NW>
 cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
-  constexpr int smem = 10 * 64 * HD * 2;
+  constexpr int smem = attn_smem<HD, NKG, NW>();
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = set_attr<HD, NKG>();
+    cudaError_t e = set_attr<HD, NKG, NW>();
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
-  const int rows_per_cta = 16 * (4 / NKG);
+  const int rows_per_cta = 16 * (NW / NKG);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((rows + rows_per_cta - 1) / rows_per_cta, p.n_kv_heads, p.n_split);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute la[2];
@@ -389,22 +400,24 @@ cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
   }
   cfg.attrs = la;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<HD, NKG>, p);
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<HD, NKG, NW>, p);
 }
 
 template <int HD>
 cudaError_t launch_nkg(const AttnParams& p, cudaStream_t st, bool pdl) {
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
-  if (rows <= 16) return launch_hd<HD, 4>(p, st, pdl);
-  if (rows <= 32) return launch_hd<HD, 2>(p, st, pdl);
-  return launch_hd<HD, 1>(p, st, pdl);
+  if (rows <= 16) return launch_hd<HD, 4, 4>(p, st, pdl);
+  if (rows <= 32) return launch_hd<HD, 2, 4>(p, st, pdl);
+  if (rows <= 64) return launch_hd<HD, 1, 4>(p, st, pdl);
+  // many query rows (full forwards, GQA): eight warps share each K/V tile
+  return launch_hd<HD, 1, 8>(p, st, pdl);
 }
 
 }  // namespace
 
 int attn_rows_per_cta(int M, int n_heads, int n_kv_heads) {
   const int rows = M * (n_heads / n_kv_heads);
-  return rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
+  return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
 }
 
 cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl) {
@@ -419,12 +432,14 @@ cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl) {
 cudaError_t gemm_tc_init_attributes();
 
 cudaError_t init_kernel_attributes() {
-  cudaError_t e = set_attr<64, 1>();
-  if (e == cudaSuccess) e = set_attr<64, 2>();
-  if (e == cudaSuccess) e = set_attr<64, 4>();
-  if (e == cudaSuccess) e = set_attr<128, 1>();
-  if (e == cudaSuccess) e = set_attr<128, 2>();
-  if (e == cudaSuccess) e = set_attr<128, 4>();
+  cudaError_t e = set_attr<64, 1, 4>();
+  if (e == cudaSuccess) e = set_attr<64, 2, 4>();
+  if (e == cudaSuccess) e = set_attr<64, 4, 4>();
+  if (e == cudaSuccess) e = set_attr<64, 1, 8>();
+  if (e == cudaSuccess) e = set_attr<128, 1, 4>();
+  if (e == cudaSuccess) e = set_attr<128, 2, 4>();
+  if (e == cudaSuccess) e = set_attr<128, 4, 4>();
+  if (e == cudaSuccess) e = set_attr<128, 1, 8>();
   if (e == cudaSuccess) e = gemm_tc_init_attributes();
   if (e == cudaSuccess) e = chain_init_attributes();
   return e;
