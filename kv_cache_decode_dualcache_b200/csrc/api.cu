@@ -424,7 +424,9 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
     return FDLLM_OK;
   }
   // Few query rows (block steps): split the keys so that the (row tile, KV
-  // head, split) CTAs fill the SMs once, at least 2 key tiles per split.
+  // head, split) CTAs fill the SMs once, at least 2 key tiles per split
+  // (measured: one key tile per split, with two single-buffered CTAs per SM
+  // and clusters of 8, is slower).
   const int rep = c.n_heads / c.n_kv_heads;
   const int rows_per_cta = attn_rows_per_cta(M, c.n_heads, c.n_kv_heads);
   const int ctas = ((M * rep + rows_per_cta - 1) / rows_per_cta) * c.n_kv_heads;
@@ -698,7 +700,7 @@ int forward_chain(fdllm_ctx* ctx, int M, int L, float* dbg, int* n_part) {
     A.next = ctx->chain_sync + next0 + pr.first[ci] * CHAIN_DONE_STRIDE;
     {
       ProfScope ps(ctx, "chain.step", pr.bytes[ci], pr.flops[ci]);
-      KL(launch_chain(A, ctx->num_sms, ctx->stream));
+      KL(launch_chain(A, ctx->num_sms, ctx->stream, ctx->pdl && ci > 0));
     }
     if ((int)ci < c.n_layers) {
       int rc = run_attention(ctx, (int)ci, M, L);

@@ -355,10 +355,15 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
   }
 }
 
-// Shared memory: Q hi and lo planes of 16 * NW / NKG rows, then two buffers
-// of the four K/V planes of a 64-key tile.
+// Shared memory: Q hi and lo planes of 16 * NW / NKG rows, then nbuf
+// buffers of the four K/V planes of a 64-key tile (one buffer when a CTA
+// has a single key tile), which the key-group and split merges reuse.
 template <int HD, int NKG, int NW>
-constexpr int attn_smem() { return 2 * (16 * (NW / NKG) * HD * 2) + 8 * 64 * HD * 2; }
+constexpr int attn_smem(int nbuf = 2) {
+  return 2 * (16 * (NW / NKG) * HD * 2) +
+         (nbuf * 4 * 64 * HD * 2 > NW * 32 * (HD / 2 + 4) * 4 ? nbuf * 4 * 64 * HD * 2
+                                                               : NW * 32 * (HD / 2 + 4) * 4);
+}
 
 template <int HD, int NKG, int NW>
 cudaError_t set_attr() {
@@ -370,7 +375,8 @@ cudaError_t set_attr() {
 
 template <int HD, int NKG, int NW>
 cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
-  constexpr int smem = attn_smem<HD, NKG, NW>();
+  // a single key tile per CTA needs one K/V buffer: two CTAs fit on an SM
+  const int smem = attn_smem<HD, NKG, NW>(p.keys_per_split <= 64 ? 1 : 2);
   static bool attr = false;
   if (!attr) {
     cudaError_t e = set_attr<HD, NKG, NW>();

@@ -111,10 +111,10 @@ FD_DEV int ld_relaxed(const int* p) {
 FD_DEV bool grid_wait(const int* ctr, int target, int* err, int* gabort) {
   if (ld_relaxed(ctr) < target) {
     const uint64_t t0 = global_timer_ns();
-    uint32_t ns = 128;
+    uint32_t ns = 64;
     for (uint32_t it = 1;; ++it) {
       __nanosleep(ns);
-      if (ns < 1024) ns *= 2;
+      if (ns < 256) ns *= 2;
       if (ld_relaxed(ctr) >= target) break;
       if ((it & 7u) == 0) {
         if (*(volatile int*)gabort) return false;
@@ -368,7 +368,10 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
         const Geom P = geom_of(A.ph[p]);
         if (P.type != CH_GEMM) continue;
         const CUtensorMap* amap = &A.ph[p].amap;
+        // phase 0 reads the previous kernel's output (programmatic launch:
+        // wait until that kernel has completed)
         bool ready = p == 0;
+        if (p == 0) pdl_wait();
         for (;;) {
           const int slot = qi % UQ;
           if (!mbar_wait(&uq_full[slot], (qi / UQ) & 1u, err, abort_flag)) { ok = false; break; }
@@ -658,10 +661,11 @@ cudaError_t chain_init_attributes() {
   return cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
 }
 
-cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st) {
+cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st, bool after_kernel) {
   if (args.M < 1 || args.M > TOK || args.d % 512 || args.d > CHAIN_NORM_GROUPS * 512 ||
       args.M * (args.d / 512) > NORM_MAX_ITEMS * grid ||
-      args.n_phases < 1 || args.n_phases > CHAIN_MAX_PHASES)
+      args.n_phases < 1 || args.n_phases > CHAIN_MAX_PHASES ||
+      (after_kernel && args.ph[0].type != CH_GEMM))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -669,8 +673,21 @@ cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st) {
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = st;
   cudaLaunchAttribute la[1];
-  la[0].id = cudaLaunchAttributeCooperative;  // phases wait on every CTA of the grid
-  la[0].val.cooperative = 1;
+  if (after_kernel) {
+    // Programmatic launch after the attention kernel: CTAs start as its CTAs
+    // retire, and the weight stream begins at once; only the first phase's
+    // activation loads wait for the attention output (pdl_wait).  Phases
+    // wait on every CTA of the grid, so all grid CTAs must become resident:
+    // the grid is one CTA per SM (the shared memory admits no second), and
+    // the preceding kernel's CTAs never wait on this one, so every SM frees
+    // up; if that assumption is ever broken the bounded phase waits end the
+    // launch with DEV_ERR_TIMEOUT instead of hanging.
+    la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[0].val.programmaticStreamSerializationAllowed = 1;
+  } else {
+    la[0].id = cudaLaunchAttributeCooperative;  // phases wait on every CTA of the grid
+    la[0].val.cooperative = 1;
+  }
   cfg.attrs = la;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, chain_kernel, args);

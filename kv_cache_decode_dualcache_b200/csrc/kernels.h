@@ -214,8 +214,11 @@ struct ChainArgs {
 };
 static_assert(sizeof(ChainArgs) <= 32764, "kernel parameters are limited to 32 KB");
 
-// Cooperative launch of grid CTAs (one per SM).
-cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st);
+// Launch of grid CTAs (one per SM): cooperative, or with after_kernel a
+// programmatic dependent launch behind the preceding kernel of the stream
+// (the program must then begin with a GEMM phase, whose activation loads
+// wait for that kernel).
+cudaError_t launch_chain(const ChainArgs& args, int grid, cudaStream_t st, bool after_kernel);
 cudaError_t chain_init_attributes();
 int chain_smem_bytes();
 

@@ -113,6 +113,82 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x,
   }
 }
 
+// bf16 model with d % 4 == 0: as rmsnorm_kernel<__nv_bfloat16>, four
+// consecutive features per thread and access (16-byte h loads and stores,
+// 8-byte embedding loads and two-term stores).
+__global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__ x, int r0,
+                                                         const __nv_bfloat16* __restrict__ embed,
+                                                         int vocab, float* __restrict__ h,
+                                                         int h_row0, int d,
+                                                         const float* __restrict__ g, float eps,
+                                                         __half* __restrict__ a, int* err,
+                                                         const StepParams* sp, int rows_from_lm0) {
+  constexpr int V4 = RMS_VPT / 4;
+  __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x;
+  if (sp) {
+    if (x) r0 = sp->r0;
+    if (rows_from_lm0) h_row0 = sp->lm0;
+  }
+  float* hr = h + (size_t)(h_row0 + row) * d;
+  float4 v[V4];
+  if (x) {
+    int tok = x[r0 + row];
+    if (tok < 0 || tok >= vocab) {
+      if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
+      tok = 0;
+    }
+    const __nv_bfloat16* er = embed + (size_t)tok * d;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const int j = (threadIdx.x + k * 256) * 4;
+      if (j < d) {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(er + j));
+        const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        v[k] = make_float4(__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1));
+      } else {
+        v[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const int j = (threadIdx.x + k * 256) * 4;
+      if (j < d) *reinterpret_cast<float4*>(hr + j) = v[k];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const int j = (threadIdx.x + k * 256) * 4;
+      v[k] = j < d ? *reinterpret_cast<const float4*>(hr + j) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+  }
+  float ss = 0.0f;
+#pragma unroll
+  for (int k = 0; k < V4; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  const size_t r_hi = (size_t)pair_row(row) * d, r_lo = r_hi + (size_t)PAIR_LO * d;
+#pragma unroll
+  for (int k = 0; k < V4; ++k) {
+    const int j = (threadIdx.x + k * 256) * 4;
+    if (j < d) {
+      const float4 gn = __ldg(reinterpret_cast<const float4*>(g + j));
+      __half h0, l0, h1, l1, h2, l2, h3, l3;
+      split_f16(v[k].x * inv * gn.x, h0, l0);
+      split_f16(v[k].y * inv * gn.y, h1, l1);
+      split_f16(v[k].z * inv * gn.z, h2, l2);
+      split_f16(v[k].w * inv * gn.w, h3, l3);
+      __half2 hh[2] = {__halves2half2(h0, h1), __halves2half2(h2, h3)};
+      __half2 ll[2] = {__halves2half2(l0, l1), __halves2half2(l2, l3)};
+      *reinterpret_cast<uint2*>(a + r_hi + j) = *reinterpret_cast<const uint2*>(hh);
+      *reinterpret_cast<uint2*>(a + r_lo + j) = *reinterpret_cast<const uint2*>(ll);
+    }
+  }
+}
+
 // ------------------------------------------------------- merge + select
 __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
                                     int mask_id, float tau, int select, float* conf, int* tok,
@@ -328,6 +404,9 @@ cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed,
   if (f32)
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, x, r0,
                     (const float*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
+  if (d % 4 == 0)
+    return launch_k(pdl, rmsnorm_v4_kernel, dim3(M), dim3(256), 0, st, x, r0,
+                    (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, (__half*)a, err, sp, 0);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, x, r0,
                   (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
 }
@@ -341,6 +420,10 @@ cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, nx, 0,
                     (const float*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
                     (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+  if (d % 4 == 0)
+    return launch_k(pdl, rmsnorm_v4_kernel, dim3(M), dim3(256), 0, st, nx, 0,
+                    (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps,
+                    (__half*)a, (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
                   (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
                   (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
