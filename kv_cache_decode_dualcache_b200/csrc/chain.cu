@@ -645,6 +645,10 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
     if (!ok) *abort_flag = 1;
   }
 
+  // lanes 1..31 of the single-thread role warps reach this point long before
+  // their lane 0: reconverge every warp first, so that the CTA barrier below
+  // counts each warp once, with all of its threads
+  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     __syncwarp();

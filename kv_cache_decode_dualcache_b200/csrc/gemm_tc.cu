@@ -343,6 +343,10 @@ __global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
     }
   }
 
+  // lanes 1..31 of the single-thread role warps reach this point long before
+  // their lane 0: reconverge every warp first, so that the CTA barrier below
+  // counts each warp once, with all of its threads
+  __syncwarp();
   __syncthreads();
   if (lmhead && warp >= 2) {
     SoftmaxState* out = reinterpret_cast<SoftmaxState*>(ep.lm_part) + (size_t)blockIdx.x * gs.M;
