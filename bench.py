@@ -182,6 +182,31 @@ def _traffic_record():
     return None
 
 
+# ---------------------------------------------------------------- replicas
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank passes its own device-timed
+    milliseconds and gets the maximum (identity on one rank)."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, steps, gen_tokens_per_step, ms_max):
+    """Whole-job throughput of independent replicas: every rank generated
+    steps * gen_tokens_per_step tokens within the slowest rank's time."""
+    return world * steps * gen_tokens_per_step / (ms_max * 1e-3)
+
+
+def replica_prompt(shape, prompt_len, rank):
+    """Rank r decodes its own sequence: the workload's prompt recipe with
+    salt r (rank 0 gets the single-GPU prompt)."""
+    from kv_cache_decode_dualcache_b200 import synth
+    return synth.make_prompt(shape, prompt_len, salt=rank).numpy()
+
+
 # ---------------------------------------------------------------- CPU oracle
 def oracle_sample(wl, weights_host, step_counts, sample_layers=4):
     """The float64 oracle, as it stands, on a bounded sample: one block-start
@@ -294,7 +319,7 @@ def run_fdllm(args, wl):
                   if not k.startswith("layers.") or int(k.split(".")[1]) < 4}
     del w
     torch.cuda.empty_cache()
-    prompt = synth.make_prompt(shape, P, salt=rank).numpy()
+    prompt = replica_prompt(shape, P, rank)
     prompt_host = torch.from_numpy(prompt).pin_memory()
     prompt_dev = prompt_host.to(f"cuda:{local}")
     out_dev = torch.empty(G, dtype=torch.int32, device=f"cuda:{local}")
@@ -320,11 +345,8 @@ def run_fdllm(args, wl):
     ms = e0.elapsed_time(e1)
     launches = dec.launch_count(reset=True)
     clocks = sampler.stop() if sampler else None
-    t = torch.tensor([ms], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * args.steps * G / (ms_max * 1e-3)
+    ms_max = max_over_ranks(ms, world, f"cuda:{local}")
+    value = job_tokens_per_s(world, args.steps, G, ms_max)
     tokens = out_dev.cpu().numpy()
 
     # ---- end to end: host buffers through the C call
@@ -342,10 +364,8 @@ def run_fdllm(args, wl):
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()
-    t2 = torch.tensor([e2.elapsed_time(e3)], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = world * args.steps * G / (float(t2.item()) * 1e-3)
+    e2e_value = job_tokens_per_s(world, args.steps, G,
+                                 max_over_ranks(e2.elapsed_time(e3), world, f"cuda:{local}"))
     steps_per_gen = e2e_steps / args.steps
     h2d = P * 4
     d2h = G * 4 + int(round(steps_per_gen)) * 20   # tokens + per-step state / error words
@@ -446,11 +466,8 @@ def run_fdllm_batch(args, wl):
     torch.cuda.synchronize()
     launches = dec.launch_count(reset=True)
     clocks = sampler.stop() if sampler else None
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    value = world * args.steps * wl.batch * G / (ms * 1e-3)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{local}")
+    value = job_tokens_per_s(world, args.steps, wl.batch * G, ms)
     timing = dec.generate_batch(prompts, G, B, tau, wl.cache_mode, timing=True)[2]
     fdllm.fdllm_profile_enable(dec.ctx, True)
     dec.generate_batch(prompts, G, B, tau, wl.cache_mode)
@@ -481,6 +498,49 @@ def run_fdllm_batch(args, wl):
     return 0
 
 
+def run_kv_similarity(args, wl):
+    """The approximate cache's premise on this workload: cosine of the K/V a
+    full forward gives at the first block's start and after that block's
+    first denoising step, per layer, over the positions a DualCache step
+    takes from the cache (prefix and suffix); fdllm_kv_similarity on the
+    GPU.  Random weights: the numbers show the diagnostic, not a trained
+    model's behaviour."""
+    import numpy as np
+    import torch
+    from kv_cache_decode_dualcache_b200 import build, fdllm, synth
+    torch.cuda.set_device(0)
+    build.build()
+    shape = wl.shape
+    P, G, B = wl.prompt_len, wl.gen_len, wl.block_size
+    dec = fdllm.Decoder(shape, P + G, device=0)
+    w = synth.make_weights(shape, device="cuda")
+    dec.load_weights(w)
+    del w
+    prompt = synth.make_prompt(shape, P).numpy()
+    x_a = np.concatenate([prompt, np.full(G, shape.mask_id)]).astype(np.int32)
+    r = dec.step_debug(x_a, x_a, P, B, wl.tau, "dual", logits=False)
+    x_b = x_a.copy()
+    x_b[P:P + B][r["unmask"]] = r["tok"][r["unmask"]]
+    dec.kv_similarity(x_a, x_b)  # warm-up (allocates the cache copy)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    cos = dec.kv_similarity(x_a, x_b)
+    ms = (time.perf_counter() - t0) * 1e3
+    reused = np.r_[0:P, P + B:P + G]
+    layers = [{"layer": li,
+               "k_min": round(float(cos[li, 0, reused].min()), 6),
+               "k_mean": round(float(cos[li, 0, reused].mean()), 6),
+               "v_min": round(float(cos[li, 1, reused].min()), 6),
+               "v_mean": round(float(cos[li, 1, reused].mean()), 6)} for li in range(shape.n_layers)]
+    line = {"metric": f"K/V cosine similarity, block start vs after its first step ({wl.name})",
+            "unit": "cosine", "unmasked_by_the_step": int(r["unmask"].sum()),
+            "positions_reused": int(reused.size), "call_ms": round(ms, 2),
+            "data": "synthetic (random N(0,0.02) weights)", "layers": layers}
+    print(json.dumps(line), flush=True)
+    dec.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -494,6 +554,8 @@ def main():
     ap.add_argument("--cache-mode", default=None, choices=["none", "prefix", "dual"],
                     help="override the workload's cache mode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-similarity", action="store_true",
+                    help="print the K/V similarity diagnostic for the workload instead")
     ap.add_argument("--ref-cached-steps", type=int, default=18,
                     help="cached steps per generation assumed by the reference arm")
     args = ap.parse_args()
@@ -505,6 +567,8 @@ def main():
                                  cache_mode=args.cache_mode or wl.cache_mode)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.kv_similarity:
+        return run_kv_similarity(args, wl)
     if wl.batch > 1:
         return run_fdllm_batch(args, wl)
     return run_fdllm(args, wl)

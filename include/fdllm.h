@@ -225,6 +225,25 @@ FDLLM_API int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, cons
                      int L, int block_start, int block_size, float tau, int cache_mode,
                      float* logits, float* conf, int32_t* tok, uint8_t* unmask);
 
+/* Similarity of the K/V activations of two token sequences (diagnostic).
+ * The approximate block cache rests on the observation that the K/V
+ * activations of adjacent denoising steps are nearly identical (cosine
+ * similarity close to 1): ccyt168.com Fast-dLLM overview, section 一
+ * "核心技术", item 1 (双向缓存策略 / 高相似度验证, Fig. 2), and the
+ * techwalker.com Fast-dLLM article, section "核心创新：适合扩散模型的KV缓存".
+ * This call measures it for the loaded weights: a full forward over ids_a
+ * (e.g. the sequence at the block start, whose K/V a DualCache step reuses)
+ * and one over ids_b (e.g. the sequence some steps later), both of L tokens,
+ * then writes cos_out[(layer * 2 + kv) * L + pos] (caller-owned, 2 *
+ * n_layers * L doubles): the cosine of the two sequences' K (kv = 0) or V
+ * (kv = 1) at that layer and position, over its n_kv_heads * head_dim
+ * values (float64 accumulation; 1 for two zero vectors).  The first call
+ * allocates a device copy of the K/V cache.  Leaves the cache holding
+ * ids_b's K/V.  Errors: ARG (NULL, L out of range, id out of range), STATE
+ * (no weights), OOM, CUDA. */
+FDLLM_API int fdllm_kv_similarity(fdllm_ctx* ctx, const int32_t* ids_a, const int32_t* ids_b,
+                                  int L, double* cos_out);
+
 /* Copy K and V of one layer for positions [pos0, pos0 + n) from the cache to
  * host float buffers k_out, v_out ([n, n_kv_heads, head_dim] each).  Used to
  * check that the cache after a refresh equals a full recompute.  Errors: ARG

@@ -86,6 +86,8 @@ struct fdllm_ctx {
   CUtensorMap m_head;
 
   void* kv_pool = nullptr;
+  void* kv_snap = nullptr;          // fdllm_kv_similarity: copy of the K/V pool
+  double* kv_cos = nullptr;         // fdllm_kv_similarity: [n_layers][2][max_seq] cosines
   int kv_planes = 2;        // fp32: K, V; bf16: K hi, K lo, V hi, V lo
   int n_pages = 0;
   size_t q_plane = 0;       // elements per q plane (bf16 two-term q)
@@ -1422,6 +1424,42 @@ int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, const int32_t*
   CK(cudaMemcpy(tok, ctx->tok, sizeof(int32_t) * B, cudaMemcpyDeviceToHost));
   CK(cudaMemcpy(unmask, ctx->unmask, B, cudaMemcpyDeviceToHost));
   if (logits) CK(cudaMemcpy(logits, dbg, sizeof(float) * B * c.vocab, cudaMemcpyDeviceToHost));
+  return FDLLM_OK;
+}
+
+int fdllm_kv_similarity(fdllm_ctx* ctx, const int32_t* ids_a, const int32_t* ids_b, int L,
+                        double* cos_out) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  if (!ctx->weights_loaded) return fail(ctx, FDLLM_ERR_STATE, "weights are not loaded");
+  const fdllm_config& c = ctx->cfg;
+  if (!ids_a || !ids_b || !cos_out) return fail(ctx, FDLLM_ERR_ARG, "NULL argument");
+  if (L < 1 || L > c.max_seq) return fail(ctx, FDLLM_ERR_ARG, "bad L");
+  for (int i = 0; i < L; ++i)
+    if (ids_a[i] < 0 || ids_a[i] >= c.vocab || ids_b[i] < 0 || ids_b[i] >= c.vocab)
+      return fail(ctx, FDLLM_ERR_ARG, "token id out of range");
+  CK(cudaSetDevice(ctx->device));
+  const size_t kv_bytes = ctx->cap_kv * ctx->esz;
+  if (!ctx->kv_snap) {
+    ctx->kv_snap = dalloc(ctx, kv_bytes);
+    ctx->kv_cos = (double*)dalloc(ctx, sizeof(double) * 2 * c.n_layers * c.max_seq);
+    if (!ctx->kv_snap || !ctx->kv_cos)
+      return fail(ctx, FDLLM_ERR_OOM, "similarity scratch allocation failed");
+  }
+  // a full forward over each sequence writes the K/V of every position
+  int rc, n_part = 0;
+  CK(cudaMemsetAsync(ctx->state, 0, sizeof(DecodeState), ctx->stream));
+  CK(cudaMemcpyAsync(ctx->x, ids_a, sizeof(int32_t) * L, cudaMemcpyHostToDevice, ctx->stream));
+  if ((rc = set_step_params(ctx, 0, 0, 0, 1.0f))) return rc;
+  if ((rc = forward(ctx, 0, L, L, 0, 1, nullptr, &n_part))) return rc;
+  CK(cudaMemcpyAsync(ctx->kv_snap, ctx->kv_pool, kv_bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+  CK(cudaMemcpyAsync(ctx->x, ids_b, sizeof(int32_t) * L, cudaMemcpyHostToDevice, ctx->stream));
+  if ((rc = forward(ctx, 0, L, L, 0, 1, nullptr, &n_part))) return rc;
+  KL(launch_kv_cosine(ctx->kv_snap, ctx->kv_pool, ctx->page_table, ctx->n_pages, ctx->kv_planes,
+                      c.n_layers, c.n_kv_heads, c.head_dim, ctx->f32 ? 1 : 0, L, ctx->kv_cos,
+                      ctx->stream));
+  if ((rc = sync_state(ctx))) return rc;
+  CK(cudaMemcpy(cos_out, ctx->kv_cos, sizeof(double) * 2 * c.n_layers * L,
+                cudaMemcpyDeviceToHost));
   return FDLLM_OK;
 }
 

@@ -229,6 +229,12 @@ struct DecodeState {
   int pad;
 };
 
+// out[(layer * 2 + kv) * L + pos], pos < L: cosine of K (kv = 0) / V (kv = 1)
+// of cache a and cache b (same paged layout and page table), float64.
+cudaError_t launch_kv_cosine(const void* a, const void* b, const int* page_table, int n_pages,
+                             int planes, int n_layers, int Hkv, int hd, int f32, int L,
+                             double* out, cudaStream_t st);
+
 // Merge LM-head partials into conf/tok for n rows and, when select != 0,
 // apply the threshold-or-fallback unmask rule to x[s .. s+n).
 // With sp, s = sp->s and tau = sp->tau.

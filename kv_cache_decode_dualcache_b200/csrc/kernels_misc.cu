@@ -189,6 +189,64 @@ __global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__
   }
 }
 
+// ------------------------------------------------------- K/V similarity
+// out[(layer * 2 + kv) * L + pos] = cosine of the K (kv = 0) or V (kv = 1)
+// activations of one position and layer in two caches of the same layout,
+// over its n_kv_heads * head_dim values (two-term fp16 terms summed for the
+// bf16 model), accumulated in float64 in a fixed order.  One CTA per
+// (position, kv, layer).
+__global__ void __launch_bounds__(128) kv_cosine_kernel(const void* __restrict__ a,
+                                                        const void* __restrict__ b,
+                                                        const int* __restrict__ page_table,
+                                                        int n_pages, int planes, int Hkv, int hd,
+                                                        int f32, int L, double* __restrict__ out) {
+  __shared__ double red[3][4];
+  const int pos = blockIdx.x, kv = blockIdx.y, layer = blockIdx.z;
+  const int page = page_table[pos / KV_PAGE], slot = pos % KV_PAGE;
+  const size_t plane_elems = (size_t)Hkv * KV_PAGE * hd;
+  const size_t base = ((size_t)layer * n_pages + page) * planes * plane_elems;
+  double dot = 0.0, na = 0.0, nb = 0.0;
+  for (int i = threadIdx.x; i < Hkv * hd; i += blockDim.x) {
+    const int h = i / hd, d = i - h * hd;
+    const size_t off = (size_t)h * KV_PAGE * hd + (size_t)slot * hd + d;
+    double x, y;
+    if (f32) {
+      const size_t e = base + (size_t)kv * plane_elems + off;
+      x = reinterpret_cast<const float*>(a)[e];
+      y = reinterpret_cast<const float*>(b)[e];
+    } else {
+      const size_t hi = base + (size_t)(2 * kv) * plane_elems + off, lo = hi + plane_elems;
+      const __half* ha = reinterpret_cast<const __half*>(a);
+      const __half* hb = reinterpret_cast<const __half*>(b);
+      x = (double)__half2float(ha[hi]) + (double)__half2float(ha[lo]);
+      y = (double)__half2float(hb[hi]) + (double)__half2float(hb[lo]);
+    }
+    dot += x * y;
+    na += x * x;
+    nb += y * y;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    na += __shfl_xor_sync(0xffffffffu, na, o);
+    nb += __shfl_xor_sync(0xffffffffu, nb, o);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = dot;
+    red[1][w] = na;
+    red[2][w] = nb;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s[3];
+    for (int q = 0; q < 3; ++q) s[q] = ((red[q][0] + red[q][1]) + red[q][2]) + red[q][3];
+    // two zero vectors are identical; a zero and a non-zero one are not alike
+    const double den = sqrt(s[1]) * sqrt(s[2]);
+    out[((size_t)layer * 2 + kv) * L + pos] =
+        den > 0.0 ? s[0] / den : ((s[1] == 0.0 && s[2] == 0.0) ? 1.0 : 0.0);
+  }
+}
+
 // ------------------------------------------------------- merge + select
 __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
                                     int mask_id, float tau, int select, float* conf, int* tok,
@@ -427,6 +485,15 @@ cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
                   (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
                   (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+}
+
+cudaError_t launch_kv_cosine(const void* a, const void* b, const int* page_table, int n_pages,
+                             int planes, int n_layers, int Hkv, int hd, int f32, int L,
+                             double* out, cudaStream_t st) {
+  if (L < 1 || n_layers < 1 || Hkv < 1 || hd < 1) return cudaErrorInvalidValue;
+  kv_cosine_kernel<<<dim3(L, 2, n_layers), 128, 0, st>>>(a, b, page_table, n_pages, planes, Hkv,
+                                                          hd, f32, L, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x, int s,

@@ -29,7 +29,7 @@ DTYPES = {"fp32": 0, "bf16": 1}
 
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
             "fdllm_generate_batch", "fdllm_generate_fixed_k",
-            "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention",
+            "fdllm_step_debug", "fdllm_read_kv", "fdllm_kv_similarity", "fdllm_gemm", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
             "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
 
@@ -106,6 +106,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                      i32, P(ctypes.c_float), P(ctypes.c_float),
                                      P(ctypes.c_int32), P(ctypes.c_uint8)]
     lib.fdllm_read_kv.argtypes = [vp, i32, i32, i32, P(ctypes.c_float), P(ctypes.c_float)]
+    lib.fdllm_kv_similarity.argtypes = [vp, P(ctypes.c_int32), P(ctypes.c_int32), i32,
+                                        P(ctypes.c_double)]
     lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32]
     lib.fdllm_attention.argtypes = [vp, vp, vp, i32, i32, i32]
     lib.fdllm_gemm_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
@@ -117,7 +119,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_launch_count.restype = ctypes.c_int64
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
-                 "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv",
+                 "fdllm_kv_similarity", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
                  "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -284,6 +287,20 @@ def fdllm_read_kv(ctx, layer: int, pos0: int, n: int, n_kv_heads: int, head_dim:
     return k, v
 
 
+def fdllm_kv_similarity(ctx, ids_a, ids_b, n_layers: int):
+    """Cosines [n_layers, 2 (K, V), L] of the two sequences' K/V activations
+    (full forward over each; see the header)."""
+    lib = load_library()
+    a = np.ascontiguousarray(np.asarray(ids_a, dtype=np.int32))
+    b = np.ascontiguousarray(np.asarray(ids_b, dtype=np.int32))
+    if a.shape != b.shape or a.ndim != 1:
+        raise ValueError("ids_a and ids_b must be 1-D sequences of the same length")
+    out = np.empty((n_layers, 2, a.size), dtype=np.float64)
+    _check(lib.fdllm_kv_similarity(ctx, _i32_ptr(a), _i32_ptr(b), int(a.size),
+                                   out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))), ctx)
+    return out
+
+
 def _pair_rows(m: int) -> int:
     return 2 * ((m + 31) // 32) * 32
 
@@ -425,6 +442,9 @@ class Decoder:
                    tau: float, cache_mode="dual", logits: bool = True):
         return fdllm_step_debug(self.ctx, snapshot_ids, current_ids, block_start, block_size, tau,
                                 cache_mode, self.shape.vocab if logits else None)
+
+    def kv_similarity(self, ids_a, ids_b):
+        return fdllm_kv_similarity(self.ctx, ids_a, ids_b, self.shape.n_layers)
 
     def read_kv(self, layer: int, pos0: int, n: int):
         return fdllm_read_kv(self.ctx, layer, pos0, n, self.shape.n_kv_heads, self.shape.head_dim)

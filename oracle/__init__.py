@@ -32,6 +32,8 @@ Modules:
                   the teacher-forced single step.
 * ``theorem``   - a toy "model" built from an explicit joint table, used to
                   check the (n+1)·eps <= 1 statement by brute force.
+* ``similarity``- cosine similarity of two steps' K/V activations per layer
+                  and position (the diagnostic behind the approximate cache).
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against closed forms, independent library routines (torch CPU float64),
