@@ -962,7 +962,6 @@ GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_
   // keep that near -4e-7, the level of a plain float32 dot product; the
   // epilogue warps sum the chains with round-to-nearest float32 adds.
   g.kc = nt == 256 ? 16 : 8;
-  if (const char* kc = std::getenv("FDLLM_KC_EXPERIMENT")) g.kc = std::atoi(kc);
   return g;
 }
 
