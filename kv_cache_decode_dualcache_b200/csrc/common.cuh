@@ -445,6 +445,15 @@ FD_DEV void ld_cluster_v4(uint32_t addr, float* v) {
 }
 
 // Named barrier among `count` threads (a multiple of 32).
+// Atomic add at gpu scope with acquire-release semantics: releases the
+// writes ordered before it (after a CTA barrier, the whole CTA's) and
+// acquires those released by the earlier additions, in one instruction.
+FD_DEV int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 FD_DEV void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
