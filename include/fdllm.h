@@ -244,6 +244,18 @@ FDLLM_API int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, cons
 FDLLM_API int fdllm_kv_similarity(fdllm_ctx* ctx, const int32_t* ids_a, const int32_t* ids_b,
                                   int L, double* cos_out);
 
+/* Failure-path self-test.  Every device-side wait of the library (TMA and
+ * MMA barriers, the block-step kernel's phase and row waits) is bounded: a
+ * wait that runs past its limit (2 s) records a timeout in the context's
+ * device error word and its kernel returns, and the call that launched it
+ * returns FDLLM_ERR_TIMEOUT.  This call runs one wait that nothing can
+ * complete through that same bounded wait and returns what a real timeout
+ * returns: FDLLM_ERR_TIMEOUT, after about 2 s, with the error word cleared
+ * and the context still usable.  No fault, trap or hang is involved.  The
+ * pages have no counterpart; it tests the library's own failure detection.
+ * Errors: ARG (NULL ctx), CUDA. */
+FDLLM_API int fdllm_selftest_wait_timeout(fdllm_ctx* ctx);
+
 /* Copy K and V of one layer for positions [pos0, pos0 + n) from the cache to
  * host float buffers k_out, v_out ([n, n_kv_heads, head_dim] each).  Used to
  * check that the cache after a refresh equals a full recompute.  Errors: ARG

@@ -1426,6 +1426,13 @@ int fdllm_step_debug(fdllm_ctx* ctx, const int32_t* snapshot_ids, const int32_t*
   return FDLLM_OK;
 }
 
+int fdllm_selftest_wait_timeout(fdllm_ctx* ctx) {
+  if (!ctx) return FDLLM_ERR_ARG;
+  CK(cudaSetDevice(ctx->device));
+  KL(launch_wait_timeout(ctx->err_dev, ctx->stream));
+  return sync_state(ctx);  // DEV_ERR_TIMEOUT -> FDLLM_ERR_TIMEOUT; clears the error word
+}
+
 int fdllm_kv_similarity(fdllm_ctx* ctx, const int32_t* ids_a, const int32_t* ids_b, int L,
                         double* cos_out) {
   if (!ctx) return FDLLM_ERR_ARG;

@@ -229,6 +229,9 @@ struct DecodeState {
   int pad;
 };
 
+// A bounded device wait that runs out (see fdllm_selftest_wait_timeout).
+cudaError_t launch_wait_timeout(int* err, cudaStream_t st);
+
 // out[(layer * 2 + kv) * L + pos], pos < L: cosine of K (kv = 0) / V (kv = 1)
 // of cache a and cache b (same paged layout and page table), float64.
 cudaError_t launch_kv_cosine(const void* a, const void* b, const int* page_table, int n_pages,

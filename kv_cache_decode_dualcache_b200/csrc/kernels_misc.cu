@@ -189,6 +189,20 @@ __global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__
   }
 }
 
+// ------------------------------------------------------- failure path
+// One wait that nothing completes (an mbarrier expecting an arrival that no
+// thread makes), through the same bounded mbar_wait the tcgen05 kernels use:
+// after its limit it records DEV_ERR_TIMEOUT in the error word and returns.
+__global__ void wait_timeout_kernel(int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, err, nullptr);
+}
+
 // ------------------------------------------------------- K/V similarity
 // out[(layer * 2 + kv) * L + pos] = cosine of the K (kv = 0) or V (kv = 1)
 // activations of one position and layer in two caches of the same layout,
@@ -485,6 +499,11 @@ cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
                   (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
                   (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+}
+
+cudaError_t launch_wait_timeout(int* err, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 32, 0, st>>>(err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_kv_cosine(const void* a, const void* b, const int* page_table, int n_pages,

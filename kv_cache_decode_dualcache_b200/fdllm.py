@@ -29,7 +29,8 @@ DTYPES = {"fp32": 0, "bf16": 1}
 
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
             "fdllm_generate_batch", "fdllm_generate_fixed_k",
-            "fdllm_step_debug", "fdllm_read_kv", "fdllm_kv_similarity", "fdllm_gemm", "fdllm_attention",
+            "fdllm_step_debug", "fdllm_read_kv", "fdllm_kv_similarity", "fdllm_selftest_wait_timeout",
+            "fdllm_gemm", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
             "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
 
@@ -108,6 +109,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_read_kv.argtypes = [vp, i32, i32, i32, P(ctypes.c_float), P(ctypes.c_float)]
     lib.fdllm_kv_similarity.argtypes = [vp, P(ctypes.c_int32), P(ctypes.c_int32), i32,
                                         P(ctypes.c_double)]
+    lib.fdllm_selftest_wait_timeout.argtypes = [vp]
     lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32]
     lib.fdllm_attention.argtypes = [vp, vp, vp, i32, i32, i32]
     lib.fdllm_gemm_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
@@ -120,7 +122,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
                  "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv",
-                 "fdllm_kv_similarity", "fdllm_gemm", "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_kv_similarity", "fdllm_selftest_wait_timeout", "fdllm_gemm",
+                 "fdllm_attention", "fdllm_gemm_noalloc",
                  "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
