@@ -1,0 +1,64 @@
+"""bench.py's reporting arithmetic, on synthetic profile records (no GPU):
+the dominant kernel class, achieved = algorithmic bytes (FLOPs) / time,
+frac = achieved / peak, the block step against 8 TB/s, and the DRAM
+traffic record of the current chain kernel."""
+import hashlib
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from kv_cache_decode_dualcache_b200 import synth  # noqa: E402
+
+
+def _stat(name, launches, ms, gbytes=0.0, tflop=0.0):
+    return {"name": name, "launches": launches, "total_ms": ms, "bytes": gbytes * 1e9,
+            "flops": tflop * 1e12}
+
+
+def test_hbm_bound_class_dominates():
+    stats = [_stat("chain.step", 33, 100.0, gbytes=300.0),          # 3 TB/s
+             _stat("gemm.qkv.full", 32, 40.0, tflop=20.0),
+             _stat("attn.step", 32, 10.0, gbytes=0.5)]
+    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured", 123.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 3000.0) < 1e-6
+    assert abs(r["frac"] - 0.5) < 1e-9
+    assert r["traffic"] == 123.0 and r["launches"] == 33
+    assert abs(r["share_of_kernel_time"] - 100.0 / 150.0) < 1e-3
+
+
+def test_tensor_bound_class_dominates():
+    stats = [_stat("chain.step", 33, 10.0, gbytes=30.0),
+             _stat("gemm.qkv.full", 32, 40.0, tflop=20.0),
+             _stat("gemm.ffn_up.full", 32, 60.0, tflop=40.0)]
+    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured", 123.0)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 60.0 / 0.1) < 1e-6       # 60 TFLOP in 100 ms
+    assert abs(r["frac"] - 600.0 / 1400.0) < 1e-4
+    assert r["traffic"] is None                          # no capture of this class
+
+
+def test_block_step_roofline_of_the_headline_workload():
+    wl = synth.WORKLOADS["llada8b-p256-g256"]
+    r = bench.block_step_roofline(wl, 4.0, 6000.0)
+    # weights of one block step (bf16) + K and V of all 512 positions
+    want = 2 * synth.step_weight_params(wl.shape) + 32 * 512 * 32 * 128 * 2 * 2
+    assert r["bytes_per_step"] == want
+    assert abs(r["frac_of_8TBps"] - want / 4e-3 / 8e12) < 1e-4
+    assert abs(r["frac_of_measured"] - want / 4e-3 / 6e12) < 1e-4
+
+
+def test_traffic_record_follows_the_chain_kernel_source():
+    path = os.path.join(ROOT, "profiles", "chain_traffic.txt")
+    rec = dict(l.split(":", 1) for l in open(path) if ":" in l and not l.startswith("#"))
+    src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", "chain.cu"),
+               "rb").read()
+    got = bench._traffic_record()
+    if rec["chain_sha256"].strip() == hashlib.sha256(src).hexdigest():
+        assert got == float(rec["bytes_per_launch"])
+    else:                       # kernel changed since the counters were taken
+        assert got is None
