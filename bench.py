@@ -264,10 +264,23 @@ def run_reference(args, wl):
         if i >= args.warmup:
             vals.append(r)
     v = sum(r["tok_s"] for r in vals) / len(vals)
+    sample_s = [round(r["sample_s"], 3) for r in vals]
     line = {"impl": "reference", "metric": metric_name(wl), "value": v, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            # an estimate: each "step" times one bounded sample, not a whole
+            # generation; ms_per_step is the estimated time of one generation
             "ms_per_step": 1e3 * wl.gen_len / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "estimated": True,
+            "estimate": {"measured_sample_seconds": sample_s,
+                         "timed_region_seconds": round(sum(sample_s), 3),
+                         "layers_run": sample_layers, "layers_model": wl.shape.n_layers,
+                         "layer_scale": wl.shape.n_layers / sample_layers,
+                         "refresh_steps_per_generation": counts[0],
+                         "cached_steps_per_generation": counts[1],
+                         "step_counts_from": "the GPU decoder's schedule on this workload "
+                                             "(--ref-cached-steps; the float64 oracle cannot "
+                                             "run the whole generation in minutes)"},
             "config": _config(wl, 1),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["threads"],
                              "kind": "oracle",
@@ -420,10 +433,10 @@ def run_fdllm(args, wl):
 
 def run_fdllm_batch(args, wl):
     """Variable-length batch (independent sequences, per-sequence block
-    schedules) through fdllm_generate_batch; value = generated tokens of the
-    whole batch per second of device time (host prompts in, tokens out: the
-    batched entry point is host-buffer only, so value and e2e time the same
-    call)."""
+    schedules, one shared weight stream per global step) through
+    fdllm_generate_batch; value = generated tokens of the whole batch per
+    second of device time (host prompts in, tokens out: the batched entry
+    point is host-buffer only, so value and e2e time the same call)."""
     import numpy as np
     import torch
     from kv_cache_decode_dualcache_b200 import build, fdllm, synth
@@ -445,7 +458,8 @@ def run_fdllm_batch(args, wl):
     lens = synth.make_batch_prompt_lengths(wl.batch)
     prompts = [synth.make_prompt(shape, n, salt=rank * 1000 + i).numpy() for i, n in enumerate(lens)]
     stream = torch.cuda.Stream()
-    dec = fdllm.Decoder(shape, max(lens) + G, device=local, stream=stream.cuda_stream)
+    dec = fdllm.Decoder(shape, max(lens) + G, device=local, stream=stream.cuda_stream,
+                        max_batch=wl.batch)
     w = synth.make_weights(shape, device="cuda")
     dec.load_weights(w)
     del w
@@ -479,7 +493,9 @@ def run_fdllm_batch(args, wl):
         cfg = _config(wl, world)
         cfg.update({"prompt_lens": lens, "batch_per_gpu": wl.batch,
                     "global_batch": wl.batch * world,
-                    "batching": "sequences run in turn through the single-sequence path"})
+                    "batching": f"continuous batching over {wl.batch} sequence slots: one "
+                                "forward per global step over every active sequence's rows "
+                                "(shared weight stream)"})
         line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
@@ -541,6 +557,29 @@ def run_kv_similarity(args, wl):
     return 0
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_replicas(n: int, argv, script: str = None, timeout_s: float = 3600.0) -> int:
+    """Run `script argv` as n ranks of one node under torch.distributed.run
+    (rendezvous on 127.0.0.1), passing their output through; returns the
+    launcher's exit code.  bench.py uses it when --gpus N > 1 is given without
+    a launcher around it."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={_free_port()}",
+           script or os.path.abspath(__file__)] + list(argv)
+    try:
+        return subprocess.run(cmd, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        print(f"bench.py: the {n} replica ranks did not finish within {timeout_s:.0f} s",
+              file=sys.stderr)
+        return 124
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -559,6 +598,13 @@ def main():
     ap.add_argument("--ref-cached-steps", type=int, default=18,
                     help="cached steps per generation assumed by the reference arm")
     args = ap.parse_args()
+    world_env = os.environ.get("WORLD_SIZE")
+    if args.gpus > 1 and world_env is None:
+        # no launcher around this process: start the N replica ranks here
+        return launch_replicas(args.gpus, sys.argv[1:])
+    if world_env is not None and int(world_env) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}", file=sys.stderr)
+        return 2
     from kv_cache_decode_dualcache_b200 import synth
     wl = synth.WORKLOADS[args.workload]
     if args.tau is not None or args.cache_mode is not None:

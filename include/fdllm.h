@@ -85,7 +85,7 @@ typedef enum {
 /* Model shape and numerics.  Requirements (FDLLM_ERR_ARG otherwise):
  * n_layers >= 1; d_model, ffn_dim and n_heads*head_dim multiples of 64;
  * head_dim in {32, 64, 128}; n_heads a multiple of n_kv_heads;
- * 0 <= mask_id < vocab; vocab >= 2; max_seq >= 1; max_batch == 1. */
+ * 0 <= mask_id < vocab; vocab >= 2; max_seq >= 1; 1 <= max_batch <= 64. */
 typedef struct {
   int32_t n_layers;
   int32_t d_model;
@@ -99,7 +99,8 @@ typedef struct {
   float rms_eps;       /* RMSNorm: h / sqrt(mean(h^2) + eps) * g */
   float logit_scale;   /* z = logit_scale * (RMSNorm(h) W_head^T) */
   int32_t dtype;       /* fdllm_dtype */
-  int32_t max_batch;   /* sequences per call; only 1 is supported */
+  int32_t max_batch;   /* sequence slots: sequences fdllm_generate_batch decodes at once
+                          (each slot holds a K/V cache of max_seq positions) */
   int32_t max_seq;     /* largest prompt_len + gen_len */
 } fdllm_config;
 
@@ -141,6 +142,20 @@ typedef struct {
   int32_t collect_timing;   /* in: 1 = time each step with CUDA events */
   double refresh_ms;        /* out (timing only): summed time of full-forward steps */
   double cached_ms;         /* out (timing only): summed time of cached steps */
+  /* Optional per-step trace (in: caller-owned host arrays, trace_cap > 0 to
+   * enable; filled by fdllm_generate, fdllm_generate_device and
+   * fdllm_generate_fixed_k, not by fdllm_generate_batch).  For denoising step
+   * i < trace_cap of the generation: trace_block[i] = its block index and,
+   * for row j < block_size of that block, trace_conf[i * block_size + j] =
+   * the confidence, trace_tok[...] = the argmax token and trace_unmask[...]
+   * = 1 when the step unmasked the row.  Steps beyond trace_cap are not
+   * recorded.  The values are read back after each step from the buffers the
+   * step's own kernels wrote, so the trace does not change the launches. */
+  int32_t trace_cap;
+  int32_t* trace_block;
+  float* trace_conf;
+  int32_t* trace_tok;
+  uint8_t* trace_unmask;
 } fdllm_stats;
 
 /* Create a decoder context on CUDA device `device`.  cuda_stream is a
@@ -159,6 +174,13 @@ FDLLM_API int fdllm_create(const fdllm_config* cfg, int device, void* cuda_strea
  * inputs.  Errors: SHAPE (unknown/missing/duplicate name, wrong numel or
  * dtype), OOM, CUDA. */
 FDLLM_API int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensors);
+
+/* Number of GEMM weights of the bf16 model whose conversion to fp16 at
+ * fdllm_load_weights was not exact (non-zero bf16 values below 2^-17 in
+ * magnitude, where the fp16 grid spacing is 2^-24; each such weight is off by
+ * at most 2^-25).  0 for the fp32 model or before weights are loaded.
+ * Returns -1 for a NULL ctx. */
+FDLLM_API int64_t fdllm_inexact_weight_count(const fdllm_ctx* ctx);
 
 /* Generate gen_len tokens after prompt_ids (host, prompt_len ids) with block
  * size block_size, threshold tau and cache mode cache_mode; writes the
@@ -195,17 +217,31 @@ FDLLM_API int fdllm_generate_fixed_k(fdllm_ctx* ctx, const int32_t* prompt_ids, 
 /* Variable-length batch: `batch` independent sequences, prompts[i] (host)
  * holding prompt_lens[i] ids, each generating gen_len tokens with the same
  * block size, tau and cache mode on its own block schedule (its blocks start
- * at its own prompt end).  out_tokens (host, caller-owned, batch * gen_len)
- * receives sequence i's tokens at [i * gen_len, (i + 1) * gen_len);
+ * at its own prompt end; the readings of the block procedure are those of
+ * fdllm_generate, per sequence).  out_tokens (host, caller-owned, batch *
+ * gen_len) receives sequence i's tokens at [i * gen_len, (i + 1) * gen_len);
  * out_steps (host, batch) its step counts; stats (optional) the totals over
- * the batch, with steps_per_block (when not NULL) holding batch * gen_len /
- * block_size entries, sequence by sequence.  Results equal fdllm_generate on
- * each sequence alone.  The sequences run one after another through the
- * single-sequence path (each step streams the weights for one sequence):
- * this entry point fixes the batched interface, not a kernel path that
- * shares the weight stream across sequences.  Every sequence's arguments are
- * checked before any work (errors as fdllm_generate; ARG for batch < 1 or
- * NULL arrays). */
+ * the batch (refresh_steps / cached_steps count sequence steps; with timing,
+ * refresh_ms sums the global steps that held a full forward, cached_ms the
+ * others), with steps_per_block (when not NULL) holding batch * gen_len /
+ * block_size entries, sequence by sequence, and the trace (when trace_cap >
+ * 0) of sequence i's step k at index i * trace_cap + k.
+ *
+ * With max_batch > 1 the sequences share the weight stream: up to max_batch
+ * of them occupy the context's slots at once, and every global step runs ONE
+ * forward over the rows all of them need (a full forward for a sequence at a
+ * block start, or every step with the cache off; its block rows in a
+ * DualCache step; rows [s, L) in a prefix-cache step), with per-row RoPE
+ * positions and K/V destinations, attention per sequence over its own cache
+ * pages, and the unmask rule per sequence.  A sequence that finishes frees
+ * its slot for the next waiting one (continuous batching).  Each sequence's
+ * decode is the single-sequence algorithm; its results equal fdllm_generate
+ * on it alone up to the rounding of the batched GEMM's reduction order (the
+ * fp32 model's kernels sum in a fixed order per output, so there they are
+ * identical).  With max_batch == 1 the sequences run one after another
+ * through the single-sequence path.  Every sequence's arguments are checked
+ * before any work (errors as fdllm_generate; ARG for batch < 1 or NULL
+ * arrays). */
 FDLLM_API int fdllm_generate_batch(fdllm_ctx* ctx, int batch, const int32_t* const* prompts,
                                    const int* prompt_lens, int gen_len, int block_size, float tau,
                                    int cache_mode, int32_t* out_tokens, int* out_steps,

@@ -38,6 +38,8 @@ constexpr int kMaxLmRows = 256;
 constexpr int kMaxAttnSplit = 8;   // key splits = CTAs of one thread-block cluster
 constexpr int kAttnSplitMaxM = 64;
 constexpr int kSpRing = 8;
+constexpr int kMaxBatch = 64;      // sequence slots of a context
+constexpr int kMaxLmChunk = 512;   // LM-head rows per launch of a batched step
 
 thread_local std::string g_create_error = "no error";
 
@@ -89,7 +91,9 @@ struct fdllm_ctx {
   void* kv_snap = nullptr;          // fdllm_kv_similarity: copy of the K/V pool
   double* kv_cos = nullptr;         // fdllm_kv_similarity: [n_layers][2][max_seq] cosines
   int kv_planes = 2;        // fp32: K, V; bf16: K hi, K lo, V hi, V lo
-  int n_pages = 0;
+  int n_pages = 0;          // pages per layer over every sequence slot
+  int pages_per_seq = 0;    // slot q owns pages [q * pages_per_seq, (q + 1) * pages_per_seq)
+  int rows_cap = 0;         // forward rows the activation buffers hold (max_batch * max_seq)
   size_t q_plane = 0;       // elements per q plane (bf16 two-term q)
   int* page_table = nullptr;
   float2* rope = nullptr;
@@ -113,13 +117,27 @@ struct fdllm_ctx {
   DecodeState* state_host = nullptr;
   int* err_dev = nullptr;
   int* err_host = nullptr;
+  unsigned long long* inexact_dev = nullptr;  // bf16 -> fp16 weight conversions that changed a value
+  int64_t inexact_weights = 0;
   int* check = nullptr;        // self-check record (FDLLM_CHECKS builds)
   size_t cap_h = 0, cap_q = 0, cap_kv = 0, cap_f = 0;
   CUtensorMap m_a[3], m_o[3], m_f[3];
+  // tcgen05 attention of many-query forwards: q (3-D, hi plane then lo
+  // plane) and K/V pool (2-D, one row per (layer, page, plane, head, slot))
+  CUtensorMap m_q3, m_kv;
+  bool use_attn_tc = true;
   std::map<std::tuple<int, int, int, int>, GemmShape> plans;
   int64_t launches = 0;
   bool pdl = true;              // programmatic dependent launch between kernels
   bool graphs = true;           // replay each step kind from a captured CUDA graph
+  // batched decode (fdllm_generate_batch): per-slot decode states and the
+  // per-step row / tile / select tables (one device buffer, one pinned
+  // staging copy, one upload per step)
+  DecodeState* states = nullptr;
+  DecodeState* states_host = nullptr;
+  uint8_t* btab = nullptr;
+  uint8_t* btab_host = nullptr;
+  size_t btab_bytes = 0;
   StepParams* sp = nullptr;     // device step scalars (read by the kernels)
   StepParams* sp_host = nullptr;  // pinned ring of kSpRing slots: a pending async copy
   int sp_slot = 0;                // never reads a slot overwritten after it was queued
@@ -275,6 +293,22 @@ bool make_map(fdllm_ctx* ctx, CUtensorMap* m, const void* base, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+// q planes [2 * rows][heads][hd] (hi plane rows, then lo plane rows) as a
+// 3-D map with boxes of {64 dims, rep heads, 128 / rep positions}.
+bool make_q_map(fdllm_ctx* ctx, CUtensorMap* m, const void* q, uint64_t rows_per_plane) {
+  const fdllm_config& c = ctx->cfg;
+  const int rep = c.n_heads / c.n_kv_heads;
+  if (rep < 1 || rep > 128) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)c.head_dim, (cuuint64_t)c.n_heads, 2 * rows_per_plane};
+  cuuint64_t strides[2] = {(cuuint64_t)c.head_dim * 2, (cuuint64_t)c.n_heads * c.head_dim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rep, (cuuint32_t)(128 / rep)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(q), dims, strides,
+                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int check_config(const fdllm_config* c, std::string* why) {
   auto bad = [&](const char* m) { *why = m; return FDLLM_ERR_ARG; };
   if (!c) return bad("config is NULL");
@@ -294,7 +328,7 @@ int check_config(const fdllm_config* c, std::string* why) {
     return bad("the bf16 attention kernel needs head_dim 64 or 128");
   if (c->dtype == FDLLM_DTYPE_BF16 && (c->n_kv_heads * c->head_dim) % 64)
     return bad("n_kv_heads * head_dim must be a multiple of 64");
-  if (c->max_batch != 1) return bad("max_batch must be 1");
+  if (c->max_batch < 1 || c->max_batch > kMaxBatch) return bad("max_batch must be in [1, 64]");
   if (c->max_seq < 1 || c->max_seq > (1 << 20)) return bad("max_seq out of range");
   if (!(c->rms_eps >= 0.0f) || !std::isfinite(c->rope_theta) || !(c->rope_theta > 0.0f) ||
       !std::isfinite(c->logit_scale))
@@ -420,6 +454,26 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   const double qo_bytes = (ctx->f32 ? 2.0 : 4.0) * M * c.n_heads * c.head_dim * es;
   const double att_flops = 4.0 * M * c.n_heads * (double)L * c.head_dim;
   const std::string att_tag = M <= 64 ? "attn.step" : "attn.full";
+  const int rep = c.n_heads / c.n_kv_heads;
+  const int tc_ctas = rep <= 128 ? ((M + 128 / rep - 1) / (128 / rep)) * c.n_kv_heads : 0;
+  if (ctx->tc && ctx->use_attn_tc && M * rep >= 128 &&
+      (M > kAttnSplitMaxM || 2 * tc_ctas >= ctx->num_sms) && attn_tc_supported(ap)) {
+    // many query rows: tcgen05 + TMA attention, one CTA per 128-row query tile
+    // and KV head (block-sized forwards with few such tiles go to the
+    // key-split kernel, which spreads the keys over the SMs)
+    CUtensorMap qm;
+    const CUtensorMap* qmap = &ctx->m_q3;
+    int q_lo_rows = ctx->rows_cap;
+    if (q) {
+      q_lo_rows = M;
+      if (!make_q_map(ctx, &qm, q, (uint64_t)M))
+        return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for q");
+      qmap = &qm;
+    }
+    ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
+    KL(launch_attn_tc(qmap, &ctx->m_kv, ap, q_lo_rows, ctx->err_dev, ctx->stream, ctx->pdl));
+    return FDLLM_OK;
+  }
   if (!ctx->tc) {
     ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
     KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
@@ -429,7 +483,6 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   // head, split) CTAs fill the SMs once, at least 2 key tiles per split
   // (measured: one key tile per split, with two single-buffered CTAs per SM
   // and clusters of 8, is slower).
-  const int rep = c.n_heads / c.n_kv_heads;
   const int rows_per_cta = attn_rows_per_cta(M, c.n_heads, c.n_kv_heads);
   const int ctas = ((M * rep + rows_per_cta - 1) / rows_per_cta) * c.n_kv_heads;
   const int key_tiles = (L + 63) / 64;
@@ -502,6 +555,323 @@ int forward(fdllm_ctx* ctx, int r0, int M, int L, int lm0, int n_lm, float* dbg,
   ep.dbg_logits = dbg;
   return run_gemm(ctx, "lm_head", ctx->lm_head, &ctx->m_head, ctx->a, ctx->m_a, 0, c.vocab, n_lm,
                   d, ep, n_part);
+}
+
+int sync_state(fdllm_ctx* ctx);
+
+// ----------------------------------------------------- batched steps
+// One forward over the rows of several sequences (slots) at once, so every
+// GEMM streams the weights once for all of them.  The host writes the
+// step's tables into ctx->btab: per forward row its position and slot, the
+// attention tiles (each within one sequence, keys [0, L) of that slot), the
+// LM-head rows (each sequence's block rows) and the select segments.
+struct BatchFwd {
+  int M = 0;                       // forward rows
+  const RowInfo* rows = nullptr;   // [M]
+  const AttnTile* tiles = nullptr;
+  int n_tiles = 0;
+  int max_L = 0;
+  const int* lm_src = nullptr;     // [m_lm]: forward row of LM-head row k
+  int m_lm = 0;
+  const SelectSeg* segs = nullptr; // [n_segs], in LM-row order
+  std::vector<std::pair<int, int>> chunks;  // LM-head launches: segments [first, last)
+  std::vector<SelectSeg> host_segs;
+  float tau = 0.0f;
+  int fixed_k = 0;
+};
+
+int run_attention_batched(fdllm_ctx* ctx, int layer, const BatchFwd& bf) {
+  const fdllm_config& c = ctx->cfg;
+  AttnParams ap{};
+  ap.q = ctx->q;
+  ap.q_plane = ctx->q_plane;
+  ap.o = ctx->o;
+  ap.kv_pool = ctx->kv_pool;
+  ap.kv_planes = ctx->kv_planes;
+  ap.page_table = ctx->page_table;
+  ap.n_pages = ctx->n_pages;
+  ap.layer = layer;
+  ap.M = bf.M;
+  ap.L = bf.max_L;
+  ap.n_heads = c.n_heads;
+  ap.n_kv_heads = c.n_kv_heads;
+  ap.head_dim = c.head_dim;
+  ap.n_split = 1;
+  ap.keys_per_split = ((bf.max_L + 63) / 64) * 64;
+  ap.tiles = bf.tiles;
+  ap.n_tiles = bf.n_tiles;
+  ap.pages_per_seq = ctx->pages_per_seq;
+  const double es = (double)ctx->esz;
+  ProfScope ps(ctx, "attn.batch",
+               (double)ctx->kv_planes * bf.max_L * c.n_kv_heads * c.head_dim * es,
+               4.0 * bf.M * c.n_heads * (double)bf.max_L * c.head_dim);
+  if (ctx->tc) KL(launch_attn_mma(ap, ctx->stream, ctx->pdl));
+  else KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
+  return FDLLM_OK;
+}
+
+// The batched forward, then per LM chunk: final norm of its rows, LM head,
+// merge + select of its sequences.
+int forward_batched(fdllm_ctx* ctx, const BatchFwd& bf) {
+  const fdllm_config& c = ctx->cfg;
+  const int d = c.d_model, hq = c.n_heads * c.head_dim, hkv = c.n_kv_heads * c.head_dim;
+  const int nqkv = hq + 2 * hkv;
+  const int M = bf.M;
+  const double es = (double)ctx->esz;
+  const RowMap gather{bf.rows, c.max_seq, nullptr};
+  {
+    ProfScope ps(ctx, "embed_rmsnorm", (double)M * d * (2.0 * es + 4.0), 0.0);
+    KL(launch_embed_rmsnorm(ctx->x, 0, M, ctx->embed, d, c.vocab, ctx->layers[0].attn_norm,
+                            c.rms_eps, ctx->h, ctx->a, ctx->f32, ctx->err_dev, nullptr,
+                            ctx->stream, ctx->pdl, gather));
+  }
+  int rc;
+  for (int l = 0; l < c.n_layers; ++l) {
+    LayerW& lw = ctx->layers[l];
+    EpiParams ep = epi_base(ctx, EPI_QKV);
+    ep.sp = nullptr;
+    ep.pos0 = 0;
+    ep.rows = bf.rows;
+    ep.pages_per_seq = ctx->pages_per_seq;
+    ep.q_out = ctx->q;
+    ep.layer = l;
+    if ((rc = run_gemm(ctx, "qkv", lw.wqkv, &lw.m_qkv, ctx->a, ctx->m_a, 0, nqkv, M, d, ep))) return rc;
+    if ((rc = run_attention_batched(ctx, l, bf))) return rc;
+    ep = epi_base(ctx, EPI_RESID);
+    ep.sp = nullptr;
+    ep.h = ctx->h;
+    if ((rc = run_gemm(ctx, "o", lw.wo, &lw.m_o, ctx->o, ctx->m_o, 0, d, M, hq, ep))) return rc;
+    {
+      ProfScope ps(ctx, "rmsnorm", (double)M * d * (es + 4.0), 0.0);
+      KL(launch_rmsnorm(ctx->h, 0, M, d, lw.ffn_norm, c.rms_eps, ctx->a, ctx->f32, nullptr, false,
+                        ctx->stream, ctx->pdl));
+    }
+    ep = epi_base(ctx, EPI_SWIGLU);
+    ep.sp = nullptr;
+    ep.f_out = ctx->f;
+    if ((rc = run_gemm(ctx, "ffn_up", lw.wgu, &lw.m_gu, ctx->a, ctx->m_a, 0, 2 * c.ffn_dim, M, d, ep)))
+      return rc;
+    ep = epi_base(ctx, EPI_RESID);
+    ep.sp = nullptr;
+    ep.h = ctx->h;
+    if ((rc = run_gemm(ctx, "ffn_down", lw.wd, &lw.m_d, ctx->f, ctx->m_f, 0, d, M, c.ffn_dim, ep)))
+      return rc;
+    if (l + 1 < c.n_layers) {
+      ProfScope ps(ctx, "rmsnorm", (double)M * d * (es + 4.0), 0.0);
+      KL(launch_rmsnorm(ctx->h, 0, M, d, ctx->layers[l + 1].attn_norm, c.rms_eps, ctx->a,
+                        ctx->f32, nullptr, false, ctx->stream, ctx->pdl));
+    }
+  }
+  // LM head per chunk of sequences; partials of chunk j after those of chunks < j
+  size_t part_off = 0;
+  for (const auto& ch : bf.chunks) {
+    const int k0 = bf.host_segs[ch.first].k0;
+    const int k1 = bf.host_segs[ch.second - 1].k0 + bf.host_segs[ch.second - 1].n;
+    const int mc = k1 - k0;
+    {
+      ProfScope ps(ctx, "rmsnorm", (double)mc * d * (es + 4.0), 0.0);
+      KL(launch_rmsnorm(ctx->h, 0, mc, d, ctx->final_norm, c.rms_eps, ctx->a, ctx->f32, nullptr,
+                        false, ctx->stream, ctx->pdl, RowMap{nullptr, 0, bf.lm_src + k0}));
+    }
+    const GemmShape gs = plan_gemm(ctx, c.vocab, mc, d, false, true);
+    if (part_off + (size_t)gs.grid * mc > ctx->lm_part_cap)
+      return fail(ctx, FDLLM_ERR_CUDA, "LM-head partial buffer too small");
+    float* part = reinterpret_cast<float*>(reinterpret_cast<SoftmaxState*>(ctx->lm_part) + part_off);
+    EpiParams ep = epi_base(ctx, EPI_LMHEAD);
+    ep.sp = nullptr;
+    ep.lm_part = part;
+    int n_part = 0;
+    if ((rc = run_gemm(ctx, "lm_head", ctx->lm_head, &ctx->m_head, ctx->a, ctx->m_a, 0, c.vocab, mc,
+                       d, ep, &n_part)))
+      return rc;
+    ProfScope ps(ctx, "merge_select", (double)n_part * mc * 12.0, 0.0);
+    // segment k0 relative to the chunk; conf / tok / unmask by global LM row
+    KL(launch_merge_select_seg(part, n_part, mc, bf.segs + ch.first, ch.second - ch.first, ctx->x,
+                               c.max_seq, c.mask_id, bf.tau, bf.fixed_k, ctx->conf + k0,
+                               ctx->tok + k0, ctx->unmask + k0, ctx->states, ctx->stream,
+                               ctx->pdl));
+    part_off += (size_t)n_part * mc;
+  }
+  return FDLLM_OK;
+}
+
+// Continuous batching over the context's sequence slots: every global step
+// runs one batched forward over all active sequences (each in its own block
+// schedule: a full forward at a block start or with the cache off, the block
+// rows in DualCache steps, rows [s, L) in prefix-cache steps); a sequence
+// that finishes leaves its slot to the next waiting one.
+int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts,
+                        const int* prompt_lens, int G, int B, float tau, int mode, int fixed_k,
+                        int32_t* out_tokens, int* out_steps, fdllm_stats* stats) {
+  const fdllm_config& c = ctx->cfg;
+  const int n_slots = std::min(batch, c.max_batch);
+  const int n_blocks = G / B;
+  const int rep = c.n_heads / c.n_kv_heads;
+  const int rpc = attn_rows_per_cta(-1, c.n_heads, c.n_kv_heads);
+  struct Slot {
+    int seq = -1, P = 0, L = 0, b = 0, nb = 0, steps = 0;
+    bool first = true;
+  };
+  std::vector<Slot> slots(n_slots);
+  int next = 0;
+  CK(cudaSetDevice(ctx->device));
+  auto admit = [&](int q) -> int {
+    Slot& S = slots[q];
+    S = Slot();
+    if (next >= batch) return FDLLM_OK;
+    S.seq = next++;
+    S.P = prompt_lens[S.seq];
+    S.L = S.P + G;
+    int* xq = ctx->x + (size_t)q * c.max_seq;
+    if (S.P > 0)
+      CK(cudaMemcpyAsync(xq, prompts[S.seq], sizeof(int32_t) * S.P, cudaMemcpyHostToDevice,
+                         ctx->stream));
+    KL(launch_fill_masked(xq, S.P, S.L, c.mask_id, ctx->stream));
+    CK(cudaMemsetAsync(ctx->states + q, 0, sizeof(DecodeState), ctx->stream));
+    return FDLLM_OK;
+  };
+  int rc;
+  for (int q = 0; q < n_slots; ++q)
+    if ((rc = admit(q))) return rc;
+  const bool timing = stats && stats->collect_timing;
+  const bool trace = stats && stats->trace_cap > 0;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (timing) {
+    CK(cudaEventCreate(&e0));
+    CK(cudaEventCreate(&e1));
+  }
+  int refresh = 0, cached = 0;
+  double refresh_ms = 0, cached_ms = 0;
+  std::vector<RowInfo> rows;
+  std::vector<AttnTile> tiles;
+  std::vector<int> lm_src;
+  std::vector<float> h_conf;
+  std::vector<int32_t> h_tok;
+  std::vector<uint8_t> h_unmask;
+  for (;;) {
+    BatchFwd bf;
+    bf.tau = tau;
+    bf.fixed_k = fixed_k;
+    rows.clear();
+    tiles.clear();
+    lm_src.clear();
+    bool any_full = false;
+    for (int q = 0; q < n_slots; ++q) {
+      const Slot& S = slots[q];
+      if (S.seq < 0) continue;
+      const int s = S.P + S.b * B;
+      const bool full = S.first || mode == FDLLM_CACHE_NONE;
+      any_full = any_full || full;
+      const int r_lo = full ? 0 : s;
+      const int r_hi = (full || mode == FDLLM_CACHE_PREFIX) ? S.L : s + B;
+      const int q0 = (int)rows.size(), m = r_hi - r_lo;
+      for (int pos = r_lo; pos < r_hi; ++pos) rows.push_back(RowInfo{pos, q});
+      if (ctx->tc) {
+        for (int r0 = 0; r0 < m * rep; r0 += rpc) tiles.push_back(AttnTile{q0, m, r0, S.L, q, {0, 0, 0}});
+      } else {
+        for (int j = 0; j < m; ++j) tiles.push_back(AttnTile{q0 + j, 1, 0, S.L, q, {0, 0, 0}});
+      }
+      bf.max_L = std::max(bf.max_L, S.L);
+      bf.host_segs.push_back(SelectSeg{(int)lm_src.size(), B, q, s});
+      for (int j = 0; j < B; ++j) lm_src.push_back(q0 + (s - r_lo) + j);
+    }
+    if (bf.host_segs.empty()) break;
+    // LM-head chunks of at most kMaxLmChunk rows; select k0 relative to the chunk
+    std::vector<SelectSeg> dev_segs = bf.host_segs;
+    for (int i = 0; i < (int)bf.host_segs.size();) {
+      int j = i, rows_c = 0;
+      while (j < (int)bf.host_segs.size() && rows_c + bf.host_segs[j].n <= kMaxLmChunk)
+        rows_c += bf.host_segs[j++].n;
+      for (int k = i; k < j; ++k) dev_segs[k].k0 -= bf.host_segs[i].k0;
+      bf.chunks.push_back({i, j});
+      i = j;
+    }
+    // one upload of the step's tables
+    auto align = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    const size_t o_rows = 0, o_tiles = align(rows.size() * sizeof(RowInfo));
+    const size_t o_lm = o_tiles + align(tiles.size() * sizeof(AttnTile));
+    const size_t o_seg = o_lm + align(lm_src.size() * sizeof(int));
+    const size_t used = o_seg + dev_segs.size() * sizeof(SelectSeg);
+    if (used > ctx->btab_bytes) return fail(ctx, FDLLM_ERR_CUDA, "batched-step tables too large");
+    std::memcpy(ctx->btab_host + o_rows, rows.data(), rows.size() * sizeof(RowInfo));
+    std::memcpy(ctx->btab_host + o_tiles, tiles.data(), tiles.size() * sizeof(AttnTile));
+    std::memcpy(ctx->btab_host + o_lm, lm_src.data(), lm_src.size() * sizeof(int));
+    std::memcpy(ctx->btab_host + o_seg, dev_segs.data(), dev_segs.size() * sizeof(SelectSeg));
+    CK(cudaMemcpyAsync(ctx->btab, ctx->btab_host, used, cudaMemcpyHostToDevice, ctx->stream));
+    bf.M = (int)rows.size();
+    bf.rows = reinterpret_cast<const RowInfo*>(ctx->btab + o_rows);
+    bf.tiles = reinterpret_cast<const AttnTile*>(ctx->btab + o_tiles);
+    bf.n_tiles = (int)tiles.size();
+    bf.lm_src = reinterpret_cast<const int*>(ctx->btab + o_lm);
+    bf.m_lm = (int)lm_src.size();
+    bf.segs = reinterpret_cast<const SelectSeg*>(ctx->btab + o_seg);
+    if (timing) CK(cudaEventRecord(e0, ctx->stream));
+    if ((rc = forward_batched(ctx, bf))) return rc;
+    if (timing) CK(cudaEventRecord(e1, ctx->stream));
+    CK(cudaMemcpyAsync(ctx->states_host, ctx->states, sizeof(DecodeState) * n_slots,
+                       cudaMemcpyDeviceToHost, ctx->stream));
+    if ((rc = sync_state(ctx))) return rc;  // also the error word
+    if (timing) {
+      float ms = 0;
+      CK(cudaEventElapsedTime(&ms, e0, e1));
+      (any_full ? refresh_ms : cached_ms) += ms;
+    }
+    if (trace) {
+      h_conf.resize(bf.m_lm);
+      h_tok.resize(bf.m_lm);
+      h_unmask.resize(bf.m_lm);
+      CK(cudaMemcpy(h_conf.data(), ctx->conf, sizeof(float) * bf.m_lm, cudaMemcpyDeviceToHost));
+      CK(cudaMemcpy(h_tok.data(), ctx->tok, sizeof(int32_t) * bf.m_lm, cudaMemcpyDeviceToHost));
+      CK(cudaMemcpy(h_unmask.data(), ctx->unmask, bf.m_lm, cudaMemcpyDeviceToHost));
+    }
+    for (const SelectSeg& sg : bf.host_segs) {
+      Slot& S = slots[sg.seq];
+      const DecodeState& st = ctx->states_host[sg.seq];
+      const bool full = S.first || mode == FDLLM_CACHE_NONE;
+      (full ? refresh : cached) += 1;
+      if (trace && S.steps < stats->trace_cap) {
+        const size_t idx = (size_t)S.seq * stats->trace_cap + S.steps;
+        if (stats->trace_block) stats->trace_block[idx] = S.b;
+        if (stats->trace_conf) std::memcpy(stats->trace_conf + idx * B, &h_conf[sg.k0], 4 * B);
+        if (stats->trace_tok) std::memcpy(stats->trace_tok + idx * B, &h_tok[sg.k0], 4 * B);
+        if (stats->trace_unmask) std::memcpy(stats->trace_unmask + idx * B, &h_unmask[sg.k0], B);
+      }
+      S.steps += 1;
+      S.nb += 1;
+      S.first = false;
+      if (st.remaining == 0) {
+        if (stats && stats->steps_per_block)
+          stats->steps_per_block[(size_t)S.seq * n_blocks + S.b] = S.nb;
+        S.b += 1;
+        S.nb = 0;
+        S.first = true;
+        if (S.b == n_blocks) {
+          out_steps[S.seq] = S.steps;
+          CK(cudaMemcpy(out_tokens + (size_t)S.seq * G, ctx->x + (size_t)sg.seq * c.max_seq + S.P,
+                        sizeof(int32_t) * G, cudaMemcpyDeviceToHost));
+          if ((rc = admit(sg.seq))) return rc;
+        }
+      } else if (st.unmasked < 1 || S.nb >= B) {
+        return fail(ctx, FDLLM_ERR_CUDA, "decode step made no progress");
+      }
+    }
+  }
+  CK(cudaStreamSynchronize(ctx->stream));
+  if (timing) {
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+  }
+  if (stats) {
+    int total = 0;
+    for (int i = 0; i < batch; ++i) total += out_steps[i];
+    stats->steps = total;
+    stats->refresh_steps = refresh;
+    stats->cached_steps = cached;
+    stats->n_blocks = n_blocks * batch;
+    stats->refresh_ms = refresh_ms;
+    stats->cached_ms = cached_ms;
+  }
+  return FDLLM_OK;
 }
 
 // ----------------------------------------------------- block-step chains
@@ -871,6 +1241,17 @@ int generate_impl(fdllm_ctx* ctx, const int32_t* prompt, bool prompt_dev, int P,
       if ((rc = run_step(ctx, mode, first, s, B, L, tau, nullptr))) return rc;
       if (timing) CK(cudaEventRecord(e1, ctx->stream));
       if ((rc = sync_state(ctx))) return rc;
+      if (stats && stats->trace_cap > 0 && total + nb < stats->trace_cap) {
+        // the step's own outputs (the stream is idle after sync_state)
+        const size_t at = (size_t)(total + nb) * B;
+        if (stats->trace_block) stats->trace_block[total + nb] = b;
+        if (stats->trace_conf)
+          CK(cudaMemcpy(stats->trace_conf + at, ctx->conf, sizeof(float) * B, cudaMemcpyDeviceToHost));
+        if (stats->trace_tok)
+          CK(cudaMemcpy(stats->trace_tok + at, ctx->tok, sizeof(int32_t) * B, cudaMemcpyDeviceToHost));
+        if (stats->trace_unmask)
+          CK(cudaMemcpy(stats->trace_unmask + at, ctx->unmask, B, cudaMemcpyDeviceToHost));
+      }
       const bool full = first || mode == FDLLM_CACHE_NONE;
       if (timing) {
         float ms = 0;
@@ -993,6 +1374,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   }
   ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
   if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
+  if (const char* at = std::getenv("FDLLM_ATTN_TC")) ctx->use_attn_tc = std::strcmp(at, "0") != 0;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {
@@ -1000,6 +1382,8 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
     dfree_all(ctx);
     if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);
     if (ctx->state_host) cudaFreeHost(ctx->state_host);
+    if (ctx->states_host) cudaFreeHost(ctx->states_host);
+    if (ctx->btab_host) cudaFreeHost(ctx->btab_host);
     if (ctx->err_host) cudaFreeHost(ctx->err_host);
     if (ctx->sp_host) cudaFreeHost(ctx->sp_host);
     delete ctx;
@@ -1032,17 +1416,20 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   const fdllm_config& c = *cfg;
   const int S = c.max_seq;
   const int hq = c.n_heads * c.head_dim, hkv = c.n_kv_heads * c.head_dim;
-  ctx->n_pages = (S + KV_PAGE - 1) / KV_PAGE;
+  ctx->pages_per_seq = (S + KV_PAGE - 1) / KV_PAGE;
+  ctx->n_pages = ctx->pages_per_seq * c.max_batch;
   ctx->kv_planes = ctx->f32 ? 2 : 4;
   const size_t kv_elems =
       (size_t)c.n_layers * ctx->n_pages * ctx->kv_planes * c.n_kv_heads * KV_PAGE * c.head_dim;
-  const size_t rows = (size_t)S;
+  // a batched forward holds up to every slot's whole sequence
+  const size_t rows = (size_t)S * c.max_batch;
+  ctx->rows_cap = (int)rows;
   // activation matrices: plain rows (fp32) or two-term pair rows (bf16)
   const size_t arows = ctx->f32 ? rows : pair_rows(rows);
   ctx->q_plane = ctx->f32 ? 0 : rows * hq;
   ctx->kv_pool = dalloc(ctx, kv_elems * ctx->esz);
   ctx->page_table = (int*)dalloc(ctx, sizeof(int) * ctx->n_pages);
-  ctx->rope = (float2*)dalloc(ctx, sizeof(float2) * rows * (c.head_dim / 2));
+  ctx->rope = (float2*)dalloc(ctx, sizeof(float2) * S * (c.head_dim / 2));
   ctx->x = (int*)dalloc(ctx, sizeof(int) * rows);
   ctx->h = (float*)dalloc(ctx, sizeof(float) * rows * c.d_model);
   ctx->a = dalloc(ctx, ctx->esz * arows * c.d_model);
@@ -1050,17 +1437,27 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->o = dalloc(ctx, ctx->esz * arows * hq);
   ctx->f = dalloc(ctx, ctx->esz * arows * c.ffn_dim);
   const int max_n = std::max(std::max(c.vocab, 2 * c.ffn_dim), std::max(hq + 2 * hkv, c.d_model));
-  ctx->n_counters = ((max_n + 127) / 128) * ((S + 31) / 32);
+  ctx->n_counters = (int)(((max_n + 127) / 128) * ((rows + 31) / 32));
   ctx->counters = (int*)dalloc(ctx, sizeof(int) * ctx->n_counters);
   if (ctx->tc) ctx->ws = (float*)dalloc(ctx, kWorkspaceBytes);
+  // LM-head rows per launch: a block (<= kMaxLmRows) or a batched chunk
+  const int lm_rows = c.max_batch > 1 ? kMaxLmChunk : kMaxLmRows;
   const size_t max_parts = std::max<size_t>((size_t)ctx->num_sms,
-                                            (size_t)((c.vocab + 127) / 128) * ((kMaxLmRows + 31) / 32));
-  ctx->lm_part_cap = max_parts * kMaxLmRows;
+                                            (size_t)((c.vocab + 127) / 128) * ((lm_rows + 31) / 32));
+  // per-launch partials; a batched step keeps every chunk's partials at once
+  const int lm_total = c.max_batch * kMaxLmRows;
+  ctx->lm_part_cap = max_parts * (size_t)std::max(lm_rows, lm_total);
   ctx->lm_part = (float*)dalloc(ctx, sizeof(SoftmaxState) * ctx->lm_part_cap);
-  ctx->conf = (float*)dalloc(ctx, sizeof(float) * kMaxLmRows);
-  ctx->tok = (int*)dalloc(ctx, sizeof(int) * kMaxLmRows);
-  ctx->unmask = (uint8_t*)dalloc(ctx, kMaxLmRows);
+  ctx->conf = (float*)dalloc(ctx, sizeof(float) * lm_total);
+  ctx->tok = (int*)dalloc(ctx, sizeof(int) * lm_total);
+  ctx->unmask = (uint8_t*)dalloc(ctx, lm_total);
   ctx->state = (DecodeState*)dalloc(ctx, sizeof(DecodeState));
+  ctx->states = (DecodeState*)dalloc(ctx, sizeof(DecodeState) * c.max_batch);
+  // batched-step tables: rows, attention tiles (one per query row at most),
+  // LM-head row sources, select segments
+  ctx->btab_bytes = rows * sizeof(RowInfo) + rows * sizeof(AttnTile) +
+                    (size_t)lm_total * sizeof(int) + (size_t)c.max_batch * sizeof(SelectSeg) + 1024;
+  ctx->btab = (uint8_t*)dalloc(ctx, ctx->btab_bytes);
   ctx->err_dev = (int*)dalloc(ctx, sizeof(int));
   ctx->check = (int*)dalloc(ctx, 4 * sizeof(int));
   ctx->sp = (StepParams*)dalloc(ctx, sizeof(StepParams));
@@ -1072,10 +1469,13 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
                   (void*)ctx->h, ctx->a, ctx->q, ctx->o, ctx->f, (void*)ctx->counters,
                   (void*)ctx->lm_part,
                   (void*)ctx->conf, (void*)ctx->tok, (void*)ctx->unmask, (void*)ctx->state,
+                  (void*)ctx->states, (void*)ctx->btab,
                   (void*)ctx->err_dev, (void*)ctx->check, (void*)ctx->sp})
     if (!p) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (ctx->tc && !ctx->ws) return bail(FDLLM_ERR_OOM, "device allocation failed");
   if (cudaMallocHost(&ctx->state_host, sizeof(DecodeState)) != cudaSuccess ||
+      cudaMallocHost(&ctx->states_host, sizeof(DecodeState) * c.max_batch) != cudaSuccess ||
+      cudaMallocHost(&ctx->btab_host, ctx->btab_bytes) != cudaSuccess ||
       cudaMallocHost(&ctx->err_host, sizeof(int)) != cudaSuccess ||
       cudaMallocHost(&ctx->sp_host, kSpRing * sizeof(StepParams)) != cudaSuccess)
     return bail(FDLLM_ERR_OOM, "pinned host allocation failed");
@@ -1085,8 +1485,8 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   std::vector<int> pt(ctx->n_pages);
   for (int i = 0; i < ctx->n_pages; ++i) pt[i] = i;
   const int half = c.head_dim / 2;
-  std::vector<float2> rt(rows * half);
-  for (size_t p = 0; p < rows; ++p)
+  std::vector<float2> rt((size_t)S * half);
+  for (size_t p = 0; p < (size_t)S; ++p)
     for (int i = 0; i < half; ++i) {
       const double inv = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
       const double ang = (double)p * inv;
@@ -1112,6 +1512,12 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
           !make_map(ctx, &ctx->m_f[i], ctx->f, arows, c.ffn_dim, nt))
         return bail(FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation buffer");
     }
+    // K/V pool rows of head_dim elements: (layer, page, plane, KV head, slot)
+    const uint64_t kv_rows = (uint64_t)c.n_layers * ctx->n_pages * ctx->kv_planes * c.n_kv_heads *
+                             KV_PAGE;
+    if (!make_q_map(ctx, &ctx->m_q3, ctx->q, rows) ||
+        !make_map(ctx, &ctx->m_kv, ctx->kv_pool, kv_rows, c.head_dim, 64))
+      return bail(FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for q or the K/V cache");
   }
   *out = ctx;
   return FDLLM_OK;
@@ -1160,6 +1566,13 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
   for (Want& w : want)
     if (!w.got) return fail(ctx, FDLLM_ERR_SHAPE, "missing tensor " + w.name);
   CK(cudaSetDevice(ctx->device));
+  if (ctx->tc) {
+    if (!ctx->inexact_dev) {
+      ctx->inexact_dev = (unsigned long long*)dalloc(ctx, sizeof(unsigned long long));
+      if (!ctx->inexact_dev) return fail(ctx, FDLLM_ERR_OOM, "counter allocation failed");
+    }
+    CK(cudaMemset(ctx->inexact_dev, 0, sizeof(unsigned long long)));
+  }
   const size_t es = ctx->esz;
   const size_t per_layer = ((size_t)(hq + 2 * hkv) * d + (size_t)d * hq + 2ull * F * d +
                             (size_t)d * F) * es + 2 * sizeof(float) * d;
@@ -1207,7 +1620,8 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
   // two-term fp16 activations keep 22 significant bits.  The embedding
   // table stays bf16 (read directly into the float32 residual stream).
   auto to_f16 = [&](void* p, size_t n) -> cudaError_t {
-    return ctx->tc ? launch_bf16_to_f16(p, n, ctx->err_dev, nullptr) : cudaSuccess;
+    return ctx->tc ? launch_bf16_to_f16(p, n, ctx->err_dev, ctx->inexact_dev, nullptr)
+                   : cudaSuccess;
   };
   CK(to_f16(ctx->lm_head, (size_t)V * d));
   CK(norm_to(ctx->final_norm, "final_norm"));
@@ -1287,9 +1701,19 @@ int fdllm_load_weights(fdllm_ctx* ctx, const fdllm_tensor* tensors, int n_tensor
                   "a GEMM weight is NaN or outside the fp16 range (|w| > 65504)");
     }
   }
+  if (ctx->tc) {
+    unsigned long long n_inexact = 0;
+    CK(cudaMemcpy(&n_inexact, ctx->inexact_dev, sizeof(n_inexact), cudaMemcpyDeviceToHost));
+    ctx->inexact_weights = (int64_t)n_inexact;
+  }
   ctx->weights = arena;
   ctx->weights_loaded = true;
   return FDLLM_OK;
+}
+
+int64_t fdllm_inexact_weight_count(const fdllm_ctx* ctx) {
+  if (!ctx) return -1;
+  return ctx->weights_loaded ? ctx->inexact_weights : 0;
 }
 
 int fdllm_generate(fdllm_ctx* ctx, const int32_t* prompt_ids, int prompt_len, int gen_len,
@@ -1337,6 +1761,10 @@ int fdllm_generate_batch(fdllm_ctx* ctx, int batch, const int32_t* const* prompt
         return fail(ctx, FDLLM_ERR_ARG, "prompt id out of range or equal to the mask id");
   }
   const int n_blocks = gen_len / block_size;
+  if (c.max_batch > 1 && batch > 1)
+    return generate_batch_impl(ctx, batch, prompts, prompt_lens, gen_len, block_size, tau,
+                               cache_mode, 0, out_tokens, out_steps, stats);
+  // one slot: each sequence in turn through the single-sequence path
   fdllm_stats tot{};
   if (stats) tot.collect_timing = stats->collect_timing;
   for (int i = 0; i < batch; ++i) {
@@ -1621,6 +2049,8 @@ int fdllm_destroy(fdllm_ctx* ctx) {
   ctx->step_graphs.clear();
   dfree_all(ctx);
   if (ctx->state_host) cudaFreeHost(ctx->state_host);
+  if (ctx->states_host) cudaFreeHost(ctx->states_host);
+  if (ctx->btab_host) cudaFreeHost(ctx->btab_host);
   if (ctx->err_host) cudaFreeHost(ctx->err_host);
   if (ctx->sp_host) cudaFreeHost(ctx->sp_host);
   if (ctx->own_stream && ctx->stream) cudaStreamDestroy(ctx->stream);

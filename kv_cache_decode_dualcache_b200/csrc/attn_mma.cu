@@ -92,30 +92,40 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
   const int rg = warp % NRG, kg = warp / NRG;
   const int H = p.n_heads, Hkv = p.n_kv_heads, rep = H / Hkv;
   const int g = blockIdx.y;
-  const int rows_total = p.M * rep;
-  const int row0 = blockIdx.x * (16 * NRG);
+  pdl_trigger();
+  pdl_wait();
+  // one sequence: row tiles of the M query positions over keys [0, p.L);
+  // batched forward: this CTA's tile of one sequence's segment
+  int rows_total = p.M * rep, row0 = blockIdx.x * (16 * NRG), qbase = 0, L = p.L;
+  const int* ptab = p.page_table;
+  if (p.tiles) {
+    const AttnTile tl = p.tiles[blockIdx.x];
+    rows_total = tl.m * rep;
+    row0 = tl.r0;
+    qbase = tl.q0;
+    L = tl.L;
+    ptab = p.page_table + (size_t)tl.seq * p.pages_per_seq;
+  }
   const int key_lo = blockIdx.z * p.keys_per_split;
-  const int key_hi = min(p.L, key_lo + p.keys_per_split);
+  const int key_hi = min(L, key_lo + p.keys_per_split);
   const int n_kt = (key_hi - key_lo + 63) / 64;
 
   const __half* qg = reinterpret_cast<const __half*>(p.q);
   const uint16_t* pool = reinterpret_cast<const uint16_t*>(p.kv_pool);
-  pdl_trigger();
-  pdl_wait();
 
   // ---- Q tiles (hi and lo planes), 16 * NRG rows
   for (int idx = tid; idx < 16 * NRG * CH; idx += NT) {
     const int i = idx / CH, ch = idx % CH;
     const int r = row0 + i;
     const bool ok = r < rows_total;
-    const int m = ok ? r / rep : 0, jj = ok ? r % rep : 0;
+    const int m = ok ? qbase + r / rep : 0, jj = ok ? r % rep : 0;
     const __half* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
     cp_async16(q_s + swz<HD>(i, ch), src, ok ? 16 : 0);
     cp_async16(q_s + QT + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
   }
   auto load_kv = [&](int kt, int buf) {
     const int k0 = key_lo + kt * 64;
-    const int page = p.page_table[k0 / KV_PAGE];
+    const int page = ptab[k0 / KV_PAGE];
     const size_t plane = (size_t)Hkv * KV_PAGE * HD;
     const size_t base = ((size_t)p.layer * p.n_pages + page) * 4 * plane + (size_t)g * KV_PAGE * HD;
     for (int idx = tid; idx < 64 * CH; idx += NT) {
@@ -338,7 +348,7 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
     if (!writer) break;
     const int rr = row0 + rg * 16 + (lane >> 2) + 8 * r;
     if (rr >= rows_total) continue;
-    const int m = rr / rep, head = g * rep + rr % rep;
+    const int m = qbase + rr / rep, head = g * rep + rr % rep;
     const float inv = 1.0f / lrow[r];
     __half* o = reinterpret_cast<__half*>(p.o);
     const size_t hi_off = (size_t)pair_row(m) * hq + (size_t)head * HD;
@@ -386,7 +396,8 @@ cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
   const int rows_per_cta = 16 * (NW / NKG);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((rows + rows_per_cta - 1) / rows_per_cta, p.n_kv_heads, p.n_split);
+  cfg.gridDim = dim3(p.tiles ? p.n_tiles : (rows + rows_per_cta - 1) / rows_per_cta,
+                     p.n_kv_heads, p.n_split);
   cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -411,6 +422,8 @@ cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
 
 template <int HD>
 cudaError_t launch_nkg(const AttnParams& p, cudaStream_t st, bool pdl) {
+  // batched forwards tile every segment into 64-row tiles (attn_rows_per_cta(-1, ..))
+  if (p.tiles) return launch_hd<HD, 1, 4>(p, st, pdl);
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
   if (rows <= 16) return launch_hd<HD, 4, 4>(p, st, pdl);
   if (rows <= 32) return launch_hd<HD, 2, 4>(p, st, pdl);
@@ -422,12 +435,15 @@ cudaError_t launch_nkg(const AttnParams& p, cudaStream_t st, bool pdl) {
 }  // namespace
 
 int attn_rows_per_cta(int M, int n_heads, int n_kv_heads) {
+  if (M < 0) return 64;  // batched forwards (AttnParams::tiles)
   const int rows = M * (n_heads / n_kv_heads);
   return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
 }
 
 cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl) {
-  if (p.kv_planes != 4 || p.n_split < 1 || p.n_split > kMaxSplit) return cudaErrorInvalidValue;
+  if (p.kv_planes != 4 || p.n_split < 1 || p.n_split > kMaxSplit ||
+      (p.tiles && (p.n_split != 1 || p.n_tiles < 1)))
+    return cudaErrorInvalidValue;
   switch (p.head_dim) {
     case 64: return launch_nkg<64>(p, st, pdl);
     case 128: return launch_nkg<128>(p, st, pdl);
@@ -448,6 +464,7 @@ cudaError_t init_kernel_attributes() {
   if (e == cudaSuccess) e = set_attr<128, 1, 8>();
   if (e == cudaSuccess) e = gemm_tc_init_attributes();
   if (e == cudaSuccess) e = chain_init_attributes();
+  if (e == cudaSuccess) e = attn_tc_init_attributes();
   return e;
 }
 

@@ -244,6 +244,19 @@ FD_DEV void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, uint64_t* b
       : "memory");
 }
 
+FD_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                        int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Shared-memory writes of this thread (generic proxy) become visible to the
+// tensor core's and TMA's reads of shared memory (async proxy).
+FD_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // L2 policy for data read once (streamed weights): evicted first, so the
 // activations, partial tiles and K/V the step re-reads stay in L2.
 FD_DEV uint64_t make_policy_evict_first() {
@@ -292,6 +305,21 @@ FD_DEV uint64_t smem_desc_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// Descriptor of an MN-major operand tile stored with the 128-byte swizzle:
+// rows of 128 bytes hold 64 consecutive MN elements for one K index, 8 rows
+// (8 K indices) form a 1024-byte swizzle atom.  lbo_bytes = distance between
+// 64-element atoms along MN, sbo_bytes = distance between 8-row groups
+// along K.
+FD_DEV uint64_t smem_desc_sw128_mn(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: D f32, A and B both fp16 (f16 = true)
 // or both bf16, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_f32acc(int n, bool f16) {
@@ -300,6 +328,11 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int n, bool f16) {
          | ((f16 ? 0u : 1u) << 10)          // B format: the same as A
          | ((uint32_t)(n >> 3) << 17)       // N >> 3
          | ((uint32_t)(128 >> 4) << 24);    // M >> 4
+}
+
+// As idesc_f32acc with the B operand MN-major (its N elements contiguous).
+__host__ __device__ constexpr uint32_t idesc_f32acc_bmn(int n, bool f16) {
+  return idesc_f32acc(n, f16) | (1u << 16);
 }
 
 FD_DEV void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,

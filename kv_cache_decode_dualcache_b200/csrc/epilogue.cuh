@@ -32,6 +32,12 @@ FD_DEV size_t kv_offset_pg(const EpiParams& ep, int page, int pos, int plane, in
          (size_t)slot * ep.head_dim + dim;
 }
 
+// Batched forward (ep.rows set): position and K/V page of token row tok.
+FD_DEV int row_pos(const EpiParams& ep, int tok) { return __ldg(&ep.rows[tok].pos); }
+FD_DEV int row_page(const EpiParams& ep, int tok, int pos) {
+  return __ldg(&ep.page_table[__ldg(&ep.rows[tok].seq) * ep.pages_per_seq + pos / KV_PAGE]);
+}
+
 // One 32-token chunk of a 128-feature output tile.
 //   tile: [32][128] float in shared memory, fully written before the call.
 //   n0:   first feature of the tile; t0: token row of tile row 0.
@@ -85,6 +91,35 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
     case EPI_QKV: {
       // fp32 model: natural row order, RoPE partners through the tile
       if (n >= ep.N) break;
+      if (ep.rows) {
+        // batched forward: every row has its own position and slot
+        const int hd = ep.head_dim, half = hd / 2;
+        const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
+        const int dh = n % hd;
+        const bool is_q = n < hq, is_v = n >= hq + hk;
+        float* kv = reinterpret_cast<float*>(ep.kv_pool);
+        for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
+          const int tok = t0 + t;
+          const int pos = row_pos(ep, tok);
+          float y = tile[t * 128 + e];
+          if (!is_v) {
+            const float2 c = __ldg(&ep.rope[(size_t)pos * half + (dh % half)]);
+            y = dh < half ? y * c.x - tile[t * 128 + e + half] * c.y
+                          : y * c.x + tile[t * 128 + e - half] * c.y;
+          }
+          if (is_q) {
+            const size_t i = (size_t)tok * hq + n;
+            if (FD_CHECK(i < ep.cap_q, ep.check, 4, i, ep.cap_q))
+              reinterpret_cast<float*>(ep.q_out)[i] = y;
+          } else {
+            const int page = row_page(ep, tok, pos);
+            const size_t i = is_v ? kv_offset_pg(ep, page, pos, 1, (n - hq - hk) / hd, dh)
+                                  : kv_offset_pg(ep, page, pos, 0, (n - hq) / hd, dh);
+            if (FD_CHECK(i < ep.cap_kv, ep.check, 5, i, ep.cap_kv)) kv[i] = y;
+          }
+        }
+        break;
+      }
       const int hd = ep.head_dim, half = hd / 2;
       const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
       const int dh = n % hd;
@@ -189,12 +224,64 @@ FD_DEV __host__ int rope_slab_dim(int r, int hd) {
   return 16 * (r >> 5) + (r & 15) + ((r >> 4) & 1) * (hd / 2);
 }
 
+// The QKV epilogue of epi_regs in a batched forward: as the one-sequence
+// path, with each row's position and K/V page looked up (rows of one chunk
+// may belong to different sequences).
+FD_DEV void epi_regs_qkv_rows(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0,
+                              int e, int nt) {
+  const int lane = e & 31;
+  const int n = n0 + e;
+  const int hd = ep.head_dim, half = hd / 2;
+  const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
+  const int region = n < hq ? 0 : (n < hq + hk ? 1 : 2);  // q, k, v (uniform per warp)
+  const int rn = n - (region == 0 ? 0 : (region == 1 ? hq : hq + hk));
+  const int head = rn / hd;
+  const int r = rn - head * hd;
+  const int dim = region < 2 ? rope_slab_dim(r, hd) : r;
+  const bool second = lane >= 16;  // holds dim + hd/2 of the rotate-half pair
+#pragma unroll
+  for (int t = 0; t < CHUNK_T; ++t) {
+    if (t >= nt) break;
+    const int tok = t0 + t;
+    const int pos = row_pos(ep, tok);
+    float y = v[t];
+    if (region < 2) {
+      const float2 cs = __ldg(&ep.rope[(size_t)pos * half + (dim % half)]);
+      const float p = __shfl_xor_sync(0xffffffffu, y, 16);
+      y = second ? (y * cs.x + p * cs.y) : (y * cs.x - p * cs.y);
+    }
+    __half hi, lo;
+    split_f16(y, hi, lo);
+    if (region == 0) {
+      __half* q = reinterpret_cast<__half*>(ep.q_out);
+      const size_t i = (size_t)tok * hq + head * hd + dim;
+      if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
+        q[i] = hi;
+        q[ep.q_plane + i] = lo;
+      }
+    } else {
+      const int page = row_page(ep, tok, pos);
+      const int plane = region == 1 ? 0 : 2;
+      __half* kv = reinterpret_cast<__half*>(ep.kv_pool);
+      const size_t i0 = kv_offset_pg(ep, page, pos, plane, head, dim);
+      const size_t i1 = kv_offset_pg(ep, page, pos, plane + 1, head, dim);
+      if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
+        kv[i0] = hi;
+        kv[i1] = lo;
+      }
+    }
+  }
+}
+
 // Epilogue of one 32-token chunk held in registers by the 128 threads of an
 // epilogue warpgroup: v[t] = output feature n0 + e of token row t0 + t.
 // e = tile row = 32 * (warp % 4) + lane.  Shuffles stay within a warp and
 // control flow is warp-uniform (N and the q / k / v region boundaries are
 // multiples of 64 for the QKV and SwiGLU layouts).  EPI_LMHEAD is not
-// handled here: it needs all 128 features of a token (epi_chunk).
+// handled here: it needs all 128 features of a token (epi_chunk).  ROWS:
+// the batched forward's per-row positions (a separate instantiation, so the
+// one-sequence code is compiled without that path).
+template <bool ROWS = false>
 FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0, int e) {
   const int lane = e & 31;
   const int n = n0 + e;
@@ -249,6 +336,10 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
     }
     case EPI_QKV: {
       if (n >= ep.N) break;  // warp-uniform
+      if constexpr (ROWS) {
+        epi_regs_qkv_rows(ep, v, n0, t0, e, nt);
+        break;
+      }
       const int hd = ep.head_dim, half = hd / 2;
       const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
       const int region = n < hq ? 0 : (n < hq + hk ? 1 : 2);  // q, k, v (uniform per warp)
@@ -365,8 +456,9 @@ FD_DEV void epi_staged_f16(const EpiParams& ep, const float (&v)[CHUNK_T], int n
     named_bar(bar, EPI_THREADS);
     return;
   }
-  // EPI_QKV: the tile is 128 / hd heads of one region (q, k or v); N and the
-  // region bounds are multiples of 64, so a warp is wholly inside or outside
+  // EPI_QKV (one sequence: the chain kernel's block rows): the tile is
+  // 128 / hd heads of one region (q, k or v); N and the region bounds are
+  // multiples of 64, so a warp is wholly inside or outside
   const int hd = ep.head_dim, half = hd / 2;
   const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
   const bool valid = n < ep.N;

@@ -42,7 +42,7 @@ namespace {
 
 constexpr int BK = 64;                    // K elements per stage (128 bytes of bf16)
 constexpr int A_STAGE_BYTES = 128 * BK * 2;
-constexpr int LM_MAX_ROWS = 256;          // largest M for the LM-head epilogue
+constexpr int LM_MAX_ROWS = 512;          // largest M for the LM-head epilogue
 
 
 template <int NT> struct TcCfg;
@@ -87,7 +87,7 @@ FD_DEV UnitCoord decode_unit(const GemmShape& gs, int u) {
   return c;
 }
 
-template <int NT>
+template <int NT, bool ROWS>
 __global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap,
                    const __grid_constant__ CUtensorMap amap, GemmShape gs, EpiParams ep,
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
             named_bar(1, EPI_ALL);
             epi_chunk(ep, tile, n0, tg0 + ch * CHUNK_T, e, lm);
           } else {
-            epi_regs(ep, v, n0, tg0 + ch * CHUNK_T, e);
+            epi_regs<ROWS>(ep, v, n0, tg0 + ch * CHUNK_T, e);
           }
         }
       }
@@ -364,8 +364,12 @@ __global__ void __launch_bounds__(TcLayout<NT>::THREADS, 1)
 
 template <int NT>
 cudaError_t set_attr_nt() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcLayout<NT>::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<NT, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       TcLayout<NT>::SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gemm_tc_kernel<NT, true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, TcLayout<NT>::SMEM);
 }
 
 template <int NT>
@@ -377,7 +381,11 @@ cudaError_t launch_nt(const CUtensorMap* w_map, const CUtensorMap* act_map, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_k(pdl, gemm_tc_kernel<NT>, dim3(gs.grid), dim3(TcLayout<NT>::THREADS),
+  // the batched forward's per-row positions get their own instantiation
+  if (ep.rows)
+    return launch_k(pdl, gemm_tc_kernel<NT, true>, dim3(gs.grid), dim3(TcLayout<NT>::THREADS),
+                    (size_t)TcLayout<NT>::SMEM, st, *w_map, *act_map, gs, ep, sc);
+  return launch_k(pdl, gemm_tc_kernel<NT, false>, dim3(gs.grid), dim3(TcLayout<NT>::THREADS),
                   (size_t)TcLayout<NT>::SMEM,
                   st, *w_map, *act_map, gs, ep, sc);
 }

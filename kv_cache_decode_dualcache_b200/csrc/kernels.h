@@ -29,6 +29,14 @@ struct StepParams {
   int fixed_k;       // > 0: unmask the fixed_k most confident masked positions instead
 };
 
+// Batched forward (rows of several sequences in one pass): the sequence
+// slot and absolute position of every row of the forward.  Slot q's token ids
+// live at x[q * seq_stride ..], its K/V pages at page_table[q * pages_per_seq ..].
+struct RowInfo {
+  int pos;
+  int seq;
+};
+
 // Everything a GEMM epilogue needs.  Token index t is the row within the
 // GEMM's activation operand (0..M-1); feature index n is the output column.
 struct EpiParams {
@@ -61,6 +69,9 @@ struct EpiParams {
   float* lm_part;    // [n_part][M] of (m, s, arg) triples
   float* dbg_logits; // optional [M, N] float logits (mask id included)
   const StepParams* sp;  // when set, pos0 = sp->r0 (device-side step scalars)
+  const RowInfo* rows;   // batched forward: row t has position rows[t].pos in slot rows[t].seq
+                         // (NULL: one sequence, row t at position pos0 + t)
+  int pages_per_seq;     // batched forward: page-table entries per slot
   // Capacities (elements) of the output buffers, used only by builds with
   // FDLLM_CHECKS, where every store is bounds-checked and a violation is
   // recorded in check[0..3] (count, code, index, aux) instead of performed.
@@ -131,6 +142,15 @@ cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int
                              bool pdl = false);
 int gemm_tc_smem_bytes(int nt);
 
+// Batched attention: CTA x-index i covers query rows [r0, r0 + rows) (rows
+// of (position, head-in-group) pairs) of one sequence's segment, whose
+// positions are rows q0 .. q0 + m - 1 of the forward; its keys are [0, L) of
+// slot seq.
+struct AttnTile {
+  int q0, m, r0, L, seq;
+  int pad[3];
+};
+
 struct AttnParams {
   const void* q;       // [M, H, hd] (fp32) or fp16 hi/lo planes of [M, H, hd] (bf16 model)
   size_t q_plane;      // elements per q plane (bf16 model)
@@ -144,25 +164,47 @@ struct AttnParams {
   int n_heads, n_kv_heads, head_dim;
   int n_split;         // key splits, <= 8: one thread-block cluster per (row tile, KV head)
   int keys_per_split;  // multiple of 64
+  const AttnTile* tiles;  // batched forward: one entry per CTA along x (NULL: one sequence)
+  int n_tiles;
+  int pages_per_seq;
 };
 
 cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl = false);
+// tcgen05 + TMA attention for many query rows (see attn_tc.cu).  qmap: 3-D
+// map {head_dim, n_heads, 2 * q_lo_rows} over the q hi plane followed by the
+// lo plane (boxes {64, rep, 128 / rep}); kvmap: 2-D map {head_dim, rows} over
+// the K/V pool, one row per (layer, page, plane, KV head, slot) (boxes
+// {64, 64}); both with the 128-byte swizzle.
+bool attn_tc_supported(const AttnParams& p);
+cudaError_t launch_attn_tc(const CUtensorMap* qmap, const CUtensorMap* kvmap, const AttnParams& p,
+                           int q_lo_rows, int* err, cudaStream_t st, bool pdl = false);
+cudaError_t attn_tc_init_attributes();
 // Query rows per CTA of launch_attn_mma for M query positions (16, 32 or 64).
 int attn_rows_per_cta(int M, int n_heads, int n_kv_heads);
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl = false);
+
+// Row sources of the norm kernels in a batched forward (all NULL: one
+// sequence).  rows: the embedding gather reads x[rows[i].seq * seq_stride +
+// rows[i].pos]; src: RMSNorm output row i reads h row src[i].
+struct RowMap {
+  const RowInfo* rows;
+  int seq_stride;
+  const int* src;
+};
 
 // h[i] = embed[x[r0+i]]; a[i] = RMSNorm(h[i]) * g, i in [0, M).  With sp,
 // r0 = sp->r0.  bf16 model: bf16 embedding rows, a in two-term fp16 pair rows.
 cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
                                  int vocab, const float* g, float eps, float* h, void* a,
                                  int f32, int* err, const StepParams* sp, cudaStream_t st,
-                                 bool pdl = false);
+                                 bool pdl = false, RowMap rm = RowMap{nullptr, 0, nullptr});
 // a[i] = RMSNorm(h[h_row0 + i]) * g, i in [0, M).  bf16 model: two-term fp16
 // pair rows.
 // With sp and rows_from_lm0, h_row0 = sp->lm0.
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
                            void* a, int f32, const StepParams* sp, bool rows_from_lm0,
-                           cudaStream_t st, bool pdl = false);
+                           cudaStream_t st, bool pdl = false,
+                           RowMap rm = RowMap{nullptr, 0, nullptr});
 
 // ------------------------------------------------ block-step chain kernel
 // One launch runs a program of phases of the DualCache block step (bf16
@@ -246,12 +288,30 @@ cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x,
                                 uint8_t* unmask, DecodeState* state, const StepParams* sp,
                                 cudaStream_t st, bool pdl = false);
 
+// Batched decode: LM-head rows [k0, k0 + n) belong to the block [s, s + n)
+// of the sequence in slot seq.
+struct SelectSeg {
+  int k0, n, seq, s;
+};
+
+// merge + select per sequence: block i of the grid handles segs[i] (n <= 256)
+// with the partials of all m_lm LM-head rows, the slot's token ids at
+// x + seq * seq_stride and its state states[seq]; conf / tok / unmask are
+// indexed by LM-head row.  fixed_k > 0 selects the fixed-count rule.
+cudaError_t launch_merge_select_seg(const float* lm_part, int n_part, int m_lm,
+                                    const SelectSeg* segs, int n_segs, int* x, int seq_stride,
+                                    int mask_id, float tau, int fixed_k, float* conf, int* tok,
+                                    uint8_t* unmask, DecodeState* states, cudaStream_t st,
+                                    bool pdl = false);
+
 cudaError_t launch_fill_masked(int* x, int from, int to, int mask_id, cudaStream_t st,
                                bool pdl = false);
 cudaError_t launch_check_prompt(const int* x, int n, int vocab, int mask_id, int* err,
                                 cudaStream_t st, bool pdl = false);
 // In place: n bf16 values -> fp16 (round to nearest even).  A value outside
-// the fp16 range sets DEV_ERR_RANGE in *err.
-cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, cudaStream_t st);
+// the fp16 range sets DEV_ERR_RANGE in *err; values the conversion changes
+// are counted into *inexact (may be NULL).
+cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, unsigned long long* inexact,
+                               cudaStream_t st);
 
 }  // namespace fd

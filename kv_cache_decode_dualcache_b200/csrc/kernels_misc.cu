@@ -48,7 +48,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x,
                                                       float* __restrict__ h, int h_row0, int d,
                                                       const float* __restrict__ g, float eps,
                                                       void* __restrict__ a, int* err,
-                                                      const StepParams* sp, int rows_from_lm0) {
+                                                      const StepParams* sp, int rows_from_lm0,
+                                                      RowMap rm) {
   // The row stays in registers (d <= 256 * RMS_VPT): every load is issued
   // before any store.
   constexpr int VPT = RMS_VPT;
@@ -60,10 +61,12 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x,
     if (x) r0 = sp->r0;
     if (rows_from_lm0) h_row0 = sp->lm0;
   }
-  float* hr = h + (size_t)(h_row0 + row) * d;
+  // batched forward: the output row's h row and token come from the row map
+  float* hr = h + (size_t)(rm.src ? rm.src[row] : h_row0 + row) * d;
   float v[VPT];
   if (x) {
-    int tok = x[r0 + row];
+    int tok = rm.rows ? x[(size_t)rm.rows[row].seq * rm.seq_stride + rm.rows[row].pos]
+                      : x[r0 + row];
     if (tok < 0 || tok >= vocab) {
       if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
       tok = 0;
@@ -122,7 +125,8 @@ __global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__
                                                          int h_row0, int d,
                                                          const float* __restrict__ g, float eps,
                                                          __half* __restrict__ a, int* err,
-                                                         const StepParams* sp, int rows_from_lm0) {
+                                                         const StepParams* sp, int rows_from_lm0,
+                                                         RowMap rm) {
   constexpr int V4 = RMS_VPT / 4;
   __shared__ float red[32];
   pdl_trigger();
@@ -132,10 +136,12 @@ __global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__
     if (x) r0 = sp->r0;
     if (rows_from_lm0) h_row0 = sp->lm0;
   }
-  float* hr = h + (size_t)(h_row0 + row) * d;
+  // batched forward: the output row's h row and token come from the row map
+  float* hr = h + (size_t)(rm.src ? rm.src[row] : h_row0 + row) * d;
   float4 v[V4];
   if (x) {
-    int tok = x[r0 + row];
+    int tok = rm.rows ? x[(size_t)rm.rows[row].seq * rm.seq_stride + rm.rows[row].pos]
+                      : x[r0 + row];
     if (tok < 0 || tok >= vocab) {
       if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
       tok = 0;
@@ -262,24 +268,20 @@ __global__ void __launch_bounds__(128) kv_cosine_kernel(const void* __restrict__
 }
 
 // ------------------------------------------------------- merge + select
-__global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
-                                    int mask_id, float tau, int select, float* conf, int* tok,
-                                    uint8_t* unmask, DecodeState* state, const StepParams* sp) {
-  __shared__ float s_conf[256];
-  __shared__ int s_tok[256];
-  __shared__ int s_best;
-  pdl_trigger();
-  pdl_wait();
-  int fixed_k = 0;
-  if (sp) {
-    s = sp->s;
-    tau = sp->tau;
-    fixed_k = sp->fixed_k;
-  }
+// Merge of the LM-head partials of n rows (row t's partial of producer q at
+// part[q * stride + t]) into conf / tok, then, when select is set, the
+// unmask rule on the block x[s .. s + n): every masked position with
+// conf >= tau (or, with fixed_k > 0, the fixed_k most confident masked
+// ones), else the single most confident masked position; the chosen
+// positions take their argmax token.  One CTA of at least n threads.
+FD_DEV void merge_select_body(const SoftmaxState* part, int n_part, int stride, int n, int* x,
+                              int s, int mask_id, float tau, int fixed_k, int select,
+                              float* conf, int* tok, uint8_t* unmask, DecodeState* state,
+                              float* s_conf, int* s_tok, int* s_best) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int t = warp; t < n; t += blockDim.x >> 5) {
     SoftmaxState st = sm_empty();
-    for (int q = lane; q < n_part; q += 32) st = sm_merge(st, part[(size_t)q * n + t]);
+    for (int q = lane; q < n_part; q += 32) st = sm_merge(st, part[(size_t)q * stride + t]);
     st = warp_sm_merge(st);
     if (lane == 0) {
       // conf = exp(z_max - logsumexp) = 1 / sum exp(z - z_max)
@@ -320,10 +322,10 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
         if (best < 0 || cj > bc) { best = j; bc = cj; }
       }
     }
-    s_best = best;
+    *s_best = best;
   }
   __syncthreads();
-  const bool u = pass || (n_pass == 0 && i == s_best);
+  const bool u = pass || (n_pass == 0 && i == *s_best);
   if (valid) unmask[i] = u ? 1 : 0;
   const int n_left = __syncthreads_count(masked && !u);
   const int n_un = __syncthreads_count(u);
@@ -335,12 +337,63 @@ __global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n,
   }
 }
 
-__global__ void bf16_to_f16_kernel(uint16_t* p, size_t n, int* err) {
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const float v = __uint_as_float((uint32_t)p[i] << 16);
-    if (!(fabsf(v) <= 65504.0f)) atomicOr(err, DEV_ERR_RANGE);  // also NaN
-    p[i] = __half_as_ushort(__float2half_rn(v));
+__global__ void merge_select_kernel(const SoftmaxState* part, int n_part, int n, int* x, int s,
+                                    int mask_id, float tau, int select, float* conf, int* tok,
+                                    uint8_t* unmask, DecodeState* state, const StepParams* sp) {
+  __shared__ float s_conf[256];
+  __shared__ int s_tok[256];
+  __shared__ int s_best;
+  pdl_trigger();
+  pdl_wait();
+  int fixed_k = 0;
+  if (sp) {
+    s = sp->s;
+    tau = sp->tau;
+    fixed_k = sp->fixed_k;
+  }
+  merge_select_body(part, n_part, n, n, x, s, mask_id, tau, fixed_k, select, conf, tok, unmask,
+                    state, s_conf, s_tok, &s_best);
+}
+
+// Batched decode: CTA i merges and selects the block of segs[i].
+__global__ void merge_select_seg_kernel(const SoftmaxState* part, int n_part, int m_lm,
+                                        const SelectSeg* segs, int* x, int seq_stride,
+                                        int mask_id, float tau, int fixed_k, float* conf,
+                                        int* tok, uint8_t* unmask, DecodeState* states) {
+  __shared__ float s_conf[256];
+  __shared__ int s_tok[256];
+  __shared__ int s_best;
+  pdl_trigger();
+  pdl_wait();
+  const SelectSeg sg = segs[blockIdx.x];
+  merge_select_body(part + sg.k0, n_part, m_lm, sg.n, x + (size_t)sg.seq * seq_stride, sg.s,
+                    mask_id, tau, fixed_k, 1, conf + sg.k0, tok + sg.k0, unmask + sg.k0,
+                    states + sg.seq, s_conf, s_tok, &s_best);
+}
+
+// In place bf16 -> fp16 (round to nearest even).  Values outside the fp16
+// range (and NaN) set DEV_ERR_RANGE; conversions that change the value (bf16
+// values below 2^-17 in magnitude, under the fp16 subnormal grid) are counted
+// into *inexact, one atomic per warp and iteration that saw any.
+__global__ void bf16_to_f16_kernel(uint16_t* p, size_t n, int* err,
+                                   unsigned long long* inexact) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t n_iter = (n + stride - 1) / stride;
+  const size_t i0 = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  // every thread runs the same number of iterations, so the ballot below is
+  // taken by the full warp
+  for (size_t k = 0; k < n_iter; ++k) {
+    const size_t i = i0 + k * stride;
+    bool changed = false;
+    if (i < n) {
+      const float v = __uint_as_float((uint32_t)p[i] << 16);
+      if (!(fabsf(v) <= 65504.0f)) atomicOr(err, DEV_ERR_RANGE);  // also NaN
+      const __half h = __float2half_rn(v);
+      changed = __half2float(h) != v && v == v;
+      p[i] = __half_as_ushort(h);
+    }
+    const unsigned b = __ballot_sync(0xffffffffu, changed);
+    if (b && (threadIdx.x & 31) == 0 && inexact) atomicAdd(inexact, (unsigned long long)__popc(b));
   }
 }
 
@@ -426,8 +479,17 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   pdl_wait();
   float* qs = sh;               // [hd]
   float* sc = sh + p.head_dim;  // [L]
-  const int m = blockIdx.x, head = blockIdx.y;
+  const int head = blockIdx.y;
   const int hd = p.head_dim, H = p.n_heads, Hkv = p.n_kv_heads;
+  // batched forward: one tile per query row (its forward row, keys, slot)
+  int m = blockIdx.x, L = p.L;
+  const int* ptab = p.page_table;
+  if (p.tiles) {
+    const AttnTile tl = p.tiles[blockIdx.x];
+    m = tl.q0;
+    L = tl.L;
+    ptab = p.page_table + (size_t)tl.seq * p.pages_per_seq;
+  }
   const int g = head / (H / Hkv);
   const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)m * H + head) * hd;
   for (int d = threadIdx.x; d < hd; d += blockDim.x) qs[d] = to_f(q[d]);
@@ -436,13 +498,13 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   const T* kp = reinterpret_cast<const T*>(p.kv_pool);
   const VT* vp = reinterpret_cast<const VT*>(p.kv_pool);
   auto off = [&](int pos, int kv) {
-    const int page = p.page_table[pos / KV_PAGE];
+    const int page = ptab[pos / KV_PAGE];
     return ((((size_t)p.layer * p.n_pages + page) * p.kv_planes + kv) * Hkv + g) *
                (size_t)(KV_PAGE * hd) +
            (size_t)(pos % KV_PAGE) * hd;
   };
   float mx = -INFINITY;
-  for (int j = threadIdx.x; j < p.L; j += blockDim.x) {
+  for (int j = threadIdx.x; j < L; j += blockDim.x) {
     const T* kr = kp + off(j, 0);
     float dot = 0.0f;
     for (int d = 0; d < hd; ++d) dot = fmaf(qs[d], to_f(kr[d]), dot);
@@ -451,7 +513,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   }
   mx = block_max(mx, red);
   float sum = 0.0f;
-  for (int j = threadIdx.x; j < p.L; j += blockDim.x) {
+  for (int j = threadIdx.x; j < L; j += blockDim.x) {
     const float e = expf(sc[j] - mx);
     sc[j] = e;
     sum += e;
@@ -461,7 +523,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
   T* o = reinterpret_cast<T*>(p.o) + ((size_t)m * H + head) * hd;
   for (int d = threadIdx.x; d < hd; d += blockDim.x) {
     float acc = 0.0f;
-    for (int j = 0; j < p.L; ++j) acc = fmaf(sc[j], to_f(vp[off(j, 1) + d]), acc);
+    for (int j = 0; j < L; ++j) acc = fmaf(sc[j], to_f(vp[off(j, 1) + d]), acc);
     o[d] = from_f<T>(acc / sum);
   }
 }
@@ -471,34 +533,35 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnParams p) {
 cudaError_t launch_embed_rmsnorm(const int* x, int r0, int M, const void* embed, int d,
                                  int vocab, const float* g, float eps, float* h, void* a,
                                  int f32, int* err, const StepParams* sp, cudaStream_t st,
-                                 bool pdl) {
+                                 bool pdl, RowMap rm) {
   if (M <= 0) return cudaSuccess;
   if (f32)
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, x, r0,
-                    (const float*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
+                    (const float*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0, rm);
   if (d % 4 == 0)
     return launch_k(pdl, rmsnorm_v4_kernel, dim3(M), dim3(256), 0, st, x, r0,
-                    (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, (__half*)a, err, sp, 0);
+                    (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, (__half*)a, err, sp, 0,
+                    rm);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, x, r0,
-                  (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0);
+                  (const __nv_bfloat16*)embed, vocab, h, 0, d, g, eps, a, err, sp, 0, rm);
 }
 
 cudaError_t launch_rmsnorm(const float* h, int h_row0, int M, int d, const float* g, float eps,
                            void* a, int f32, const StepParams* sp, bool rows_from_lm0,
-                           cudaStream_t st, bool pdl) {
+                           cudaStream_t st, bool pdl, RowMap rm) {
   if (M <= 0) return cudaSuccess;
   const int* nx = nullptr;
   if (f32)
     return launch_k(pdl, rmsnorm_kernel<float>, dim3(M), dim3(256), 0, st, nx, 0,
                     (const float*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
-                    (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+                    (int*)nullptr, sp, rows_from_lm0 ? 1 : 0, rm);
   if (d % 4 == 0)
     return launch_k(pdl, rmsnorm_v4_kernel, dim3(M), dim3(256), 0, st, nx, 0,
                     (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps,
-                    (__half*)a, (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+                    (__half*)a, (int*)nullptr, sp, rows_from_lm0 ? 1 : 0, rm);
   return launch_k(pdl, rmsnorm_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, st, nx, 0,
                   (const __nv_bfloat16*)nullptr, 0, const_cast<float*>(h), h_row0, d, g, eps, a,
-                  (int*)nullptr, sp, rows_from_lm0 ? 1 : 0);
+                  (int*)nullptr, sp, rows_from_lm0 ? 1 : 0, rm);
 }
 
 cudaError_t launch_wait_timeout(int* err, cudaStream_t st) {
@@ -525,10 +588,23 @@ cudaError_t launch_merge_select(const float* lm_part, int n_part, int n, int* x,
                   select, conf, tok, unmask, state, sp);
 }
 
-cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, cudaStream_t st) {
+cudaError_t launch_merge_select_seg(const float* lm_part, int n_part, int m_lm,
+                                    const SelectSeg* segs, int n_segs, int* x, int seq_stride,
+                                    int mask_id, float tau, int fixed_k, float* conf, int* tok,
+                                    uint8_t* unmask, DecodeState* states, cudaStream_t st,
+                                    bool pdl) {
+  if (n_segs <= 0) return cudaSuccess;
+  return launch_k(pdl, merge_select_seg_kernel, dim3(n_segs), dim3(256), 0, st,
+                  reinterpret_cast<const SoftmaxState*>(lm_part), n_part, m_lm, segs, x,
+                  seq_stride, mask_id, tau, fixed_k, conf, tok, unmask, states);
+}
+
+cudaError_t launch_bf16_to_f16(void* p, size_t n, int* err, unsigned long long* inexact,
+                               cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const size_t blocks = std::min<size_t>((n + 255) / 256, 4096);
-  bf16_to_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint16_t*>(p), n, err);
+  bf16_to_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint16_t*>(p), n, err,
+                                                       inexact);
   return cudaGetLastError();
 }
 
@@ -556,7 +632,9 @@ cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl) {
   if (p.kv_planes != 2) return cudaErrorInvalidValue;
   const size_t smem = (size_t)(p.head_dim + p.L) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  return launch_k(pdl, attn_simt_kernel, dim3(p.M, p.n_heads), dim3(128), smem, st, p);
+  // batched forward: p.L is the largest key count of the tiles
+  return launch_k(pdl, attn_simt_kernel, dim3(p.tiles ? p.n_tiles : p.M, p.n_heads), dim3(128),
+                  smem, st, p);
 }
 
 

@@ -32,7 +32,8 @@ EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_gener
             "fdllm_step_debug", "fdllm_read_kv", "fdllm_kv_similarity", "fdllm_selftest_wait_timeout",
             "fdllm_gemm", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
-            "fdllm_last_error", "fdllm_launch_count", "fdllm_destroy")
+            "fdllm_last_error", "fdllm_launch_count", "fdllm_inexact_weight_count",
+            "fdllm_destroy")
 
 
 class FdllmConfig(ctypes.Structure):
@@ -63,7 +64,11 @@ class FdllmStats(ctypes.Structure):
                 ("cached_steps", ctypes.c_int32), ("n_blocks", ctypes.c_int32),
                 ("steps_per_block", ctypes.POINTER(ctypes.c_int32)),
                 ("collect_timing", ctypes.c_int32), ("refresh_ms", ctypes.c_double),
-                ("cached_ms", ctypes.c_double)]
+                ("cached_ms", ctypes.c_double), ("trace_cap", ctypes.c_int32),
+                ("trace_block", ctypes.POINTER(ctypes.c_int32)),
+                ("trace_conf", ctypes.POINTER(ctypes.c_float)),
+                ("trace_tok", ctypes.POINTER(ctypes.c_int32)),
+                ("trace_unmask", ctypes.POINTER(ctypes.c_uint8))]
 
 
 class FdllmKernelStat(ctypes.Structure):
@@ -119,6 +124,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdllm_last_error.restype = ctypes.c_char_p
     lib.fdllm_launch_count.argtypes = [vp, i32]
     lib.fdllm_launch_count.restype = ctypes.c_int64
+    lib.fdllm_inexact_weight_count.argtypes = [vp]
+    lib.fdllm_inexact_weight_count.restype = ctypes.c_int64
     lib.fdllm_destroy.argtypes = [vp]
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
                  "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv",
@@ -140,11 +147,11 @@ def _i32_ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
 
 
-def make_config(shape, max_seq: int) -> FdllmConfig:
+def make_config(shape, max_seq: int, max_batch: int = 1) -> FdllmConfig:
     s = shape.as_dict() if hasattr(shape, "as_dict") else dict(shape)
     return FdllmConfig(s["n_layers"], s["d_model"], s["n_heads"], s["n_kv_heads"], s["head_dim"],
                        s["ffn_dim"], s["vocab"], s["mask_id"], s["rope_theta"], s["rms_eps"],
-                       s["logit_scale"], DTYPES[s["dtype"]], 1, max_seq)
+                       s["logit_scale"], DTYPES[s["dtype"]], int(max_batch), max_seq)
 
 
 class TorchAllocator:
@@ -175,9 +182,10 @@ class TorchAllocator:
 
 
 # ------------------------------------------------------------------ C names
-def fdllm_create(shape, max_seq: int, device: int = 0, stream=None, allocator=None):
+def fdllm_create(shape, max_seq: int, device: int = 0, stream=None, allocator=None,
+                 max_batch: int = 1):
     lib = load_library()
-    cfg = make_config(shape, max_seq)
+    cfg = make_config(shape, max_seq, max_batch)
     ctx = ctypes.c_void_p()
     alloc_ptr = ctypes.byref(allocator.struct) if allocator is not None else None
     stream_ptr = ctypes.c_void_p(stream) if stream else None
@@ -392,49 +400,102 @@ class GenerateStats:
     steps_per_block: list
     refresh_ms: float
     cached_ms: float
+    # per-step trace (generate(..., trace=True)): block index [steps] and, per
+    # step, the block rows' confidence / argmax / unmask flag [steps, block]
+    trace_block: Optional[np.ndarray] = None
+    trace_conf: Optional[np.ndarray] = None
+    trace_tok: Optional[np.ndarray] = None
+    trace_unmask: Optional[np.ndarray] = None
+
+
+def fdllm_inexact_weight_count(ctx) -> int:
+    return int(load_library().fdllm_inexact_weight_count(ctx))
 
 
 class Decoder:
     """One decoder context (convenience wrapper over the C calls)."""
 
-    def __init__(self, shape, max_seq: int, device: int = 0, stream=None, torch_alloc: bool = True):
+    def __init__(self, shape, max_seq: int, device: int = 0, stream=None, torch_alloc: bool = True,
+                 max_batch: int = 1):
         self.shape = shape
         self.max_seq = max_seq
+        self.max_batch = max_batch
         self.device = device
         self.allocator = TorchAllocator(device) if torch_alloc else None
-        self.ctx = fdllm_create(shape, max_seq, device, stream, self.allocator)
+        self.ctx = fdllm_create(shape, max_seq, device, stream, self.allocator, max_batch)
 
     def load_weights(self, weights: Mapping[str, object]) -> None:
         fdllm_load_weights(self.ctx, weights, self.shape.dtype)
 
     def generate(self, prompt, gen_len: int, block_size: int, tau: float, cache_mode="dual",
-                 timing: bool = False, fixed_k: Optional[int] = None):
-        """Threshold decoding (tau), or with fixed_k the fixed-count strategy."""
+                 timing: bool = False, fixed_k: Optional[int] = None, trace: bool = False):
+        """Threshold decoding (tau), or with fixed_k the fixed-count strategy.
+        With trace, the returned stats carry every step's block index and the
+        block rows' confidence, argmax token and unmask flag."""
         n_blocks = gen_len // block_size if block_size > 0 else 0
         spb = (ctypes.c_int32 * max(1, n_blocks))()
         st = FdllmStats(0, 0, 0, 0, ctypes.cast(spb, ctypes.POINTER(ctypes.c_int32)), int(timing),
                         0.0, 0.0)
+        if trace:
+            cap = max(1, gen_len)                      # every step unmasks >= 1 token
+            tb = np.zeros(cap, np.int32)
+            tc = np.zeros((cap, block_size), np.float32)
+            tt = np.zeros((cap, block_size), np.int32)
+            tu = np.zeros((cap, block_size), np.uint8)
+            st.trace_cap = cap
+            st.trace_block = _i32_ptr(tb)
+            st.trace_conf = tc.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+            st.trace_tok = _i32_ptr(tt)
+            st.trace_unmask = tu.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
         if fixed_k is not None:
             out, steps = fdllm_generate_fixed_k(self.ctx, prompt, gen_len, block_size, fixed_k,
                                                 cache_mode, st)
         else:
             out, steps = fdllm_generate(self.ctx, prompt, gen_len, block_size, tau, cache_mode, st)
-        return out, steps, GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
-                                         list(spb)[:n_blocks], st.refresh_ms, st.cached_ms)
+        gs = GenerateStats(st.steps, st.refresh_steps, st.cached_steps, list(spb)[:n_blocks],
+                           st.refresh_ms, st.cached_ms)
+        if trace:
+            n = min(steps, cap)
+            gs.trace_block, gs.trace_conf = tb[:n].copy(), tc[:n].copy()
+            gs.trace_tok, gs.trace_unmask = tt[:n].copy(), tu[:n].astype(bool)
+        return out, steps, gs
+
+    def inexact_weight_count(self) -> int:
+        return fdllm_inexact_weight_count(self.ctx)
 
     def generate_batch(self, prompts, gen_len: int, block_size: int, tau: float,
-                       cache_mode="dual", timing: bool = False):
+                       cache_mode="dual", timing: bool = False, trace: bool = False):
         """Variable-length batch: returns (tokens [batch, gen_len], steps [batch],
-        GenerateStats of the totals, steps_per_block sequence by sequence)."""
+        GenerateStats of the totals, steps_per_block sequence by sequence).
+        With trace, the stats carry per-sequence traces: trace_block[i] [steps_i],
+        trace_conf[i] / trace_tok[i] / trace_unmask[i] [steps_i, block]."""
+        n = len(prompts)
         n_blocks = gen_len // block_size if block_size > 0 else 0
-        spb = (ctypes.c_int32 * max(1, n_blocks * len(prompts)))()
+        spb = (ctypes.c_int32 * max(1, n_blocks * n))()
         st = FdllmStats(0, 0, 0, 0, ctypes.cast(spb, ctypes.POINTER(ctypes.c_int32)), int(timing),
                         0.0, 0.0)
+        if trace:
+            cap = max(1, gen_len)
+            tb = np.zeros((n, cap), np.int32)
+            tc = np.zeros((n, cap, block_size), np.float32)
+            tt = np.zeros((n, cap, block_size), np.int32)
+            tu = np.zeros((n, cap, block_size), np.uint8)
+            st.trace_cap = cap
+            st.trace_block = _i32_ptr(tb)
+            st.trace_conf = tc.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+            st.trace_tok = _i32_ptr(tt)
+            st.trace_unmask = tu.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
         out, steps = fdllm_generate_batch(self.ctx, prompts, gen_len, block_size, tau, cache_mode,
                                           st)
-        return out, steps, GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
-                                         list(spb)[:n_blocks * len(prompts)], st.refresh_ms,
-                                         st.cached_ms)
+        gs = GenerateStats(st.steps, st.refresh_steps, st.cached_steps,
+                           list(spb)[:n_blocks * n], st.refresh_ms, st.cached_ms)
+        if trace:
+            k = [min(int(v), cap) for v in steps]
+            gs.trace_block = [tb[i, :k[i]].copy() for i in range(n)]
+            gs.trace_conf = [tc[i, :k[i]].copy() for i in range(n)]
+            gs.trace_tok = [tt[i, :k[i]].copy() for i in range(n)]
+            gs.trace_unmask = [tu[i, :k[i]].astype(bool) for i in range(n)]
+        return out, steps, gs
 
     def generate_device(self, prompt_dev, gen_len: int, block_size: int, tau: float, out_dev,
                         cache_mode="dual") -> int:

@@ -104,6 +104,13 @@ WORKLOADS = {
                                                    12288, 126464, 126463, 1e4, 1e-5, 30.0, "bf16",
                                                    1),
                                         256, 32, 32, 0.9, "dual"),
+    # The same two layers with the full prompt and generation lengths (L = 512):
+    # the refresh-step GEMM and attention shapes of the LLaDA-8B workload.
+    "llada8b-2layer-p256-g256": Workload("llada8b-2layer-p256-g256",
+                                         ModelShape("llada-8b-shape-2layer", 2, 4096, 32, 32,
+                                                    128, 12288, 126464, 126463, 1e4, 1e-5, 30.0,
+                                                    "bf16", 1),
+                                         256, 256, 32, 0.9, "dual"),
 }
 
 

@@ -10,10 +10,10 @@ def require_gpu():
         pytest.skip("needs a CUDA device")
 
 
-def make_decoder(shape, weights, max_seq: int):
+def make_decoder(shape, weights, max_seq: int, max_batch: int = 1):
     import os
     from kv_cache_decode_dualcache_b200 import build, fdllm
     build.build(checks=os.environ.get("FDLLM_CHECKS") == "1")
-    dec = fdllm.Decoder(shape, max_seq)
+    dec = fdllm.Decoder(shape, max_seq, max_batch=max_batch)
     dec.load_weights(weights)
     return dec

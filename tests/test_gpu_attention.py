@@ -1,7 +1,9 @@
 """The decoder's attention kernel in isolation: random queries against the
 K/V the GPU cached for a sequence, checked against the oracle's attention
 (float64) on exactly those K/V.  Covers the no-split path (many rows) and
-the split-KV path (block-sized M), MHA and GQA, ragged key counts."""
+the split-KV path (block-sized M), MHA and GQA, ragged key counts.  Query
+sets of more than 64 positions (and 128 or more query rows per KV head) run
+the tcgen05 + TMA kernel, block-sized ones the key-split kernel."""
 import numpy as np
 import pytest
 import torch
@@ -59,7 +61,8 @@ def long_setup(request):
     return shape, dec
 
 
-@pytest.mark.parametrize("M,L", [(32, 760), (7, 700), (64, 760), (16, 577)])
+@pytest.mark.parametrize("M,L", [(32, 760), (7, 700), (64, 760), (16, 577), (256, 760),
+                                 (130, 577), (760, 760)])
 def test_attention_long_keys_split_path(long_setup, M, L):
     shape, dec = long_setup
     H, hd = shape.n_heads, shape.head_dim

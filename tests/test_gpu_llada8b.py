@@ -7,7 +7,13 @@ step), then two DualCache steps on the sequence the oracle's own unmask
 decisions produce.  Each step: logits max-abs <= 3e-2 over all 32 x 126464
 logits, confidences <= 1e-3, tokens and unmask sets identical except at
 counted near ties.  The oracle runs one float64 full forward (~40 s on 16
-host cores) and two block steps (~20 s each)."""
+host cores) and two block steps (~20 s each).
+
+A later block through the production path: the generation bench.py times
+(CUDA-graph replay, programmatic dependent launches, the chain kernel) runs
+with its per-step trace, and the oracle recomputes the first two steps of
+block 3 (a decoded prefix of prompt + three blocks, a masked suffix of four
+blocks) on the GPU's own sequence."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +22,7 @@ from kv_cache_decode_dualcache_b200 import synth
 from oracle.decode import confidence, select_unmask
 from oracle.model import Model
 from tests.gpu_util import make_decoder, require_gpu
-from tests.parity import StepReport, compare_step
+from tests.parity import StepReport, compare_step, replay_gpu_trace
 
 pytestmark = pytest.mark.gpu
 
@@ -67,7 +73,19 @@ def test_llada8b_first_block_teacher_forced(full_size):
         g = dec.step_debug(x0, x, s, B, tau, "dual")
         compare_step(g, ref, masked, tau, mask, rep, z_tol=3e-2, label=f"dual step {i + 1}")
 
-    print(f"llada8b: steps {rep.steps} max|dz| {rep.max_dz:.3g} max|dconf| {rep.max_dconf:.3g} "
-          f"near-tie exemptions {rep.exempt}")
+    print(f"llada8b first block: {rep.summary()}")
     assert rep.steps >= 2
+    assert not rep.mismatches, rep.mismatches[:5]
+
+
+def test_llada8b_later_block_production_path(full_size):
+    shape, dec, model = full_size
+    P, G, B, tau = WL.prompt_len, WL.gen_len, WL.block_size, WL.tau
+    prompt = synth.make_prompt(shape, P).numpy()
+    out, steps, st = dec.generate(prompt, G, B, tau, "dual", trace=True)
+    assert len(st.trace_block) == steps and list(np.bincount(st.trace_block)) == st.steps_per_block
+    rep = replay_gpu_trace(model, prompt, G, B, tau, "dual", out, st, blocks={3},
+                           max_steps_per_block=2, label="llada8b block 3")
+    print(f"llada8b block 3 (production path): {rep.summary()}")
+    assert rep.steps >= 1
     assert not rep.mismatches, rep.mismatches[:5]

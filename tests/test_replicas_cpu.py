@@ -77,3 +77,27 @@ def test_reference_arm_runs_on_rank_0_only():
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_bench_launches_its_own_replica_ranks():
+    # bench.launch_replicas is what `bench.py --gpus N` runs when no launcher
+    # started it: N ranks under torch.distributed.run on 127.0.0.1
+    sys.path.insert(0, ROOT)
+    import bench
+    with tempfile.TemporaryDirectory() as d:
+        out = os.path.join(d, "rank0.json")
+        rc = bench.launch_replicas(2, [out], script=os.path.join(ROOT, "tests",
+                                                                   "replica_rank_cpu.py"),
+                                   timeout_s=240)
+        assert rc == 0
+        r = json.load(open(out))
+    assert r["world"] == 2 and r["ms_max"] == 150.0 and r["local_rank"] == 0
+    assert abs(r["value"] - 2 * 3 * 256 / 0.150) < 1e-6
+
+
+def test_bench_rejects_a_world_size_that_disagrees_with_gpus():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="3", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2 and "WORLD_SIZE" in r.stderr
