@@ -50,12 +50,18 @@ def _peaks():
 
 
 def _config(wl, n):
+    big = wl.shape.n_params * wl.shape.elem_bytes > 1_000_000_000
     return {"workload": wl.name, "model_shape": wl.shape.name, "prompt_len": wl.prompt_len,
             "gen_len": wl.gen_len, "block_size": wl.block_size, "tau": wl.tau,
             "cache_mode": wl.cache_mode, "batch_per_gpu": 1, "global_batch": n,
-            "weights": f"random N(0,0.02) bf16, seed {wl.shape.seed}",
-            "l2": "no flush needed: each step streams ~16 GB of weights (> 126 MB L2)",
+            "weights": f"random N(0,0.02) {wl.shape.dtype}, seed {wl.shape.seed}",
+            "l2": ("no flush needed: each step streams the weights (> 126 MB L2)" if big else
+                   "the model fits in L2: a parity configuration, not a bandwidth measurement"),
             "parallelism": "replicas" if n > 1 else "single"}
+
+
+def _dtype(wl):
+    return "f32" if wl.shape.dtype == "fp32" else "bf16"
 
 
 class ClockSampler:
@@ -241,6 +247,23 @@ def oracle_sample(wl, weights_host, step_counts, sample_layers=4):
             "sample_s": t_refresh + t_step, "threads": torch.get_num_threads()}
 
 
+def oracle_full_generate(wl, weights_host, reps=1):
+    """Small models: the float64 oracle's whole block-wise generate of the
+    workload (every step, not a sample), timed on the host cores."""
+    import torch
+    from kv_cache_decode_dualcache_b200 import synth
+    from oracle.decode import generate
+    from oracle.model import Model
+    model = Model(wl.shape.as_dict(), weights_host)
+    prompt = synth.make_prompt(wl.shape, wl.prompt_len).numpy()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        res = generate(model, prompt, wl.gen_len, wl.block_size, wl.tau, wl.cache_mode)
+    dt = (time.perf_counter() - t0) / reps
+    return {"tok_s": wl.gen_len / dt, "sample_s": dt * reps, "steps": res.steps,
+            "threads": torch.get_num_threads()}
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -326,10 +349,11 @@ def run_fdllm(args, wl):
     w = synth.make_weights(shape, device="cuda")
     dec.load_weights(w)
     want_cpu = (not args.no_cpu_baseline) and world == 1 and rank == 0
+    small = shape.n_params < 50_000_000   # the oracle runs the whole generate
     w_host = None
     if want_cpu:
         w_host = {k: v.cpu() for k, v in w.items()
-                  if not k.startswith("layers.") or int(k.split(".")[1]) < 4}
+                  if small or not k.startswith("layers.") or int(k.split(".")[1]) < 4}
     del w
     torch.cuda.empty_cache()
     prompt = replica_prompt(shape, P, rank)
@@ -393,7 +417,14 @@ def run_fdllm(args, wl):
     timing = dec.generate(prompt, G, B, tau, wl.cache_mode, timing=True)[2]
 
     cpu = None
-    if want_cpu:
+    if want_cpu and small:
+        cores = len(os.sched_getaffinity(0))
+        torch.set_num_threads(cores)
+        r = oracle_full_generate(wl, w_host)
+        cpu = {"value": r["tok_s"], "unit": "tokens/s", "cores": r["threads"], "kind": "oracle",
+               "sample": f"the whole generate of this workload ({r['steps']} denoising steps, "
+                         f"float64 oracle, {r['sample_s']:.2f} s)"}
+    elif want_cpu:
         cores = len(os.sched_getaffinity(0))
         torch.set_num_threads(cores)
         r = oracle_sample(wl, w_host, (timing.refresh_steps, timing.cached_steps))
@@ -408,7 +439,7 @@ def run_fdllm(args, wl):
         line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
                 "config": _config(wl, world),
                 "decode": {"denoising_steps_per_generation": steps_total / args.steps,
                            "steps_per_block": timing.steps_per_block,

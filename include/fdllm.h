@@ -189,7 +189,12 @@ FDLLM_API int64_t fdllm_inexact_weight_count(const fdllm_ctx* ctx);
  * unmasks a whole block per step.  Errors: ARG (gen_len or block_size < 1,
  * gen_len % block_size != 0, prompt_len < 0, prompt_len + gen_len > max_seq,
  * an id out of range or equal to the mask id in the prompt, NaN tau, unknown
- * cache_mode, NULL outputs), STATE (no weights), CUDA, TIMEOUT. */
+ * cache_mode, NULL outputs), STATE (no weights), CUDA, TIMEOUT.
+ * Precondition of the bf16 DualCache block steps: their persistent kernel
+ * runs one CTA on every SM and its phases wait on every CTA, so the decoder
+ * needs the GPU's SMs to itself while a step runs; if another stream or
+ * process holds SMs for longer than the 2 s bound, the step ends with
+ * FDLLM_ERR_TIMEOUT (the context stays usable) instead of running slower. */
 FDLLM_API int fdllm_generate(fdllm_ctx* ctx, const int32_t* prompt_ids, int prompt_len, int gen_len,
                    int block_size, float tau, int cache_mode, int32_t* out_tokens,
                    int* out_steps, fdllm_stats* stats);
@@ -221,9 +226,10 @@ FDLLM_API int fdllm_generate_fixed_k(fdllm_ctx* ctx, const int32_t* prompt_ids, 
  * fdllm_generate, per sequence).  out_tokens (host, caller-owned, batch *
  * gen_len) receives sequence i's tokens at [i * gen_len, (i + 1) * gen_len);
  * out_steps (host, batch) its step counts; stats (optional) the totals over
- * the batch (refresh_steps / cached_steps count sequence steps; with timing,
- * refresh_ms sums the global steps that held a full forward, cached_ms the
- * others), with steps_per_block (when not NULL) holding batch * gen_len /
+ * the batch (steps = the sequences' denoising steps summed; refresh_steps /
+ * cached_steps = the global steps that did / did not hold a full forward of
+ * some sequence, refresh_ms / cached_ms their summed times with timing),
+ * with steps_per_block (when not NULL) holding batch * gen_len /
  * block_size entries, sequence by sequence, and the trace (when trace_cap >
  * 0) of sequence i's step k at index i * trace_cap + k.
  *

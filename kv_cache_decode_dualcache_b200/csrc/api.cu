@@ -151,6 +151,7 @@ struct fdllm_ctx {
   // DualCache block steps of at most 32 tokens (bf16 model) run as one
   // attention launch plus one chain-kernel launch per layer (chain.cu).
   bool use_chain = true;
+  size_t attn_l2_pf_bytes = 0;  // next weights prefetched into L2 by block-step attention
   int* chain_sync = nullptr;        // per-phase done counters of one step, then the abort word
   int chain_sync_cap = 0;
   float* norm_ss = nullptr;         // chain NORM phases: partial sums of squares [32][8]
@@ -431,7 +432,7 @@ EpiParams epi_base(fdllm_ctx* ctx, int kind) {
 }
 
 int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullptr,
-                  void* o = nullptr) {
+                  void* o = nullptr, const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
   const fdllm_config& c = ctx->cfg;
   AttnParams ap{};
   ap.q = q ? q : ctx->q;
@@ -449,6 +450,9 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   ap.head_dim = c.head_dim;
   ap.n_split = 1;
   ap.keys_per_split = ((L + 63) / 64) * 64;
+  ap.err = ctx->err_dev;
+  ap.l2_pf = l2_pf;
+  ap.l2_pf_bytes = l2_pf_bytes;
   const double es = (double)ctx->esz;
   const double kv_bytes = (double)ctx->kv_planes * L * c.n_kv_heads * c.head_dim * es;
   const double qo_bytes = (ctx->f32 ? 2.0 : 4.0) * M * c.n_heads * c.head_dim * es;
@@ -497,7 +501,7 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   }
   {
     ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
-    KL(launch_attn_mma(ap, ctx->stream, ctx->pdl));
+    KL(launch_attn_mma(&ctx->m_kv, ap, ctx->stream, ctx->pdl));
   }
   return FDLLM_OK;
 }
@@ -568,8 +572,11 @@ int sync_state(fdllm_ctx* ctx);
 struct BatchFwd {
   int M = 0;                       // forward rows
   const RowInfo* rows = nullptr;   // [M]
-  const AttnTile* tiles = nullptr;
+  const RowChunk* row_chunks = nullptr;  // [M / 32]
+  const AttnTile* tiles = nullptr;     // key-split kernel (block-sized segments)
   int n_tiles = 0;
+  const AttnTile* tc_tiles = nullptr;  // tcgen05 kernel (segments of >= 128 query rows per KV head)
+  int n_tc_tiles = 0;
   int max_L = 0;
   const int* lm_src = nullptr;     // [m_lm]: forward row of LM-head row k
   int m_lm = 0;
@@ -598,6 +605,7 @@ int run_attention_batched(fdllm_ctx* ctx, int layer, const BatchFwd& bf) {
   ap.head_dim = c.head_dim;
   ap.n_split = 1;
   ap.keys_per_split = ((bf.max_L + 63) / 64) * 64;
+  ap.err = ctx->err_dev;
   ap.tiles = bf.tiles;
   ap.n_tiles = bf.n_tiles;
   ap.pages_per_seq = ctx->pages_per_seq;
@@ -605,8 +613,18 @@ int run_attention_batched(fdllm_ctx* ctx, int layer, const BatchFwd& bf) {
   ProfScope ps(ctx, "attn.batch",
                (double)ctx->kv_planes * bf.max_L * c.n_kv_heads * c.head_dim * es,
                4.0 * bf.M * c.n_heads * (double)bf.max_L * c.head_dim);
-  if (ctx->tc) KL(launch_attn_mma(ap, ctx->stream, ctx->pdl));
-  else KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
+  if (!ctx->tc) {
+    KL(launch_attn_simt(ap, ctx->stream, ctx->pdl));
+    return FDLLM_OK;
+  }
+  if (bf.n_tc_tiles > 0) {
+    AttnParams at = ap;
+    at.tiles = bf.tc_tiles;
+    at.n_tiles = bf.n_tc_tiles;
+    KL(launch_attn_tc(&ctx->m_q3, &ctx->m_kv, at, ctx->rows_cap, ctx->err_dev, ctx->stream,
+                      ctx->pdl));
+  }
+  if (bf.n_tiles > 0) KL(launch_attn_mma(&ctx->m_kv, ap, ctx->stream, ctx->pdl));
   return FDLLM_OK;
 }
 
@@ -632,6 +650,7 @@ int forward_batched(fdllm_ctx* ctx, const BatchFwd& bf) {
     ep.sp = nullptr;
     ep.pos0 = 0;
     ep.rows = bf.rows;
+    ep.chunks = bf.row_chunks;
     ep.pages_per_seq = ctx->pages_per_seq;
     ep.q_out = ctx->q;
     ep.layer = l;
@@ -743,8 +762,11 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
   int refresh = 0, cached = 0;
   double refresh_ms = 0, cached_ms = 0;
   std::vector<RowInfo> rows;
-  std::vector<AttnTile> tiles;
+  std::vector<RowChunk> rchunks;
+  std::vector<AttnTile> tiles, tc_tiles;
   std::vector<int> lm_src;
+  const int tc_mp = 128 / rep;   // positions per tcgen05 attention tile
+  const bool tc_ok = ctx->tc && ctx->use_attn_tc && rep <= 128;
   std::vector<float> h_conf;
   std::vector<int32_t> h_tok;
   std::vector<uint8_t> h_unmask;
@@ -753,7 +775,9 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
     bf.tau = tau;
     bf.fixed_k = fixed_k;
     rows.clear();
+    rchunks.clear();
     tiles.clear();
+    tc_tiles.clear();
     lm_src.clear();
     bool any_full = false;
     for (int q = 0; q < n_slots; ++q) {
@@ -766,7 +790,15 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
       const int r_hi = (full || mode == FDLLM_CACHE_PREFIX) ? S.L : s + B;
       const int q0 = (int)rows.size(), m = r_hi - r_lo;
       for (int pos = r_lo; pos < r_hi; ++pos) rows.push_back(RowInfo{pos, q});
-      if (ctx->tc) {
+      // pad to a multiple of 32 rows: every 32-row chunk is one sequence's
+      for (int c0 = q0; c0 < (int)rows.size(); c0 += 32)
+        rchunks.push_back(RowChunk{rows[c0].pos, q, std::min(32, (int)rows.size() - c0), 0});
+      while (rows.size() % 32) rows.push_back(RowInfo{-1, q});
+      if (tc_ok && m * rep >= 128) {
+        // many query rows (a full forward or a long prefix-cache segment)
+        for (int p0 = 0; p0 < m; p0 += tc_mp)
+          tc_tiles.push_back(AttnTile{q0, m, p0 * rep, S.L, q, {0, 0, 0}});
+      } else if (ctx->tc) {
         for (int r0 = 0; r0 < m * rep; r0 += rpc) tiles.push_back(AttnTile{q0, m, r0, S.L, q, {0, 0, 0}});
       } else {
         for (int j = 0; j < m; ++j) tiles.push_back(AttnTile{q0 + j, 1, 0, S.L, q, {0, 0, 0}});
@@ -788,20 +820,27 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
     }
     // one upload of the step's tables
     auto align = [](size_t v) { return (v + 255) & ~(size_t)255; };
-    const size_t o_rows = 0, o_tiles = align(rows.size() * sizeof(RowInfo));
-    const size_t o_lm = o_tiles + align(tiles.size() * sizeof(AttnTile));
+    const size_t o_rows = 0, o_chunks = align(rows.size() * sizeof(RowInfo));
+    const size_t o_tiles = o_chunks + align(rchunks.size() * sizeof(RowChunk));
+    const size_t o_tc = o_tiles + align(tiles.size() * sizeof(AttnTile));
+    const size_t o_lm = o_tc + align(tc_tiles.size() * sizeof(AttnTile));
     const size_t o_seg = o_lm + align(lm_src.size() * sizeof(int));
     const size_t used = o_seg + dev_segs.size() * sizeof(SelectSeg);
     if (used > ctx->btab_bytes) return fail(ctx, FDLLM_ERR_CUDA, "batched-step tables too large");
     std::memcpy(ctx->btab_host + o_rows, rows.data(), rows.size() * sizeof(RowInfo));
+    std::memcpy(ctx->btab_host + o_chunks, rchunks.data(), rchunks.size() * sizeof(RowChunk));
     std::memcpy(ctx->btab_host + o_tiles, tiles.data(), tiles.size() * sizeof(AttnTile));
+    std::memcpy(ctx->btab_host + o_tc, tc_tiles.data(), tc_tiles.size() * sizeof(AttnTile));
     std::memcpy(ctx->btab_host + o_lm, lm_src.data(), lm_src.size() * sizeof(int));
     std::memcpy(ctx->btab_host + o_seg, dev_segs.data(), dev_segs.size() * sizeof(SelectSeg));
     CK(cudaMemcpyAsync(ctx->btab, ctx->btab_host, used, cudaMemcpyHostToDevice, ctx->stream));
     bf.M = (int)rows.size();
     bf.rows = reinterpret_cast<const RowInfo*>(ctx->btab + o_rows);
+    bf.row_chunks = reinterpret_cast<const RowChunk*>(ctx->btab + o_chunks);
     bf.tiles = reinterpret_cast<const AttnTile*>(ctx->btab + o_tiles);
     bf.n_tiles = (int)tiles.size();
+    bf.tc_tiles = reinterpret_cast<const AttnTile*>(ctx->btab + o_tc);
+    bf.n_tc_tiles = (int)tc_tiles.size();
     bf.lm_src = reinterpret_cast<const int*>(ctx->btab + o_lm);
     bf.m_lm = (int)lm_src.size();
     bf.segs = reinterpret_cast<const SelectSeg*>(ctx->btab + o_seg);
@@ -811,6 +850,7 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
     CK(cudaMemcpyAsync(ctx->states_host, ctx->states, sizeof(DecodeState) * n_slots,
                        cudaMemcpyDeviceToHost, ctx->stream));
     if ((rc = sync_state(ctx))) return rc;  // also the error word
+    (any_full ? refresh : cached) += 1;
     if (timing) {
       float ms = 0;
       CK(cudaEventElapsedTime(&ms, e0, e1));
@@ -827,8 +867,6 @@ int generate_batch_impl(fdllm_ctx* ctx, int batch, const int32_t* const* prompts
     for (const SelectSeg& sg : bf.host_segs) {
       Slot& S = slots[sg.seq];
       const DecodeState& st = ctx->states_host[sg.seq];
-      const bool full = S.first || mode == FDLLM_CACHE_NONE;
-      (full ? refresh : cached) += 1;
       if (trace && S.steps < stats->trace_cap) {
         const size_t idx = (size_t)S.seq * stats->trace_cap + S.steps;
         if (stats->trace_block) stats->trace_block[idx] = S.b;
@@ -1075,7 +1113,14 @@ int forward_chain(fdllm_ctx* ctx, int M, int L, float* dbg, int* n_part) {
       KL(launch_chain(A, ctx->num_sms, ctx->stream, ctx->pdl && ci > 0));
     }
     if ((int)ci < c.n_layers) {
-      int rc = run_attention(ctx, (int)ci, M, L);
+      // the next chain launch streams this layer's O-proj and then gate/up
+      // weights (contiguous in the arena): their first bytes go into L2
+      // during the attention kernel, when HBM is otherwise nearly idle
+      const LayerW& lw = ctx->layers[ci];
+      const size_t wo_bytes = (size_t)c.d_model * c.n_heads * c.head_dim * 2;
+      const size_t gu_bytes = 4ull * c.ffn_dim * c.d_model;
+      const size_t pf = std::min(ctx->attn_l2_pf_bytes, wo_bytes + gu_bytes);
+      int rc = run_attention(ctx, (int)ci, M, L, nullptr, nullptr, pf ? lw.wo : nullptr, pf);
       if (rc) return rc;
     }
   }
@@ -1375,6 +1420,8 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
   if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
   if (const char* at = std::getenv("FDLLM_ATTN_TC")) ctx->use_attn_tc = std::strcmp(at, "0") != 0;
+  if (const char* pf = std::getenv("FDLLM_ATTN_PF_MB"))
+    ctx->attn_l2_pf_bytes = (size_t)std::max(0, std::min(120, std::atoi(pf))) << 20;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {
@@ -1421,8 +1468,9 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->kv_planes = ctx->f32 ? 2 : 4;
   const size_t kv_elems =
       (size_t)c.n_layers * ctx->n_pages * ctx->kv_planes * c.n_kv_heads * KV_PAGE * c.head_dim;
-  // a batched forward holds up to every slot's whole sequence
-  const size_t rows = (size_t)S * c.max_batch;
+  // a batched forward holds up to every slot's whole sequence, each padded to
+  // a multiple of 32 rows
+  const size_t rows = (size_t)((S + 31) / 32 * 32) * c.max_batch;
   ctx->rows_cap = (int)rows;
   // activation matrices: plain rows (fp32) or two-term pair rows (bf16)
   const size_t arows = ctx->f32 ? rows : pair_rows(rows);
@@ -1455,7 +1503,8 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->states = (DecodeState*)dalloc(ctx, sizeof(DecodeState) * c.max_batch);
   // batched-step tables: rows, attention tiles (one per query row at most),
   // LM-head row sources, select segments
-  ctx->btab_bytes = rows * sizeof(RowInfo) + rows * sizeof(AttnTile) +
+  ctx->btab_bytes = rows * sizeof(RowInfo) + (rows / 32) * sizeof(RowChunk) +
+                    2 * rows * sizeof(AttnTile) +
                     (size_t)lm_total * sizeof(int) + (size_t)c.max_batch * sizeof(SelectSeg) + 1024;
   ctx->btab = (uint8_t*)dalloc(ctx, ctx->btab_bytes);
   ctx->err_dev = (int*)dalloc(ctx, sizeof(int));

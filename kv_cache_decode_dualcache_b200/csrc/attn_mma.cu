@@ -68,23 +68,32 @@ FD_DEV void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Byte offset of 16-byte chunk `ch` of row `r` in a [64][HD] 2-byte tile.
-template <int HD>
+// Byte offset of 16-byte chunk `ch` of row `r` in a [ROWS][HD] 2-byte tile
+// stored as HD / 64 sub-tiles of [ROWS][64] (128-byte rows whose 16-byte
+// chunks are XOR-swizzled by row % 8: the layout TMA writes with the
+// 128-byte swizzle, and conflict-free for ldmatrix).
+template <int HD, int ROWS>
 FD_DEV uint32_t swz(int r, int ch) {
-  return (uint32_t)(r * HD * 2 + ((ch ^ (r & 7)) << 4));
+  return (uint32_t)((ch >> 3) * (ROWS * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
 }
 
 template <int HD, int NKG, int NW>
-__global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
+__global__ void __launch_bounds__(NW * 32)
+    attn_mma_kernel(const __grid_constant__ CUtensorMap kvmap, AttnParams p) {
   constexpr int NT = NW * 32;        // threads
   constexpr int TILE = 64 * HD * 2;  // bytes of one [64][HD] 2-byte tile
   constexpr int CH = HD / 8;         // 16-byte chunks per row
   constexpr int NRG = NW / NKG;      // row groups of 16 rows
-  constexpr int QT = 16 * NRG * HD * 2;  // bytes of one Q plane
+  constexpr int QR = 16 * NRG;          // query rows of the tile
+  constexpr int QT = QR * HD * 2;        // bytes of one Q plane
   constexpr int KEYS = 64 / NKG;     // keys of a tile per key group
   constexpr int NNT = KEYS / 8;      // 8-key n-tiles per key group
-  extern __shared__ __align__(128) uint8_t sm[];
-  // layout: Q hi, Q lo, then per buffer b: K hi, K lo, V hi, V lo
+  extern __shared__ __align__(128) uint8_t sm_raw[];
+  __shared__ uint64_t kv_bar[2];   // one per K/V buffer (TMA completion)
+  // layout (1024-byte aligned for the TMA swizzle): Q hi, Q lo, then per
+  // buffer b: K hi, K lo, V hi, V lo
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t q_s = smem_u32(sm);
   auto kv_s = [&](int buf, int plane) { return q_s + 2 * QT + (buf * 4 + plane) * TILE; };
 
@@ -92,6 +101,23 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
   const int rg = warp % NRG, kg = warp / NRG;
   const int H = p.n_heads, Hkv = p.n_kv_heads, rep = H / Hkv;
   const int g = blockIdx.y;
+  if (tid == 0) {
+    mbar_init(&kv_bar[0], 1);
+    mbar_init(&kv_bar[1], 1);
+    fence_mbar_init();
+    if (p.l2_pf) {
+      // this CTA's slice of the next GEMMs' weights into L2 (they do not
+      // depend on the preceding kernel, so before waiting for it)
+      const size_t n_cta = (size_t)gridDim.x * gridDim.y * gridDim.z;
+      const size_t cid = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+      const size_t per = ((p.l2_pf_bytes / n_cta) + 15) & ~(size_t)15;
+      const size_t lo = cid * per, hi = min(p.l2_pf_bytes, lo + per);
+      const uint8_t* base = reinterpret_cast<const uint8_t*>(p.l2_pf);
+      for (size_t o = lo; o < hi; o += 65536)
+        prefetch_l2_bulk(base + o, (uint32_t)min((size_t)65536, hi - o) & ~15u);
+    }
+  }
+  __syncthreads();
   pdl_trigger();
   pdl_wait();
   // one sequence: row tiles of the M query positions over keys [0, p.L);
@@ -120,25 +146,27 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
     const bool ok = r < rows_total;
     const int m = ok ? qbase + r / rep : 0, jj = ok ? r % rep : 0;
     const __half* src = qg + ((size_t)m * H + g * rep + jj) * HD + ch * 8;
-    cp_async16(q_s + swz<HD>(i, ch), src, ok ? 16 : 0);
-    cp_async16(q_s + QT + swz<HD>(i, ch), src + p.q_plane, ok ? 16 : 0);
+    cp_async16(q_s + swz<HD, QR>(i, ch), src, ok ? 16 : 0);
+    cp_async16(q_s + QT + swz<HD, QR>(i, ch), src + p.q_plane, ok ? 16 : 0);
   }
+  cp_async_commit();
+  // K/V: one cache page (64 keys) per tile, each plane [64][HD] as HD / 64
+  // TMA boxes of [64][64]; keys past key_hi are loaded and masked below
   auto load_kv = [&](int kt, int buf) {
-    const int k0 = key_lo + kt * 64;
+    const int k0 = key_lo + kt * 64;          // key_lo is a multiple of 64
     const int page = ptab[k0 / KV_PAGE];
-    const size_t plane = (size_t)Hkv * KV_PAGE * HD;
-    const size_t base = ((size_t)p.layer * p.n_pages + page) * 4 * plane + (size_t)g * KV_PAGE * HD;
-    for (int idx = tid; idx < 64 * CH; idx += NT) {
-      const int i = idx / CH, ch = idx % CH;
-      const bool ok = (k0 + i) < key_hi;
-      const size_t e = base + (size_t)(ok ? i : 0) * HD + ch * 8;
+    fence_proxy_async_smem();                 // the buffer's earlier reads come first
+    mbar_arrive_expect_tx(&kv_bar[buf], 4 * TILE);
 #pragma unroll
-      for (int pl = 0; pl < 4; ++pl)
-        cp_async16(kv_s(buf, pl) + swz<HD>(i, ch), pool + e + pl * plane, ok ? 16 : 0);
+    for (int pl = 0; pl < 4; ++pl) {
+      const int row = (((p.layer * p.n_pages + page) * 4 + pl) * Hkv + g) * 64;
+#pragma unroll
+      for (int kh = 0; kh < HD / 64; ++kh)
+        tma_load_2d(sm + (kv_s(buf, pl) - q_s) + kh * 64 * 128, &kvmap, &kv_bar[buf], kh * 64,
+                    row);
     }
   };
-  load_kv(0, 0);
-  cp_async_commit();
+  if (tid == 0 && n_kt > 0) load_kv(0, 0);
 
   const bool warp_active = row0 + rg * 16 < rows_total;
   const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // 1/sqrt(hd) * log2(e)
@@ -149,9 +177,10 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
   float lrow[2] = {0.0f, 0.0f};
 
   for (int kt = 0; kt < n_kt; ++kt) {
-    if (kt + 1 < n_kt) load_kv(kt + 1, (kt + 1) & 1);
-    cp_async_commit();
-    cp_async_wait<1>();
+    // buffer (kt + 1) & 1 was last read in iteration kt - 1 (CTA barrier since)
+    if (tid == 0 && kt + 1 < n_kt) load_kv(kt + 1, (kt + 1) & 1);
+    if (kt == 0) cp_async_wait<0>();
+    mbar_wait(&kv_bar[kt & 1], (kt >> 1) & 1u, p.err, nullptr);
     __syncthreads();
     const int buf = kt & 1;
     if (warp_active) {
@@ -162,14 +191,14 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
         uint32_t qh[4], ql[4];
-        const uint32_t qa = swz<HD>(rg * 16 + (lane & 15), 2 * kk + (lane >> 4));
+        const uint32_t qa = swz<HD, QR>(rg * 16 + (lane & 15), 2 * kk + (lane >> 4));
         ldsm_x4(q_s + qa, qh);
         ldsm_x4(q_s + QT + qa, ql);
 #pragma unroll
         for (int np = 0; np < NNT / 2; ++np) {
           uint32_t kh[4], kl[4];
           const int key = kg * KEYS + np * 16 + (lane & 7) + ((lane >> 4) << 3);
-          const uint32_t ka = swz<HD>(key, 2 * kk + ((lane >> 3) & 1));
+          const uint32_t ka = swz<HD, 64>(key, 2 * kk + ((lane >> 3) & 1));
           ldsm_x4(kv_s(buf, 0) + ka, kh);
           ldsm_x4(kv_s(buf, 1) + ka, kl);
           mma_f16(s[2 * np], qh, kh[0], kh[1]);
@@ -236,7 +265,7 @@ __global__ void __launch_bounds__(NW * 32) attn_mma_kernel(AttnParams p) {
         for (int j = 0; j < HD / 8; j += 2) {
           uint32_t vh[4], vl[4];
           const int key = kg * KEYS + kk2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-          const uint32_t va = swz<HD>(key, j + (lane >> 4));
+          const uint32_t va = swz<HD, 64>(key, j + (lane >> 4));
           ldsm_x4_t(kv_s(buf, 2) + va, vh);
           ldsm_x4_t(kv_s(buf, 3) + va, vl);
           mma_f16(oacc[j], ah, vh[0], vh[1]);
@@ -377,16 +406,17 @@ constexpr int attn_smem(int nbuf = 2) {
 
 template <int HD, int NKG, int NW>
 cudaError_t set_attr() {
-  static_assert(attn_smem<HD, NKG, NW>() <= 232448, "exceeds the 227 KB shared memory limit");
+  static_assert(attn_smem<HD, NKG, NW>() + 1024 <= 232448, "exceeds the 227 KB shared memory limit");
   return cudaFuncSetAttribute(attn_mma_kernel<HD, NKG, NW>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              attn_smem<HD, NKG, NW>());
+                              attn_smem<HD, NKG, NW>() + 1024);
 }
 
 template <int HD, int NKG, int NW>
-cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
+cudaError_t launch_hd(const CUtensorMap* kvmap, const AttnParams& p, cudaStream_t st, bool pdl) {
   // a single key tile per CTA needs one K/V buffer: two CTAs fit on an SM
-  const int smem = attn_smem<HD, NKG, NW>(p.keys_per_split <= 64 ? 1 : 2);
+  // (+1 KB: the tiles start at a 1024-byte boundary for the TMA swizzle)
+  const int smem = attn_smem<HD, NKG, NW>(p.keys_per_split <= 64 ? 1 : 2) + 1024;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = set_attr<HD, NKG, NW>();
@@ -417,19 +447,19 @@ cudaError_t launch_hd(const AttnParams& p, cudaStream_t st, bool pdl) {
   }
   cfg.attrs = la;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<HD, NKG, NW>, p);
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<HD, NKG, NW>, *kvmap, p);
 }
 
 template <int HD>
-cudaError_t launch_nkg(const AttnParams& p, cudaStream_t st, bool pdl) {
+cudaError_t launch_nkg(const CUtensorMap* kvmap, const AttnParams& p, cudaStream_t st, bool pdl) {
   // batched forwards tile every segment into 64-row tiles (attn_rows_per_cta(-1, ..))
-  if (p.tiles) return launch_hd<HD, 1, 4>(p, st, pdl);
+  if (p.tiles) return launch_hd<HD, 1, 4>(kvmap, p, st, pdl);
   const int rows = p.M * (p.n_heads / p.n_kv_heads);
-  if (rows <= 16) return launch_hd<HD, 4, 4>(p, st, pdl);
-  if (rows <= 32) return launch_hd<HD, 2, 4>(p, st, pdl);
-  if (rows <= 64) return launch_hd<HD, 1, 4>(p, st, pdl);
+  if (rows <= 16) return launch_hd<HD, 4, 4>(kvmap, p, st, pdl);
+  if (rows <= 32) return launch_hd<HD, 2, 4>(kvmap, p, st, pdl);
+  if (rows <= 64) return launch_hd<HD, 1, 4>(kvmap, p, st, pdl);
   // many query rows (full forwards, GQA): eight warps share each K/V tile
-  return launch_hd<HD, 1, 8>(p, st, pdl);
+  return launch_hd<HD, 1, 8>(kvmap, p, st, pdl);
 }
 
 }  // namespace
@@ -440,13 +470,14 @@ int attn_rows_per_cta(int M, int n_heads, int n_kv_heads) {
   return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
 }
 
-cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl) {
+cudaError_t launch_attn_mma(const CUtensorMap* kvmap, const AttnParams& p, cudaStream_t st,
+                            bool pdl) {
   if (p.kv_planes != 4 || p.n_split < 1 || p.n_split > kMaxSplit ||
       (p.tiles && (p.n_split != 1 || p.n_tiles < 1)))
     return cudaErrorInvalidValue;
   switch (p.head_dim) {
-    case 64: return launch_nkg<64>(p, st, pdl);
-    case 128: return launch_nkg<128>(p, st, pdl);
+    case 64: return launch_nkg<64>(kvmap, p, st, pdl);
+    case 128: return launch_nkg<128>(kvmap, p, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

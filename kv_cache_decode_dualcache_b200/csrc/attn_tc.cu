@@ -97,8 +97,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
   const int rep = A.rep, MP = A.mp;
-  const int m0 = blockIdx.x * MP;                       // first query position of the tile
-  const int L = p.L;
+  // one sequence: tile x covers positions [x MP, x MP + MP) of the M query
+  // positions over keys [0, p.L); batched forward: the tile table gives the
+  // segment (forward rows q0 .. q0 + m - 1 of slot seq, keys [0, L)) and the
+  // tile's first position r0 / rep within it
+  int m0 = blockIdx.x * MP, qbase = 0, m_seg = p.M, L = p.L;
+  const int* ptab = p.page_table;
+  if (p.tiles) {
+    const AttnTile tl = p.tiles[blockIdx.x];
+    m0 = tl.r0 / rep;
+    qbase = tl.q0;
+    m_seg = tl.m;
+    L = tl.L;
+    ptab = p.page_table + (size_t)tl.seq * p.pages_per_seq;
+  }
   const int n_kt = (L + 63) / 64;
   int* err = A.err;
 
@@ -130,7 +142,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (int pl = 0; pl < 2; ++pl)
         for (int kh = 0; kh < KH; ++kh)
           tma_load_3d(smem + Lay::Q_OFF + (pl * KH + kh) * Lay::Q_SUB, &qmap, q_full, kh * 64,
-                      g * rep, (pl ? A.q_lo_rows : 0) + m0);
+                      g * rep, (pl ? A.q_lo_rows : 0) + qbase + m0);
       // K tile j is free once S_j is done, V tile j once PV_j is: K runs a
       // tile ahead of V through its own ring, so S_{j+1} never waits for a
       // load issued after PV_{j-1}
@@ -139,7 +151,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (; j < n_kt && ok; ++j) {
         const int st = j % Lay::STAGES;
         const uint32_t par = ((j / Lay::STAGES) & 1u) ^ 1u;
-        const int page = p.page_table[j];   // keys [64 j, 64 j + 64) = one cache page
+        const int page = ptab[j];   // keys [64 j, 64 j + 64) = one cache page
         for (int kv = 0; kv < 2 && ok; ++kv) {
           uint64_t* full = kv ? &v_full[st] : &k_full[st];
           if (!mbar_wait(kv ? &v_empty[st] : &k_empty[st], par, err, abort_flag)) {
@@ -314,8 +326,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     if (!ok) *abort_flag = 1;
     // ---- epilogue: O / l as two-term fp16 pair rows
     const int pos_local = row / rep, jj = row - pos_local * rep;
-    const int m = m0 + pos_local;
-    const bool valid = ok && pos_local < MP && m < p.M;
+    const int m = qbase + m0 + pos_local;   // forward row
+    const bool valid = ok && pos_local < MP && m0 + pos_local < m_seg;
     if (ok) {   // warp-uniform; the stores are per row
       const float inv = valid ? 1.0f / l_run : 0.0f;
       const int hq = p.n_heads * HD, head = g * rep + jj;
@@ -367,7 +379,7 @@ cudaError_t launch_hd(const CUtensorMap* qmap, const CUtensorMap* kvmap, const A
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int tiles = (a.p.M + a.mp - 1) / a.mp;
+  const int tiles = a.p.tiles ? a.p.n_tiles : (a.p.M + a.mp - 1) / a.mp;
   return launch_k(pdl, attn_tc_kernel<HD>, dim3(tiles, a.p.n_kv_heads), dim3(AT_THREADS),
                   (size_t)AtLayout<HD>::SMEM, st, *qmap, *kvmap, a);
 }
@@ -377,7 +389,7 @@ cudaError_t launch_hd(const CUtensorMap* qmap, const CUtensorMap* kvmap, const A
 bool attn_tc_supported(const AttnParams& p) {
   const int rep = p.n_kv_heads > 0 ? p.n_heads / p.n_kv_heads : 0;
   return p.kv_planes == 4 && (p.head_dim == 64 || p.head_dim == 128) && rep >= 1 && rep <= 128 &&
-         p.tiles == nullptr && p.n_split == 1 && p.M >= 1 && p.L >= 1;
+         p.n_split == 1 && p.M >= 1 && p.L >= 1 && (p.tiles == nullptr || p.n_tiles >= 1);
 }
 
 cudaError_t launch_attn_tc(const CUtensorMap* qmap, const CUtensorMap* kvmap, const AttnParams& p,

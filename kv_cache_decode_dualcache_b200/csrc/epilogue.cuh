@@ -32,7 +32,8 @@ FD_DEV size_t kv_offset_pg(const EpiParams& ep, int page, int pos, int plane, in
          (size_t)slot * ep.head_dim + dim;
 }
 
-// Batched forward (ep.rows set): position and K/V page of token row tok.
+// Batched forward (ep.rows set): position (-1 for a padding row) and K/V
+// page of token row tok.
 FD_DEV int row_pos(const EpiParams& ep, int tok) { return __ldg(&ep.rows[tok].pos); }
 FD_DEV int row_page(const EpiParams& ep, int tok, int pos) {
   return __ldg(&ep.page_table[__ldg(&ep.rows[tok].seq) * ep.pages_per_seq + pos / KV_PAGE]);
@@ -101,6 +102,7 @@ FD_DEV void epi_chunk(const EpiParams& ep, const float* tile, int n0, int t0, in
         for (int t = 0; t < CHUNK_T && t0 + t < ep.M; ++t) {
           const int tok = t0 + t;
           const int pos = row_pos(ep, tok);
+          if (pos < 0) continue;   // padding row of the batched forward
           float y = tile[t * 128 + e];
           if (!is_v) {
             const float2 c = __ldg(&ep.rope[(size_t)pos * half + (dh % half)]);
@@ -224,55 +226,6 @@ FD_DEV __host__ int rope_slab_dim(int r, int hd) {
   return 16 * (r >> 5) + (r & 15) + ((r >> 4) & 1) * (hd / 2);
 }
 
-// The QKV epilogue of epi_regs in a batched forward: as the one-sequence
-// path, with each row's position and K/V page looked up (rows of one chunk
-// may belong to different sequences).
-FD_DEV void epi_regs_qkv_rows(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0,
-                              int e, int nt) {
-  const int lane = e & 31;
-  const int n = n0 + e;
-  const int hd = ep.head_dim, half = hd / 2;
-  const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
-  const int region = n < hq ? 0 : (n < hq + hk ? 1 : 2);  // q, k, v (uniform per warp)
-  const int rn = n - (region == 0 ? 0 : (region == 1 ? hq : hq + hk));
-  const int head = rn / hd;
-  const int r = rn - head * hd;
-  const int dim = region < 2 ? rope_slab_dim(r, hd) : r;
-  const bool second = lane >= 16;  // holds dim + hd/2 of the rotate-half pair
-#pragma unroll
-  for (int t = 0; t < CHUNK_T; ++t) {
-    if (t >= nt) break;
-    const int tok = t0 + t;
-    const int pos = row_pos(ep, tok);
-    float y = v[t];
-    if (region < 2) {
-      const float2 cs = __ldg(&ep.rope[(size_t)pos * half + (dim % half)]);
-      const float p = __shfl_xor_sync(0xffffffffu, y, 16);
-      y = second ? (y * cs.x + p * cs.y) : (y * cs.x - p * cs.y);
-    }
-    __half hi, lo;
-    split_f16(y, hi, lo);
-    if (region == 0) {
-      __half* q = reinterpret_cast<__half*>(ep.q_out);
-      const size_t i = (size_t)tok * hq + head * hd + dim;
-      if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
-        q[i] = hi;
-        q[ep.q_plane + i] = lo;
-      }
-    } else {
-      const int page = row_page(ep, tok, pos);
-      const int plane = region == 1 ? 0 : 2;
-      __half* kv = reinterpret_cast<__half*>(ep.kv_pool);
-      const size_t i0 = kv_offset_pg(ep, page, pos, plane, head, dim);
-      const size_t i1 = kv_offset_pg(ep, page, pos, plane + 1, head, dim);
-      if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
-        kv[i0] = hi;
-        kv[i1] = lo;
-      }
-    }
-  }
-}
-
 // Epilogue of one 32-token chunk held in registers by the 128 threads of an
 // epilogue warpgroup: v[t] = output feature n0 + e of token row t0 + t.
 // e = tile row = 32 * (warp % 4) + lane.  Shuffles stay within a warp and
@@ -285,7 +238,7 @@ template <bool ROWS = false>
 FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int t0, int e) {
   const int lane = e & 31;
   const int n = n0 + e;
-  const int nt = min(CHUNK_T, ep.M - t0);
+  int nt = min(CHUNK_T, ep.M - t0);
   if (nt <= 0) return;
   switch (ep.kind) {
     case EPI_STORE: {
@@ -336,10 +289,6 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
     }
     case EPI_QKV: {
       if (n >= ep.N) break;  // warp-uniform
-      if constexpr (ROWS) {
-        epi_regs_qkv_rows(ep, v, n0, t0, e, nt);
-        break;
-      }
       const int hd = ep.head_dim, half = hd / 2;
       const int hq = ep.n_heads * hd, hk = ep.n_kv_heads * hd;
       const int region = n < hq ? 0 : (n < hq + hk ? 1 : 2);  // q, k, v (uniform per warp)
@@ -347,12 +296,24 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
       const int head = rn / hd;
       const int r = rn - head * hd;
       const int dim = region < 2 ? rope_slab_dim(r, hd) : r;
-      const int pos0 = (ep.sp ? ep.sp->r0 : ep.pos0) + t0;
+      // one sequence: rows t0.. at positions pos0.. of its pages; batched
+      // forward: the chunk's sequence and first position (t0 is a multiple
+      // of 32, and a chunk's real rows come first)
+      int pos0;
+      const int* ptab = ep.page_table;
+      if constexpr (ROWS) {
+        const RowChunk ck = ep.chunks[t0 >> 5];
+        pos0 = ck.pos0;
+        ptab += ck.seq * ep.pages_per_seq;
+        nt = min(nt, ck.n);
+      } else {
+        pos0 = (ep.sp ? ep.sp->r0 : ep.pos0) + t0;
+      }
       const bool second = lane >= 16;  // holds dim + hd/2 of the rotate-half pair
       int page0 = 0, page1 = 0;
       if (region > 0) {
-        page0 = __ldg(&ep.page_table[pos0 / KV_PAGE]);
-        page1 = __ldg(&ep.page_table[(pos0 + nt - 1) / KV_PAGE]);
+        page0 = __ldg(&ptab[pos0 / KV_PAGE]);
+        page1 = __ldg(&ptab[(pos0 + nt - 1) / KV_PAGE]);
       }
       // 16 tokens at a time: the RoPE table loads of a half are issued
       // before its stores (see EPI_RESID), in fewer registers than 32.

@@ -32,9 +32,15 @@ struct StepParams {
 // Batched forward (rows of several sequences in one pass): the sequence
 // slot and absolute position of every row of the forward.  Slot q's token ids
 // live at x[q * seq_stride ..], its K/V pages at page_table[q * pages_per_seq ..].
+// Every sequence's rows start at a multiple of 32 forward rows and are padded
+// to one (pos = -1), so each 32-row chunk belongs to one sequence and holds
+// consecutive positions: RowChunk {first position, slot, real rows}.
 struct RowInfo {
   int pos;
   int seq;
+};
+struct RowChunk {
+  int pos0, seq, n, pad;
 };
 
 // Everything a GEMM epilogue needs.  Token index t is the row within the
@@ -71,6 +77,7 @@ struct EpiParams {
   const StepParams* sp;  // when set, pos0 = sp->r0 (device-side step scalars)
   const RowInfo* rows;   // batched forward: row t has position rows[t].pos in slot rows[t].seq
                          // (NULL: one sequence, row t at position pos0 + t)
+  const RowChunk* chunks;  // batched forward: the 32-row chunks of rows
   int pages_per_seq;     // batched forward: page-table entries per slot
   // Capacities (elements) of the output buffers, used only by builds with
   // FDLLM_CHECKS, where every store is bounds-checked and a violation is
@@ -167,10 +174,21 @@ struct AttnParams {
   const AttnTile* tiles;  // batched forward: one entry per CTA along x (NULL: one sequence)
   int n_tiles;
   int pages_per_seq;
+  int* err;               // device error word (a bounded wait that runs out)
+  // optional: [l2_pf, l2_pf + l2_pf_bytes) is brought into L2 while the
+  // kernel runs (the next GEMMs' weights, read during the attention's idle
+  // HBM time); split evenly over the CTAs, 16-byte granules
+  const void* l2_pf;
+  size_t l2_pf_bytes;
 };
 
-cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st, bool pdl = false);
-// tcgen05 + TMA attention for many query rows (see attn_tc.cu).  qmap: 3-D
+// kvmap: the 2-D K/V pool map of launch_attn_tc (boxes {64, 64}); the K/V
+// tiles are staged by TMA, the queries gathered with cp.async.
+cudaError_t launch_attn_mma(const CUtensorMap* kvmap, const AttnParams& p, cudaStream_t st,
+                            bool pdl = false);
+// tcgen05 + TMA attention for many query rows (see attn_tc.cu); with
+// p.tiles, one CTA per table entry: r0 / rep = the tile's first position in
+// its segment, 128 / rep positions per tile.  qmap: 3-D
 // map {head_dim, n_heads, 2 * q_lo_rows} over the q hi plane followed by the
 // lo plane (boxes {64, rep, 128 / rep}); kvmap: 2-D map {head_dim, rows} over
 // the K/V pool, one row per (layer, page, plane, KV head, slot) (boxes

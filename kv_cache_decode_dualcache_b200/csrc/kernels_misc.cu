@@ -65,7 +65,9 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const int* __restrict__ x,
   float* hr = h + (size_t)(rm.src ? rm.src[row] : h_row0 + row) * d;
   float v[VPT];
   if (x) {
-    int tok = rm.rows ? x[(size_t)rm.rows[row].seq * rm.seq_stride + rm.rows[row].pos]
+    // (a padding row of a batched forward, pos < 0, takes token 0)
+    const int rpos = rm.rows ? rm.rows[row].pos : 0;
+    int tok = rm.rows ? (rpos < 0 ? 0 : x[(size_t)rm.rows[row].seq * rm.seq_stride + rpos])
                       : x[r0 + row];
     if (tok < 0 || tok >= vocab) {
       if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
@@ -140,7 +142,9 @@ __global__ void __launch_bounds__(256) rmsnorm_v4_kernel(const int* __restrict__
   float* hr = h + (size_t)(rm.src ? rm.src[row] : h_row0 + row) * d;
   float4 v[V4];
   if (x) {
-    int tok = rm.rows ? x[(size_t)rm.rows[row].seq * rm.seq_stride + rm.rows[row].pos]
+    // (a padding row of a batched forward, pos < 0, takes token 0)
+    const int rpos = rm.rows ? rm.rows[row].pos : 0;
+    int tok = rm.rows ? (rpos < 0 ? 0 : x[(size_t)rm.rows[row].seq * rm.seq_stride + rpos])
                       : x[r0 + row];
     if (tok < 0 || tok >= vocab) {
       if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);

@@ -111,6 +111,13 @@ WORKLOADS = {
                                                     128, 12288, 126464, 126463, 1e4, 1e-5, 30.0,
                                                     "bf16", 1),
                                          256, 256, 32, 0.9, "dual"),
+    # The batched-serving workload on the 2-layer model (every GEMM, attention
+    # and LM-head shape of one global step of the batch-16 workload per layer).
+    "llada8b-2layer-batch16": Workload("llada8b-2layer-batch16",
+                                       ModelShape("llada-8b-shape-2layer", 2, 4096, 32, 32, 128,
+                                                  12288, 126464, 126463, 1e4, 1e-5, 30.0,
+                                                  "bf16", 1),
+                                       0, 256, 32, 0.9, "dual", batch=16),
 }
 
 
