@@ -151,7 +151,6 @@ struct fdllm_ctx {
   // DualCache block steps of at most 32 tokens (bf16 model) run as one
   // attention launch plus one chain-kernel launch per layer (chain.cu).
   bool use_chain = true;
-  size_t attn_l2_pf_bytes = 0;  // next weights prefetched into L2 by block-step attention
   int* chain_sync = nullptr;        // per-phase done counters of one step, then the abort word
   int chain_sync_cap = 0;
   float* norm_ss = nullptr;         // chain NORM phases: partial sums of squares [32][8]
@@ -432,7 +431,7 @@ EpiParams epi_base(fdllm_ctx* ctx, int kind) {
 }
 
 int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullptr,
-                  void* o = nullptr, const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
+                  void* o = nullptr) {
   const fdllm_config& c = ctx->cfg;
   AttnParams ap{};
   ap.q = q ? q : ctx->q;
@@ -451,8 +450,6 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   ap.n_split = 1;
   ap.keys_per_split = ((L + 63) / 64) * 64;
   ap.err = ctx->err_dev;
-  ap.l2_pf = l2_pf;
-  ap.l2_pf_bytes = l2_pf_bytes;
   const double es = (double)ctx->esz;
   const double kv_bytes = (double)ctx->kv_planes * L * c.n_kv_heads * c.head_dim * es;
   const double qo_bytes = (ctx->f32 ? 2.0 : 4.0) * M * c.n_heads * c.head_dim * es;
@@ -1113,14 +1110,7 @@ int forward_chain(fdllm_ctx* ctx, int M, int L, float* dbg, int* n_part) {
       KL(launch_chain(A, ctx->num_sms, ctx->stream, ctx->pdl && ci > 0));
     }
     if ((int)ci < c.n_layers) {
-      // the next chain launch streams this layer's O-proj and then gate/up
-      // weights (contiguous in the arena): their first bytes go into L2
-      // during the attention kernel, when HBM is otherwise nearly idle
-      const LayerW& lw = ctx->layers[ci];
-      const size_t wo_bytes = (size_t)c.d_model * c.n_heads * c.head_dim * 2;
-      const size_t gu_bytes = 4ull * c.ffn_dim * c.d_model;
-      const size_t pf = std::min(ctx->attn_l2_pf_bytes, wo_bytes + gu_bytes);
-      int rc = run_attention(ctx, (int)ci, M, L, nullptr, nullptr, pf ? lw.wo : nullptr, pf);
+      int rc = run_attention(ctx, (int)ci, M, L);
       if (rc) return rc;
     }
   }
@@ -1420,8 +1410,6 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
   if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
   if (const char* at = std::getenv("FDLLM_ATTN_TC")) ctx->use_attn_tc = std::strcmp(at, "0") != 0;
-  if (const char* pf = std::getenv("FDLLM_ATTN_PF_MB"))
-    ctx->attn_l2_pf_bytes = (size_t)std::max(0, std::min(120, std::atoi(pf))) << 20;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {

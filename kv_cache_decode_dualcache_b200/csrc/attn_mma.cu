@@ -105,17 +105,6 @@ __global__ void __launch_bounds__(NW * 32)
     mbar_init(&kv_bar[0], 1);
     mbar_init(&kv_bar[1], 1);
     fence_mbar_init();
-    if (p.l2_pf) {
-      // this CTA's slice of the next GEMMs' weights into L2 (they do not
-      // depend on the preceding kernel, so before waiting for it)
-      const size_t n_cta = (size_t)gridDim.x * gridDim.y * gridDim.z;
-      const size_t cid = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-      const size_t per = ((p.l2_pf_bytes / n_cta) + 15) & ~(size_t)15;
-      const size_t lo = cid * per, hi = min(p.l2_pf_bytes, lo + per);
-      const uint8_t* base = reinterpret_cast<const uint8_t*>(p.l2_pf);
-      for (size_t o = lo; o < hi; o += 65536)
-        prefetch_l2_bulk(base + o, (uint32_t)min((size_t)65536, hi - o) & ~15u);
-    }
   }
   __syncthreads();
   pdl_trigger();

@@ -265,14 +265,6 @@ FD_DEV uint64_t make_policy_evict_first() {
   return p;
 }
 
-// Bring [addr, addr + bytes) of global memory into L2 (bytes a multiple of
-// 16; no completion to wait for).
-FD_DEV void prefetch_l2_bulk(const void* addr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(addr)),
-               "r"(bytes)
-               : "memory");
-}
-
 FD_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -175,11 +175,6 @@ struct AttnParams {
   int n_tiles;
   int pages_per_seq;
   int* err;               // device error word (a bounded wait that runs out)
-  // optional: [l2_pf, l2_pf + l2_pf_bytes) is brought into L2 while the
-  // kernel runs (the next GEMMs' weights, read during the attention's idle
-  // HBM time); split evenly over the CTAs, 16-byte granules
-  const void* l2_pf;
-  size_t l2_pf_bytes;
 };
 
 // kvmap: the 2-D K/V pool map of launch_attn_tc (boxes {64, 64}); the K/V
