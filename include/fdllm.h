@@ -317,7 +317,11 @@ FDLLM_API int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k
  * accumulate != 0 (the residual-add epilogue of the decoder's O and down
  * projections).  splits = 0 lets the planner pick the K split; splits > 0
  * forces it (bf16 only).  Needs K % 64 == 0 and 16-byte aligned w_dev /
- * x_dev on the bf16 model.  Errors: ARG, CUDA, TIMEOUT. */
+ * x_dev on the bf16 model.  Like the decoder, the bf16 model runs shapes
+ * with N % 256 == 0 and M > 64 on pairs of SMs (tcgen05 cta_group::2, a
+ * 256-row weight tile per pair) unless FDLLM_GEMM_PAIR=0 was set when the
+ * ctx was created; the result is the same up to float32 rounding order.
+ * Errors: ARG, CUDA, TIMEOUT. */
 FDLLM_API int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev,
                          int N, int M, int K, int splits, int accumulate);
 

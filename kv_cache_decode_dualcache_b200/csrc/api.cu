@@ -126,6 +126,8 @@ struct fdllm_ctx {
   // plane) and K/V pool (2-D, one row per (layer, page, plane, head, slot))
   CUtensorMap m_q3, m_kv;
   bool use_attn_tc = true;
+  bool use_tc2 = true;          // SM-pair GEMM for the many-token forwards
+  int tc2_pairs = 0;            // resident SM pairs of that kernel (0 = not used)
   std::map<std::tuple<int, int, int, int>, GemmShape> plans;
   int64_t launches = 0;
   bool pdl = true;              // programmatic dependent launch between kernels
@@ -357,13 +359,21 @@ GemmShape make_plan(const fdllm_ctx* ctx, int N, int M, int K, bool allow_split,
   return g;
 }
 
-GemmShape plan_gemm(fdllm_ctx* ctx, int N, int M, int K, bool allow_split, bool lm = false) {
-  const auto key = std::make_tuple(N, M, K, (allow_split ? 1 : 0) + (lm ? 2 : 0));
+GemmShape plan_gemm(fdllm_ctx* ctx, int N, int M, int K, bool allow_split, bool lm = false,
+                    bool pair = false) {
+  const auto key = std::make_tuple(N, M, K, (allow_split ? 1 : 0) + (lm ? 2 : 0) + (pair ? 4 : 0));
   auto it = ctx->plans.find(key);
   if (it != ctx->plans.end()) return it->second;
-  GemmShape g = make_plan(ctx, N, M, K, allow_split, lm);
+  GemmShape g = pair ? plan_gemm_tc2(ctx->tc2_pairs, N, M, K, kWorkspaceBytes)
+                     : make_plan(ctx, N, M, K, allow_split, lm);
   ctx->plans[key] = g;
   return g;
+}
+
+// The many-token GEMMs of the bf16 model run on SM pairs where the shape
+// allows it (N a multiple of 256, more than 64 tokens, not the LM head).
+bool use_pair_gemm(const fdllm_ctx* ctx, int N, int M, bool lm) {
+  return ctx->tc && ctx->tc2_pairs > 0 && !lm && N % 256 == 0 && M > 64;
 }
 
 const CUtensorMap* act_map(CUtensorMap* maps, int nt) { return &maps[nt_index(nt)]; }
@@ -372,7 +382,8 @@ int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* 
              const void* act, CUtensorMap* amaps, int act_row0, int N, int M, int K,
              const EpiParams& ep_in, int* n_part_out = nullptr) {
   const bool lm = ep_in.kind == EPI_LMHEAD;
-  GemmShape gs = plan_gemm(ctx, N, M, K, !lm, lm);
+  const bool pair = use_pair_gemm(ctx, N, M, lm);
+  GemmShape gs = plan_gemm(ctx, N, M, K, !lm, lm, pair);
   gs.f16 = ctx->tc ? 1 : 0;  // fp16 weights and two-term fp16 activations
   EpiParams ep = ep_in;
   ep.N = N;
@@ -396,7 +407,10 @@ int run_gemm(fdllm_ctx* ctx, const char* tag, const void* w, const CUtensorMap* 
   if (ctx->tc) {
     GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
                    ctx->n_counters};
-    KL(launch_gemm_tc(wmap, act_map(amaps, gs.nt), gs, ep, sc, ctx->stream, ctx->pdl));
+    if (pair)
+      KL(launch_gemm_tc2(wmap, act_map(amaps, 128), gs, ep, sc, ctx->stream, ctx->pdl));
+    else
+      KL(launch_gemm_tc(wmap, act_map(amaps, gs.nt), gs, ep, sc, ctx->stream, ctx->pdl));
   } else {
     KL(launch_gemm_simt((const float*)w, (const float*)act, act_row0, K, gs, ep, ctx->stream,
                         ctx->pdl));
@@ -1381,6 +1395,49 @@ GemmShape plan_gemm_tc(int num_sms, int N, int M, int K, bool allow_split, size_
   return g;
 }
 
+// Plan of the SM-pair GEMM (N a multiple of 256): 256-feature x 128-token
+// units over at most max_pairs resident pairs, the K split balancing the
+// per-pair K blocks as in plan_gemm_tc.  A unit's split partials are two
+// 128 x 128 float tiles (one per CTA); one K block moves 2 x 32 KB.
+GemmShape plan_gemm_tc2(int max_pairs, int N, int M, int K, size_t ws_bytes) {
+  GemmShape g{};
+  g.N = N;
+  g.M = M;
+  g.K = K;
+  g.n_tiles = N / 128;
+  g.kb_total = (K + 63) / 64;
+  g.nt = 256;
+  g.n_tt = (M + 127) / 128;
+  const int base_units = g.n_tiles / 2 * g.n_tt;
+  const int max_split = std::min(16, std::max(1, g.kb_total / 4));
+  const double tile_bytes = 128.0 * 128 * 4;
+  double best = 1e300;
+  int best_s = 1;
+  for (int s = 1; s <= max_split; ++s) {
+    const long long units = (long long)base_units * s;
+    if (s > 1 && (size_t)units * 2 * (size_t)tile_bytes > ws_bytes) break;
+    const int pairs = (int)std::min<long long>(units, max_pairs);
+    const double split_cost = s > 1 ? (1.0 + s) * tile_bytes / (256.0 * 64 * 2) : 0.0;
+    std::vector<double> load(pairs, 0.0);
+    for (long long u = 0; u < units; ++u) {
+      const int sp = (int)(u % s);
+      const int kb = (int)((long long)(sp + 1) * g.kb_total / s - (long long)sp * g.kb_total / s);
+      load[u % pairs] += kb + 2.0 + split_cost;
+    }
+    double mx = 0.0;
+    for (double v : load) mx = std::max(mx, v);
+    if (mx < best * 0.9) {
+      best = mx;
+      best_s = s;
+    }
+  }
+  g.splits = best_s;
+  g.units = base_units * best_s;
+  g.grid = 2 * std::min(g.units, max_pairs);
+  g.kc = 16;
+  return g;
+}
+
 }  // namespace fd
 
 // =============================================================== C ABI
@@ -1410,6 +1467,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   ctx->f32 = cfg->dtype == FDLLM_DTYPE_F32;
   if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
   if (const char* at = std::getenv("FDLLM_ATTN_TC")) ctx->use_attn_tc = std::strcmp(at, "0") != 0;
+  if (const char* gp = std::getenv("FDLLM_GEMM_PAIR")) ctx->use_tc2 = std::strcmp(gp, "0") != 0;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {
@@ -1518,6 +1576,9 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
     return bail(FDLLM_ERR_OOM, "pinned host allocation failed");
   if (ctx->tc && init_kernel_attributes() != cudaSuccess)
     return bail(FDLLM_ERR_CUDA, "setting kernel shared-memory limits failed");
+  // SM pairs for the many-token GEMM: at most one per TPC, as many as can be
+  // resident at once (a persistent grid of pairs)
+  if (ctx->tc && ctx->use_tc2) ctx->tc2_pairs = std::min(gemm_tc2_max_pairs(), ctx->num_sms / 2);
   // page table (identity for one sequence), RoPE table (angles in double)
   std::vector<int> pt(ctx->n_pages);
   for (int i = 0; i < ctx->n_pages; ++i) pt[i] = i;
@@ -1996,13 +2057,20 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
   if (splits < 0 || (splits > 0 && !ctx->tc))
     return fail(ctx, FDLLM_ERR_ARG, "bad split count");
   CK(cudaSetDevice(ctx->device));
-  GemmShape gs = plan_gemm(ctx, N, M, K, true);
+  const bool pair = use_pair_gemm(ctx, N, M, false);
+  GemmShape gs = plan_gemm(ctx, N, M, K, true, false, pair);
   if (splits > 0) {
     if (splits > gs.kb_total) return fail(ctx, FDLLM_ERR_ARG, "more splits than K blocks");
     gs.splits = splits;
-    gs.units = gs.n_tiles * gs.n_tt * splits;
-    gs.grid = std::min(gs.units, ctx->num_sms);
-    if ((size_t)gs.units * (gs.nt / 2) * 128 * sizeof(float) > kWorkspaceBytes)
+    if (pair) {
+      gs.units = gs.n_tiles / 2 * gs.n_tt * splits;
+      gs.grid = 2 * std::min(gs.units, ctx->tc2_pairs);
+    } else {
+      gs.units = gs.n_tiles * gs.n_tt * splits;
+      gs.grid = std::min(gs.units, ctx->num_sms);
+    }
+    if ((size_t)gs.n_tiles * gs.n_tt * splits * (gs.nt / 2) * 128 * sizeof(float) >
+        kWorkspaceBytes)
       return fail(ctx, FDLLM_ERR_ARG, "split workspace too large");
   }
   if (gs.n_tiles * gs.n_tt > ctx->n_counters)
@@ -2024,11 +2092,14 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
       CUtensorMap wm, xm;
       gs.f16 = 0;  // bf16 operands (see the header)
       if (!make_map(ctx, &wm, w_dev, N, K, 128, false) ||
-          !make_map(ctx, &xm, x_dev, pair_rows(M), K, gs.nt, false))
+          !make_map(ctx, &xm, x_dev, pair_rows(M), K, pair ? 128 : gs.nt, false))
         return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
       GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
                      ctx->n_counters};
-      KL(launch_gemm_tc(&wm, &xm, gs, ep, sc, ctx->stream));
+      if (pair)
+        KL(launch_gemm_tc2(&wm, &xm, gs, ep, sc, ctx->stream));
+      else
+        KL(launch_gemm_tc(&wm, &xm, gs, ep, sc, ctx->stream));
     } else {
       KL(launch_gemm_simt((const float*)w_dev, (const float*)x_dev, 0, K, gs, ep, ctx->stream));
     }

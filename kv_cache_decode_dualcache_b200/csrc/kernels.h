@@ -149,6 +149,17 @@ cudaError_t launch_gemm_simt(const float* w, const float* act, int act_row0, int
                              bool pdl = false);
 int gemm_tc_smem_bytes(int nt);
 
+// The same GEMM on pairs of SMs (gemm_tc2.cu, tcgen05 cta_group::2):
+// 256-feature x 128-token output tiles, any epilogue but the LM head.  gs comes from plan_gemm_tc2; act_map has 128-row boxes (each CTA
+// of a pair loads half of a 256-row token tile).
+GemmShape plan_gemm_tc2(int max_pairs, int N, int M, int K, size_t ws_bytes);
+cudaError_t launch_gemm_tc2(const CUtensorMap* w_map, const CUtensorMap* act_map,
+                            const GemmShape& gs, const EpiParams& ep, const GemmScratch& sc,
+                            cudaStream_t st, bool pdl = false);
+int gemm_tc2_smem_bytes();
+// Pairs of CTAs that can be resident at once (0 if none or on error).
+int gemm_tc2_max_pairs();
+
 // Batched attention: CTA x-index i covers query rows [r0, r0 + rows) (rows
 // of (position, head-in-group) pairs) of one sequence's segment, whose
 // positions are rows q0 .. q0 + m - 1 of the forward; its keys are [0, L) of
