@@ -126,6 +126,7 @@ struct fdllm_ctx {
   // plane) and K/V pool (2-D, one row per (layer, page, plane, head, slot))
   CUtensorMap m_q3, m_kv;
   bool use_attn_tc = true;
+  bool use_attn_blk = true;     // block steps' attention: tcgen05 kernel with key splits
   bool use_tc2 = true;          // SM-pair GEMM for the many-token forwards
   int tc2_pairs = 0;            // resident SM pairs of that kernel (0 = not used)
   std::map<std::tuple<int, int, int, int>, GemmShape> plans;
@@ -471,11 +472,29 @@ int run_attention(fdllm_ctx* ctx, int layer, int M, int L, const void* q = nullp
   const std::string att_tag = M <= 64 ? "attn.step" : "attn.full";
   const int rep = c.n_heads / c.n_kv_heads;
   const int tc_ctas = rep <= 128 ? ((M + 128 / rep - 1) / (128 / rep)) * c.n_kv_heads : 0;
-  if (ctx->tc && ctx->use_attn_tc && M * rep >= 128 &&
-      (M > kAttnSplitMaxM || 2 * tc_ctas >= ctx->num_sms) && attn_tc_supported(ap)) {
-    // many query rows: tcgen05 + TMA attention, one CTA per 128-row query tile
-    // and KV head (block-sized forwards with few such tiles go to the
-    // key-split kernel, which spreads the keys over the SMs)
+  if (ctx->tc && ctx->use_attn_tc && ctx->use_attn_blk && M <= kAttnSplitMaxM) {
+    // block steps: tcgen05 attention over 128-key chunks, the keys split over
+    // a cluster of up to 8 CTAs per (query-row tile, KV head) so that the
+    // grid fills the SMs once
+    AttnParams bp = ap;
+    const int rows = M * rep, rp = rows <= 32 ? 32 : 64;
+    const int ctas = ((rows + rp - 1) / rp) * c.n_kv_heads;
+    const int chunks = (L + 127) / 128;
+    const int want = std::min(std::min(8, chunks), std::max(1, ctx->num_sms / ctas));
+    const int cps = (chunks + want - 1) / want;
+    bp.keys_per_split = cps * 128;
+    bp.n_split = (chunks + cps - 1) / cps;
+    if (attn_blk_supported(bp)) {
+      ProfScope ps(ctx, att_tag, kv_bytes + qo_bytes, att_flops);
+      KL(launch_attn_blk(&ctx->m_kv, bp, ctx->stream, ctx->pdl));
+      return FDLLM_OK;
+    }
+  }
+  const bool tc_path = ctx->tc && ctx->use_attn_tc && M * rep >= 128 &&
+                       (M > kAttnSplitMaxM || 2 * tc_ctas >= ctx->num_sms) &&
+                       attn_tc_supported(ap);
+  if (tc_path) {
+    // tcgen05 + TMA attention
     CUtensorMap qm;
     const CUtensorMap* qmap = &ctx->m_q3;
     int q_lo_rows = ctx->rows_cap;
@@ -635,7 +654,16 @@ int run_attention_batched(fdllm_ctx* ctx, int layer, const BatchFwd& bf) {
     KL(launch_attn_tc(&ctx->m_q3, &ctx->m_kv, at, ctx->rows_cap, ctx->err_dev, ctx->stream,
                       ctx->pdl));
   }
-  if (bf.n_tiles > 0) KL(launch_attn_mma(&ctx->m_kv, ap, ctx->stream, ctx->pdl));
+  if (bf.n_tiles > 0) {
+    // the block segments: tcgen05 block attention (64-row tiles, every key
+    // of the segment's sequence per CTA), else the mma.sync kernel
+    AttnParams bp = ap;
+    bp.keys_per_split = ((bf.max_L + 127) / 128) * 128;
+    if (ctx->use_attn_blk && attn_blk_supported(bp))
+      KL(launch_attn_blk(&ctx->m_kv, bp, ctx->stream, ctx->pdl));
+    else
+      KL(launch_attn_mma(&ctx->m_kv, ap, ctx->stream, ctx->pdl));
+  }
   return FDLLM_OK;
 }
 
@@ -1468,6 +1496,7 @@ int fdllm_create(const fdllm_config* cfg, int device, void* cuda_stream,
   if (const char* ch = std::getenv("FDLLM_CHAIN")) ctx->use_chain = std::strcmp(ch, "0") != 0;
   if (const char* at = std::getenv("FDLLM_ATTN_TC")) ctx->use_attn_tc = std::strcmp(at, "0") != 0;
   if (const char* gp = std::getenv("FDLLM_GEMM_PAIR")) ctx->use_tc2 = std::strcmp(gp, "0") != 0;
+  if (const char* ab = std::getenv("FDLLM_ATTN_BLK")) ctx->use_attn_blk = std::strcmp(ab, "0") != 0;
   ctx->tc = !ctx->f32;
   ctx->esz = ctx->f32 ? 4 : 2;
   auto bail = [&](int code, const std::string& m) {

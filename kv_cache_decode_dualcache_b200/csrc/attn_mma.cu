@@ -473,6 +473,7 @@ cudaError_t launch_attn_mma(const CUtensorMap* kvmap, const AttnParams& p, cudaS
 
 cudaError_t gemm_tc_init_attributes();
 cudaError_t gemm_tc2_init_attributes();
+cudaError_t attn_blk_init_attributes();
 
 cudaError_t init_kernel_attributes() {
   cudaError_t e = set_attr<64, 1, 4>();
@@ -485,6 +486,7 @@ cudaError_t init_kernel_attributes() {
   if (e == cudaSuccess) e = set_attr<128, 1, 8>();
   if (e == cudaSuccess) e = gemm_tc_init_attributes();
   if (e == cudaSuccess) e = gemm_tc2_init_attributes();
+  if (e == cudaSuccess) e = attn_blk_init_attributes();
   if (e == cudaSuccess) e = chain_init_attributes();
   if (e == cudaSuccess) e = attn_tc_init_attributes();
   return e;

@@ -203,6 +203,16 @@ bool attn_tc_supported(const AttnParams& p);
 cudaError_t launch_attn_tc(const CUtensorMap* qmap, const CUtensorMap* kvmap, const AttnParams& p,
                            int q_lo_rows, int* err, cudaStream_t st, bool pdl = false);
 cudaError_t attn_tc_init_attributes();
+// tcgen05 + TMA attention of block queries (see attn_blk.cu).  One
+// sequence: at most 64 query positions, n_split <= 8 key splits of
+// keys_per_split (a multiple of 128) keys each, one thread-block cluster per
+// (query-row tile, KV head).  Batched forward (p.tiles): one CTA per table
+// entry of 64 query rows, n_split = 1, keys_per_split >= every segment's L.
+// kvmap as for launch_attn_tc.
+bool attn_blk_supported(const AttnParams& p);
+cudaError_t launch_attn_blk(const CUtensorMap* kvmap, const AttnParams& p, cudaStream_t st,
+                            bool pdl = false);
+cudaError_t attn_blk_init_attributes();
 // Query rows per CTA of launch_attn_mma for M query positions (16, 32 or 64).
 int attn_rows_per_cta(int M, int n_heads, int n_kv_heads);
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t st, bool pdl = false);

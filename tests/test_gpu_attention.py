@@ -1,9 +1,11 @@
 """The decoder's attention kernel in isolation: random queries against the
 K/V the GPU cached for a sequence, checked against the oracle's attention
 (float64) on exactly those K/V.  Covers the no-split path (many rows) and
-the split-KV path (block-sized M), MHA and GQA, ragged key counts.  Query
-sets of more than 64 positions (and 128 or more query rows per KV head) run
-the tcgen05 + TMA kernel, block-sized ones the key-split kernel."""
+the split-KV path (block-sized M), MHA and GQA, ragged key counts.  Every
+query set runs the tcgen05 + TMA kernel (block-sized ones with the keys
+split over a thread-block cluster); with FDLLM_ATTN_BLK=0 the block-sized
+ones run the mma.sync key-split kernel instead (the batched forward's
+block tiles use that one), and both are checked."""
 import numpy as np
 import pytest
 import torch
@@ -16,11 +18,20 @@ from tests.gpu_util import make_decoder, require_gpu
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["small-bf16", "small-gqa-bf16"])
+def _decoder(shape, max_seq, blk):
+    return make_decoder(shape, synth.make_weights(shape, device="cpu"), max_seq,
+                        env={"FDLLM_ATTN_BLK": "1" if blk else "0"})
+
+
+PARAMS = [("small-bf16", True), ("small-gqa-bf16", True), ("small-bf16", False),
+          ("small-gqa-bf16", False)]
+
+
+@pytest.fixture(scope="module", params=PARAMS, ids=lambda p: f"{p[0]}-{'tc' if p[1] else 'mma'}")
 def setup(request):
     require_gpu()
-    shape = synth.SHAPES[request.param]
-    dec = make_decoder(shape, synth.make_weights(shape, device="cpu"), 256)
+    shape = synth.SHAPES[request.param[0]]
+    dec = _decoder(shape, 256, request.param[1])
     prompt = synth.make_prompt(shape, 150).numpy()
     x = np.concatenate([prompt, np.full(50, shape.mask_id)])
     dec.step_debug(x, x, 150, 32, 0.9, "dual", logits=False)   # fills the cache for 200 positions
@@ -50,11 +61,11 @@ def test_attention_matches_oracle(setup, M, L, qscale):
     assert err <= tol, (err, tol)
 
 
-@pytest.fixture(scope="module", params=["small-bf16", "small-gqa-bf16"])
+@pytest.fixture(scope="module", params=PARAMS, ids=lambda p: f"{p[0]}-{'tc' if p[1] else 'mma'}")
 def long_setup(request):
     require_gpu()
-    shape = synth.SHAPES[request.param]
-    dec = make_decoder(shape, synth.make_weights(shape, device="cpu"), 1024)
+    shape = synth.SHAPES[request.param[0]]
+    dec = _decoder(shape, 1024, request.param[1])
     prompt = synth.make_prompt(shape, 700).numpy()
     x = np.concatenate([prompt, np.full(60, shape.mask_id)])
     dec.step_debug(x, x, 700, 32, 0.9, "dual", logits=False)   # caches 760 positions
@@ -81,3 +92,36 @@ def test_attention_long_keys_split_path(long_setup, M, L):
         got = from_pair_rows(o, M).double().cpu().numpy()
         assert np.isfinite(got).all()
         assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
+
+
+@pytest.fixture(scope="module", params=PARAMS, ids=lambda p: f"{p[0]}-{'tc' if p[1] else 'mma'}")
+def very_long_setup(request):
+    require_gpu()
+    shape = synth.SHAPES[request.param[0]]
+    dec = _decoder(shape, 1280, request.param[1])
+    prompt = synth.make_prompt(shape, 1150).numpy()
+    x = np.concatenate([prompt, np.full(50, shape.mask_id)])
+    dec.step_debug(x, x, 1150, 32, 0.9, "dual", logits=False)   # caches 1200 positions
+    return shape, dec
+
+
+@pytest.mark.parametrize("M,L", [(32, 1200), (16, 1100), (64, 1200), (5, 1030)])
+def test_attention_many_chunks_per_cta(very_long_setup, M, L):
+    """More 128-key chunks than a cluster has CTAs: every split of the block
+    attention runs several chunks with the online softmax between them."""
+    shape, dec = very_long_setup
+    H, hd = shape.n_heads, shape.head_dim
+    g = torch.Generator(device="cuda").manual_seed(7 * M + L)
+    q = torch.randn(M, H, hd, generator=g, device="cuda") * 8.0
+    qh, ql = split(q, torch.float16)
+    qd = torch.stack([qh, ql]).contiguous()
+    rows = 2 * ((M + 31) // 32) * 32
+    o = torch.full((rows, H * hd), float("nan"), device="cuda", dtype=torch.float16)
+    fdllm.fdllm_attention(dec.ctx, qd, o, 1, L)
+    torch.cuda.synchronize()
+    k, v = dec.read_kv(1, 0, L)
+    qx = (qh.double() + ql.double()).cpu().numpy()
+    ref = attention(qx, k.astype(np.float64), v.astype(np.float64)).reshape(M, H * hd)
+    got = from_pair_rows(o, M).double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())

@@ -74,11 +74,14 @@ def test_batch_tiny_matches_single_and_oracle(mode, slots):
 
 @pytest.mark.parametrize("name", ["small-bf16", "small-gqa-bf16"])
 @pytest.mark.parametrize("mode", ["dual", "prefix"])
-def test_batch_bf16_steps_match_oracle(name, mode):
+@pytest.mark.parametrize("blk", ["1", "0"], ids=["attn-tc", "attn-mma"])
+def test_batch_bf16_steps_match_oracle(name, mode, blk):
+    """Block segments through the tcgen05 block attention (default) and the
+    mma.sync one (FDLLM_ATTN_BLK=0)."""
     require_gpu()
     shape = synth.SHAPES[name]
     w = synth.make_weights(shape, device="cpu")
-    dec = make_decoder(shape, w, 256, max_batch=3)
+    dec = make_decoder(shape, w, 256, max_batch=3, env={"FDLLM_ATTN_BLK": blk})
     lens, G, B, tau = [128, 40, 71, 200, 0], 32, 16, 0.9
     prompts = _prompts(shape, lens, salt0=30)
     out, steps, st = dec.generate_batch(prompts, G, B, tau, mode, trace=True)

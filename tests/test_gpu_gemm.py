@@ -1,8 +1,6 @@
 """The decoder's GEMM (tcgen05 on the bf16 model) against a float64 matmul of
 the same operands: bf16 weights times two-term (hi + lo) activations, over
 token-tile widths, K splits and ragged N / M."""
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -17,16 +15,9 @@ pytestmark = pytest.mark.gpu
 def _decoder(pair):
     require_gpu()
     shape = synth.with_layers(synth.SMALL_BF16, 1)
-    old = os.environ.get("FDLLM_GEMM_PAIR")
-    os.environ["FDLLM_GEMM_PAIR"] = "1" if pair else "0"
-    try:
-        # 2 x 1024 rows: tile counters for the 24576 x 512-token case
-        return make_decoder(shape, synth.make_weights(shape, device="cpu"), 1024, max_batch=2)
-    finally:
-        if old is None:
-            del os.environ["FDLLM_GEMM_PAIR"]
-        else:
-            os.environ["FDLLM_GEMM_PAIR"] = old
+    # 2 x 1024 rows: tile counters for the 24576 x 512-token case
+    return make_decoder(shape, synth.make_weights(shape, device="cpu"), 1024, max_batch=2,
+                        env={"FDLLM_GEMM_PAIR": "1" if pair else "0"})
 
 
 @pytest.fixture(scope="module")
