@@ -134,9 +134,9 @@ def roofline_from_profile(stats, hbm, tf_sustained, peak_kind, traffic):
                "unit": "TFLOP/s"}
     per_launch_bytes = sum(s["bytes"] for s in g) / max(1, launches)
     out["frac"] = round(out["achieved"] / out["peak"], 4)
-    out["traffic"] = traffic if key == "step" else None
+    out["traffic"] = traffic.get(key)
     out["kernel"] = ("chain_kernel (DualCache block-step GEMMs + norms)" if key == "step"
-                     else "gemm_tc_kernel (full-forward launches)")
+                     else "gemm_tc2_kernel (full-forward GEMMs on SM pairs)")
     out["share_of_kernel_time"] = round(ms / total_all, 3)
     out["launches"] = launches
     out["algorithmic_bytes_per_launch"] = round(per_launch_bytes)
@@ -168,24 +168,31 @@ def block_step_roofline(wl, cached_ms, hbm):
             "note": "weights (bf16) + K,V of all L positions read once per block step"}
 
 
-def _traffic_record():
-    """ncu DRAM bytes per launch recorded for the current chain-kernel source,
-    if any (null once the kernel has changed since the counters were taken)."""
+def _traffic_record(record, source):
+    """ncu DRAM bytes per launch recorded in profiles/<record> for the current
+    source of the kernel (csrc/<source>), if any: null once the kernel has
+    changed since the counters were taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "chain_traffic.txt")
+    path = os.path.join(ROOT, "profiles", record)
     try:
         rec = {}
         for line in open(path):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 rec[k.strip()] = v.strip()
-        src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", "chain.cu"),
-                    "rb").read()
-        if rec.get("chain_sha256") == hashlib.sha256(src).hexdigest():
+        src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", source),
+                   "rb").read()
+        if rec.get("source_sha256") == hashlib.sha256(src).hexdigest():
             return float(rec["bytes_per_launch"])
     except Exception:
         pass
     return None
+
+
+def traffic_records():
+    """Per kernel class of roofline_from_profile: the recorded DRAM bytes."""
+    return {"step": _traffic_record("chain_traffic.txt", "chain.cu"),
+            "full": _traffic_record("gemm_tc2_traffic.txt", "gemm_tc2.cu")}
 
 
 # ---------------------------------------------------------------- replicas
@@ -413,7 +420,7 @@ def run_fdllm(args, wl):
     prof = fdllm.fdllm_profile_read(dec.ctx)
     fdllm.fdllm_profile_enable(dec.ctx, False)
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
-    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, _traffic_record())
+    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, traffic_records())
     timing = dec.generate(prompt, G, B, tau, wl.cache_mode, timing=True)[2]
 
     cpu = None
@@ -519,7 +526,7 @@ def run_fdllm_batch(args, wl):
     prof = fdllm.fdllm_profile_read(dec.ctx)
     fdllm.fdllm_profile_enable(dec.ctx, False)
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
-    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, _traffic_record())
+    roof = roofline_from_profile(prof, hbm, tf_sust, peak_kind, traffic_records())
     if rank == 0:
         cfg = _config(wl, world)
         cfg.update({"prompt_lens": lens, "batch_per_gpu": wl.batch,

@@ -1,7 +1,7 @@
 """bench.py's reporting arithmetic, on synthetic profile records (no GPU):
 the dominant kernel class, achieved = algorithmic bytes (FLOPs) / time,
 frac = achieved / peak, the block step against 8 TB/s, and the DRAM
-traffic record of the current chain kernel."""
+traffic records of the current chain and SM-pair GEMM kernels."""
 import hashlib
 import os
 import sys
@@ -23,7 +23,8 @@ def test_hbm_bound_class_dominates():
     stats = [_stat("chain.step", 33, 100.0, gbytes=300.0),          # 3 TB/s
              _stat("gemm.qkv.full", 32, 40.0, tflop=20.0),
              _stat("attn.step", 32, 10.0, gbytes=0.5)]
-    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured", 123.0)
+    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured",
+                                    {"step": 123.0, "full": 77.0})
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert abs(r["achieved"] - 3000.0) < 1e-6
     assert abs(r["frac"] - 0.5) < 1e-9
@@ -35,11 +36,15 @@ def test_tensor_bound_class_dominates():
     stats = [_stat("chain.step", 33, 10.0, gbytes=30.0),
              _stat("gemm.qkv.full", 32, 40.0, tflop=20.0),
              _stat("gemm.ffn_up.full", 32, 60.0, tflop=40.0)]
-    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured", 123.0)
+    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured",
+                                    {"step": 123.0, "full": None})
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["achieved"] - 60.0 / 0.1) < 1e-6       # 60 TFLOP in 100 ms
     assert abs(r["frac"] - 600.0 / 1400.0) < 1e-4
     assert r["traffic"] is None                          # no capture of this class
+    r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured",
+                                    {"step": 123.0, "full": 77.0})
+    assert r["traffic"] == 77.0
 
 
 def test_block_step_roofline_of_the_headline_workload():
@@ -52,13 +57,15 @@ def test_block_step_roofline_of_the_headline_workload():
     assert abs(r["frac_of_measured"] - want / 4e-3 / 6e12) < 1e-4
 
 
-def test_traffic_record_follows_the_chain_kernel_source():
-    path = os.path.join(ROOT, "profiles", "chain_traffic.txt")
-    rec = dict(l.split(":", 1) for l in open(path) if ":" in l and not l.startswith("#"))
-    src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", "chain.cu"),
-               "rb").read()
-    got = bench._traffic_record()
-    if rec["chain_sha256"].strip() == hashlib.sha256(src).hexdigest():
-        assert got == float(rec["bytes_per_launch"])
-    else:                       # kernel changed since the counters were taken
-        assert got is None
+def test_traffic_records_follow_their_kernel_sources():
+    for record, source, key in (("chain_traffic.txt", "chain.cu", "step"),
+                                ("gemm_tc2_traffic.txt", "gemm_tc2.cu", "full")):
+        path = os.path.join(ROOT, "profiles", record)
+        rec = dict(l.split(":", 1) for l in open(path) if ":" in l and not l.startswith("#"))
+        src = open(os.path.join(ROOT, "kv_cache_decode_dualcache_b200", "csrc", source),
+                   "rb").read()
+        got = bench.traffic_records()[key]
+        if rec["source_sha256"].strip() == hashlib.sha256(src).hexdigest():
+            assert got == float(rec["bytes_per_launch"])
+        else:                       # kernel changed since the counters were taken
+            assert got is None
