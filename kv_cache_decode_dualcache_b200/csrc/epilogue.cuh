@@ -317,6 +317,15 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
       }
       // 16 tokens at a time: the RoPE table loads of a half are issued
       // before its stores (see EPI_RESID), in fewer registers than 32.
+      // Stores: lanes 4k .. 4k + 3 hold dims d .. d + 3 (the slab
+      // permutation keeps 16-lane runs of consecutive dims); per 4 tokens
+      // they transpose their (hi, lo) values in two shuffle rounds, so that
+      // lane 4k + j stores dims d .. d + 3 of token j: 8-byte stores, a
+      // quarter of the store instructions of one 2-byte store per value
+      // (the narrow stores, each waiting for write credits, are what bound
+      // this epilogue).
+      const int l4 = lane & 3;
+      const int dim4 = dim - l4;   // first dim of the lane quad (a multiple of 4)
 #pragma unroll
       for (int h16 = 0; h16 < CHUNK_T; h16 += 16) {
         if (h16 >= nt) break;
@@ -329,33 +338,56 @@ FD_DEV void epi_regs(const EpiParams& ep, const float (&v)[CHUNK_T], int n0, int
                         : make_float2(1.0f, 0.0f);
         }
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
+        for (int t = 0; t < 16; t += 4) {
           if (h16 + t >= nt) break;
-          float y = v[h16 + t];
-          if (region < 2) {
-            const float p = __shfl_xor_sync(0xffffffffu, y, 16);
-            y = second ? (y * cs[t].x + p * cs[t].y) : (y * cs[t].x - p * cs[t].y);
+          // x[j] = (hi, lo) of token t + j at this lane's dim
+          uint32_t x[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float y = v[h16 + t + j];
+            if (region < 2) {
+              const float p = __shfl_xor_sync(0xffffffffu, y, 16);
+              y = second ? (y * cs[t + j].x + p * cs[t + j].y) : (y * cs[t + j].x - p * cs[t + j].y);
+            }
+            __half hi, lo;
+            split_f16(y, hi, lo);
+            const __half2 hl = __halves2half2(hi, lo);
+            x[j] = *reinterpret_cast<const uint32_t*>(&hl);
           }
-          __half hi, lo;
-          split_f16(y, hi, lo);
-          const int tok = t0 + h16 + t;
-          const int pos = pos0 + h16 + t;
+          // 4 x 4 transpose over the lane quad: swap bit 0, then bit 1, of
+          // (lane, token); afterwards x[k] = token t + l4 at dim dim4 + k
+          {
+            const bool b0 = l4 & 1;
+            const uint32_t s0 = __shfl_xor_sync(0xffffffffu, b0 ? x[0] : x[1], 1);
+            const uint32_t s1 = __shfl_xor_sync(0xffffffffu, b0 ? x[2] : x[3], 1);
+            if (b0) { x[0] = s0; x[2] = s1; } else { x[1] = s0; x[3] = s1; }
+            const bool b1 = l4 & 2;
+            const uint32_t s2 = __shfl_xor_sync(0xffffffffu, b1 ? x[0] : x[2], 2);
+            const uint32_t s3 = __shfl_xor_sync(0xffffffffu, b1 ? x[1] : x[3], 2);
+            if (b1) { x[0] = s2; x[1] = s3; } else { x[2] = s2; x[3] = s3; }
+          }
+          const uint2 hi4 = make_uint2(__byte_perm(x[0], x[1], 0x5410), __byte_perm(x[2], x[3], 0x5410));
+          const uint2 lo4 = make_uint2(__byte_perm(x[0], x[1], 0x7632), __byte_perm(x[2], x[3], 0x7632));
+          const int tt = h16 + t + l4;
+          if (tt >= nt) continue;
+          const int tok = t0 + tt;
+          const int pos = pos0 + tt;
           if (region == 0) {
             __half* q = reinterpret_cast<__half*>(ep.q_out);
-            const size_t i = (size_t)tok * hq + head * hd + dim;
-            if (FD_CHECK(ep.q_plane + i < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
-              q[i] = hi;
-              q[ep.q_plane + i] = lo;
+            const size_t i = (size_t)tok * hq + head * hd + dim4;
+            if (FD_CHECK(ep.q_plane + i + 3 < ep.cap_q, ep.check, 4, ep.q_plane + i, ep.cap_q)) {
+              *reinterpret_cast<uint2*>(q + i) = hi4;
+              *reinterpret_cast<uint2*>(q + ep.q_plane + i) = lo4;
             }
           } else {
             const int page = (pos / KV_PAGE == pos0 / KV_PAGE) ? page0 : page1;
             const int plane = region == 1 ? 0 : 2;
             __half* kv = reinterpret_cast<__half*>(ep.kv_pool);
-            const size_t i0 = kv_offset_pg(ep, page, pos, plane, head, dim);
-            const size_t i1 = kv_offset_pg(ep, page, pos, plane + 1, head, dim);
-            if (FD_CHECK(i1 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
-              kv[i0] = hi;
-              kv[i1] = lo;
+            const size_t i0 = kv_offset_pg(ep, page, pos, plane, head, dim4);
+            const size_t i1 = kv_offset_pg(ep, page, pos, plane + 1, head, dim4);
+            if (FD_CHECK(i1 + 3 < ep.cap_kv, ep.check, 5, i1, ep.cap_kv)) {
+              *reinterpret_cast<uint2*>(kv + i0) = hi4;
+              *reinterpret_cast<uint2*>(kv + i1) = lo4;
             }
           }
         }
