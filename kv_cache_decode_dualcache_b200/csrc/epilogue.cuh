@@ -420,19 +420,24 @@ FD_DEV void epi_staged_f16(const EpiParams& ep, const float (&v)[CHUNK_T], int n
   __half* st_hi = st;                 // [32 tokens][128 features]
   __half* st_lo = st + CHUNK_T * 128;
   if (ep.kind == EPI_SWIGLU) {
-    // 64 outputs per tile: feature j0 + f, f = 16 * (e / 32) + lane % 16
+    // 64 outputs per tile: feature j0 + f, f = 16 * (e / 32) + lane % 16.
+    // Lane l < 16 holds the gate and lane l + 16 the up value of feature f;
+    // per pair of tokens they swap one value, so that the gate lane computes
+    // token t and the up lane token t + 1: every lane of a SiLU instruction
+    // does useful work.
     const int F = ep.N / 2;
     const bool up = lane >= 16;
     const int f = 16 * (e >> 5) + (lane & 15);
 #pragma unroll
-    for (int t = 0; t < CHUNK_T; ++t) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[t], 16);
-      const float g = up ? p : v[t];
-      const float u = up ? v[t] : p;
+    for (int t = 0; t < CHUNK_T; t += 2) {
+      const float recv = __shfl_xor_sync(0xffffffffu, up ? v[t] : v[t + 1], 16);
+      const float g = up ? recv : v[t];        // gate lane: (g_t, u_t); up lane: (g_t+1, u_t+1)
+      const float u = up ? v[t + 1] : recv;
       __half hi, lo;
-      split_f16(silu_f(g) * u, hi, lo);
-      if (!up) st_hi[t * 128 + f] = hi;
-      else st_lo[t * 128 + f] = lo;
+      split_f16(silu_fast(g) * u, hi, lo);
+      const int tt = t + (up ? 1 : 0);
+      st_hi[tt * 128 + f] = hi;
+      st_lo[tt * 128 + f] = lo;
     }
     named_bar(bar, EPI_THREADS);
     // rows: 32 tokens x {hi, lo}; 64 features = 8 chunks of 8 per row
