@@ -42,9 +42,9 @@
 //
 // 256 threads (the two warps of each TMEM lane quadrant split the rows of a
 // score read-out and the features of O); thread 0 issues the TMA loads and
-// the MMAs; every wait is
-// bounded (WAIT_LIMIT_NS): a timeout sets DEV_ERR_TIMEOUT and the CTA skips
-// its remaining work but still reaches both cluster barriers.
+// the MMAs.  Every wait is bounded (WAIT_LIMIT_NS): a timeout sets
+// DEV_ERR_TIMEOUT and the CTA skips its remaining work but still reaches
+// both cluster barriers.
 #include "common.cuh"
 #include "kernels.h"
 
