@@ -234,31 +234,35 @@ __global__ void __launch_bounds__(BLK_THREADS, 1)
   }
 
   const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;   // 1/sqrt(hd) * log2(e)
+  // S^T = K Qs^T of chunk c (thread 0): once its K has landed; everyone
+  // waits on s_done for it.  Chunk 0's is issued here, chunk c + 1's right
+  // behind chunk c's PV product, so that it runs while the threads finish
+  // chunk c and its K was loaded during chunk c's softmax.
+  auto issue_s = [&](int c) {
+    if (!mbar_wait(k_full, c & 1u, err, abort_flag)) {
+      *abort_flag = 1;
+      return;
+    }
+    ++k_seen;
+    tc_fence_after();
+    const uint32_t idesc = idesc_f32acc(2 * RP, true);
+    const uint32_t kbase = smem_u32(smem + Lay::KV_OFF);
+    const uint32_t qb = smem_u32(smem + Lay::Q_OFF);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc_mma(tmem, smem_desc_sw128(kbase + t * Lay::PLANE + kh * 2 * Lay::PAGE_SUB + k * 32),
+                 smem_desc_sw128(qb + kh * Lay::Q_SUB + k * 32), idesc,
+                 (t > 0 || kh > 0 || k > 0) ? 1u : 0u);
+    tc_commit(s_done);
+  };
   bool ok = true;
+  if (tid == 0 && n_ch > 0) issue_s(0);
   for (int c = 0; c < n_ch && ok; ++c) {
     const uint32_t ph = c & 1u;
-    // ---- S^T = K Qs^T (thread 0 issues; everyone waits for it)
-    if (tid == 0) {
-      if (!mbar_wait(k_full, ph, err, abort_flag)) {
-        *abort_flag = 1;
-      } else {
-        ++k_seen;
-        tc_fence_after();
-        const uint32_t idesc = idesc_f32acc(2 * RP, true);
-        const uint32_t kbase = smem_u32(smem + Lay::KV_OFF);
-        const uint32_t qb = smem_u32(smem + Lay::Q_OFF);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int kh = 0; kh < KH; ++kh)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              tc_mma(tmem, smem_desc_sw128(kbase + t * Lay::PLANE + kh * 2 * Lay::PAGE_SUB + k * 32),
-                     smem_desc_sw128(qb + kh * Lay::Q_SUB + k * 32), idesc,
-                     (t > 0 || kh > 0 || k > 0) ? 1u : 0u);
-        tc_commit(s_done);
-      }
-    }
     __syncthreads();
     ok = *abort_flag == 0;
     if (ok) ok = mbar_wait(s_done, ph, err, abort_flag);
@@ -418,8 +422,10 @@ __global__ void __launch_bounds__(BLK_THREADS, 1)
                    idesc, (c > 0 || t > 0 || k > 0) ? 1u : 0u);
         tc_commit(pv_done);
         if (c + 1 < n_ch) {
-          // the V planes are free once this product is done
-          if (mbar_wait(pv_done, c & 1u, err, abort_flag)) {
+          // the next chunk's scores (their TMEM columns were read out before
+          // this chunk's softmax), then its V once this product is done
+          issue_s(c + 1);
+          if (*abort_flag == 0 && mbar_wait(pv_done, c & 1u, err, abort_flag)) {
             load_half(c + 1, 1, v_full);
             ++v_issued;
           } else {
