@@ -325,6 +325,16 @@ FDLLM_API int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k
 FDLLM_API int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev,
                          int N, int M, int K, int splits, int accumulate);
 
+/* fdllm_gemm with the decoder's own operand type on the bf16 model: w_dev
+ * [N, K] fp16 and x_dev the two-term fp16 pair rows (hi = fp16(x),
+ * lo = fp16(x - hi)) in the layout described for fdllm_gemm; the same
+ * kernels, tile plans, splits and float y.  The bf16 model's decoder keeps
+ * its weights and activations in exactly this form (bf16 weights are held
+ * as the fp16 values equal to them).  Errors: ARG (also on the fp32 model),
+ * CUDA, TIMEOUT. */
+FDLLM_API int fdllm_gemm_f16(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev,
+                             int N, int M, int K, int splits, int accumulate);
+
 /* Kernel-level check of the decoder's attention over the ctx's KV cache:
  * o = softmax(q K^T / sqrt(head_dim)) V with keys [0, L) of layer `layer`
  * (as left by the last forward), no mask.  fp32 model: q_dev [M, n_heads,

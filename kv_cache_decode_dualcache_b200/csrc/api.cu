@@ -2076,9 +2076,17 @@ int fdllm_read_kv(fdllm_ctx* ctx, int layer, int pos0, int n, float* k_out, floa
   return FDLLM_OK;
 }
 
-int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
-               int K, int splits, int accumulate) {
+}  // extern "C"
+
+namespace {
+
+// fdllm_gemm (operand_f16 false: bf16 operands) and fdllm_gemm_f16 (true:
+// the decoder's fp16 operands, bf16 model only).
+int gemm_entry(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
+               int K, int splits, int accumulate, bool operand_f16) {
   if (!ctx) return FDLLM_ERR_ARG;
+  if (operand_f16 && !ctx->tc)
+    return fail(ctx, FDLLM_ERR_ARG, "fp16 operands need the bf16 model's tensor-core path");
   if (!w_dev || !x_dev || !y_dev || N < 1 || M < 1 || K < 1)
     return fail(ctx, FDLLM_ERR_ARG, "bad GEMM arguments");
   if (ctx->tc && (K % 64 || ((uintptr_t)w_dev | (uintptr_t)x_dev) % 16))
@@ -2119,9 +2127,9 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
                  2.0 * (ctx->tc ? 2 : 1) * M * N * K);
     if (ctx->tc) {
       CUtensorMap wm, xm;
-      gs.f16 = 0;  // bf16 operands (see the header)
-      if (!make_map(ctx, &wm, w_dev, N, K, 128, false) ||
-          !make_map(ctx, &xm, x_dev, pair_rows(M), K, pair ? 128 : gs.nt, false))
+      gs.f16 = operand_f16 ? 1 : 0;  // bf16 or fp16 operands (see the header)
+      if (!make_map(ctx, &wm, w_dev, N, K, 128, operand_f16) ||
+          !make_map(ctx, &xm, x_dev, pair_rows(M), K, pair ? 128 : gs.nt, operand_f16))
         return fail(ctx, FDLLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
       GemmScratch sc{ctx->ws, ctx->counters, ctx->err_dev, kWorkspaceBytes / sizeof(float),
                      ctx->n_counters};
@@ -2134,6 +2142,20 @@ int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_de
     }
   }
   return sync_state(ctx);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fdllm_gemm(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N, int M,
+               int K, int splits, int accumulate) {
+  return gemm_entry(ctx, w_dev, x_dev, y_dev, N, M, K, splits, accumulate, false);
+}
+
+int fdllm_gemm_f16(fdllm_ctx* ctx, const void* w_dev, const void* x_dev, float* y_dev, int N,
+                   int M, int K, int splits, int accumulate) {
+  return gemm_entry(ctx, w_dev, x_dev, y_dev, N, M, K, splits, accumulate, true);
 }
 
 int fdllm_attention(fdllm_ctx* ctx, const void* q_dev, void* o_dev, int layer, int M, int L) {

@@ -30,7 +30,7 @@ DTYPES = {"fp32": 0, "bf16": 1}
 EXPORTED = ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
             "fdllm_generate_batch", "fdllm_generate_fixed_k",
             "fdllm_step_debug", "fdllm_read_kv", "fdllm_kv_similarity", "fdllm_selftest_wait_timeout",
-            "fdllm_gemm", "fdllm_attention",
+            "fdllm_gemm", "fdllm_gemm_f16", "fdllm_attention",
             "fdllm_gemm_noalloc", "fdllm_profile_enable", "fdllm_profile_read",
             "fdllm_last_error", "fdllm_launch_count", "fdllm_inexact_weight_count",
             "fdllm_destroy")
@@ -116,6 +116,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                         P(ctypes.c_double)]
     lib.fdllm_selftest_wait_timeout.argtypes = [vp]
     lib.fdllm_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32]
+    lib.fdllm_gemm_f16.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32]
     lib.fdllm_attention.argtypes = [vp, vp, vp, i32, i32, i32]
     lib.fdllm_gemm_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
     lib.fdllm_profile_enable.argtypes = [vp, i32]
@@ -130,7 +131,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fdllm_create", "fdllm_load_weights", "fdllm_generate", "fdllm_generate_device",
                  "fdllm_generate_batch", "fdllm_generate_fixed_k", "fdllm_step_debug", "fdllm_read_kv",
                  "fdllm_kv_similarity", "fdllm_selftest_wait_timeout", "fdllm_gemm",
-                 "fdllm_attention", "fdllm_gemm_noalloc",
+                 "fdllm_gemm_f16", "fdllm_attention", "fdllm_gemm_noalloc",
                  "fdllm_profile_enable", "fdllm_profile_read", "fdllm_destroy"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -330,6 +331,20 @@ def fdllm_gemm(ctx, w_dev, x_dev, y_dev, splits: int = 0, accumulate: bool = Fal
         raise ValueError(f"x_dev must be a contiguous [{need}, {K}] tensor")
     _check(load_library().fdllm_gemm(ctx, w_dev.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(), N,
                                      M, K, splits, int(accumulate)), ctx)
+
+
+def fdllm_gemm_f16(ctx, w_dev, x_dev, y_dev, splits: int = 0, accumulate: bool = False) -> None:
+    """fdllm_gemm with fp16 operands (bf16 model): w_dev [N, K] float16, x_dev
+    the two-term float16 pair rows [2*ceil(M/32)*32, K]; y_dev [M, N] float32."""
+    N, K = w_dev.shape
+    M = int(y_dev.shape[0])
+    if tuple(y_dev.shape) != (M, N) or not y_dev.is_contiguous():
+        raise ValueError("y_dev must be a contiguous [M, N] tensor")
+    need = _pair_rows(M)
+    if x_dev.shape[0] < need or x_dev.shape[1] != K or not x_dev.is_contiguous():
+        raise ValueError(f"x_dev must be a contiguous [{need}, {K}] tensor")
+    _check(load_library().fdllm_gemm_f16(ctx, w_dev.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(),
+                                         N, M, K, splits, int(accumulate)), ctx)
 
 
 def fdllm_gemm_noalloc(w_dev, x_dev, y_dev, splits: int = 0, stream=None) -> None:

@@ -10,14 +10,15 @@ def split(x: torch.Tensor, dtype=torch.bfloat16):
     return hi, lo
 
 
-def pair_rows(x: torch.Tensor) -> torch.Tensor:
-    """[M, K] float -> [2*ceil(M/32)*32, K] bf16: per group of 32 tokens the
-    32 hi rows, then the 32 lo rows."""
+def pair_rows(x: torch.Tensor, dtype=torch.bfloat16) -> torch.Tensor:
+    """[M, K] float -> [2*ceil(M/32)*32, K] of dtype (bf16 for the stand-alone
+    GEMM, fp16 for the decoder's own form): per group of 32 tokens the 32 hi
+    rows, then the 32 lo rows."""
     M, K = x.shape
     G = (M + 31) // 32
     pad = torch.zeros(G * 32, K, device=x.device, dtype=x.dtype)
     pad[:M] = x
-    hi, lo = split(pad)
+    hi, lo = split(pad, dtype)
     return torch.stack([hi.view(G, 32, K), lo.view(G, 32, K)], dim=1).reshape(G * 64, K)
 
 

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from kv_cache_decode_dualcache_b200 import fdllm, synth
-from tests.bf16_layout import pair_rows
+from tests.bf16_layout import from_pair_rows, pair_rows
 from tests.gpu_util import make_decoder, require_gpu
 
 pytestmark = pytest.mark.gpu
@@ -78,6 +78,28 @@ def test_gemm_pair_agrees_with_single_sm(dec, dec_single, N, M, K, splits):
     assert torch.isfinite(ys[0]).all()
     scale = ys[1].abs().max().item()
     assert (ys[0] - ys[1]).abs().max().item() <= 1e-5 * scale
+
+
+@pytest.mark.parametrize("N,M,K,splits", [(128, 32, 64, 1), (1000, 17, 512, 1), (384, 32, 4096, 4),
+                                         (512, 100, 512, 0), (768, 129, 1024, 0),
+                                         (512, 200, 2048, 5), (12288, 512, 4096, 0)])
+def test_gemm_f16_operands_match_float64(dec, N, M, K, splits):
+    """The decoder's operand form: fp16 weights (N(0, 0.05), exact in fp16)
+    times two-term fp16 activations, against a float64 matmul of exactly
+    those values, on the single-SM and SM-pair kernels."""
+    g = torch.Generator(device="cuda").manual_seed(N * 11 + M * 5 + K)
+    w = (torch.randn(N, K, generator=g, device="cuda") * 0.05).to(torch.float16)
+    x = torch.randn(M, K, generator=g, device="cuda")
+    xp = pair_rows(x, torch.float16)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    fdllm.fdllm_gemm_f16(dec.ctx, w, xp, y, splits)
+    torch.cuda.synchronize()
+    xv = from_pair_rows(xp, M).double().cpu().numpy()     # the two-term value the kernel sees
+    ref = xv @ w.double().cpu().numpy().T
+    got = y.cpu().numpy()
+    assert np.isfinite(got).all()
+    tol = 2e-5 * np.sqrt(K) * np.abs(w.float().cpu().numpy()).max() * np.abs(xv).max()
+    assert np.abs(got - ref).max() <= tol
 
 
 def test_gemm_split_results_are_deterministic(dec):
