@@ -55,6 +55,11 @@ def test_counterexample_when_condition_fails():
     a = tuple(int(np.argmax(mm)) for mm in m)
     assert a == (0, 0)
     assert joint_argmax(t) != a
+    # by hand: revealing x1 first gives x1 = 0 (marginal 2/3 - d), then
+    # p(x2 = 1 | x1 = 0) = (1/3) / (2/3 - d) beats p(x2 = 0 | x1 = 0); the
+    # other order mirrors it
+    assert sequential_greedy(t, (0, 1)) == (0, 1)
+    assert sequential_greedy(t, (1, 0)) == (1, 0)
     par = generate(JointTableModel(t), [], 2, 2, 1 - eps, "none")
     assert tuple(par.tokens) == a            # parallel decoding returns the bad pair
     seq = generate(JointTableModel(t), [], 2, 2, 1.01, "none")
