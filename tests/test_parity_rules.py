@@ -58,6 +58,15 @@ def test_difference_within_1e3_of_tau_is_exempt_and_counted():
     assert not rep.mismatches and rep.exempt == 1 and rep.exempt_log
 
 
+def test_near_tau_exemption_covers_only_near_tau_positions():
+    # position 0 differs within 1e-3 of tau (exempt on its own), position 1
+    # differs far from it: the step fails
+    ref = _ref([0.9004, 0.95, 0.2], [True, True, False])
+    gpu = _gpu(ref, unmask=[False, False, False])
+    rep = _run(gpu, ref, [True, True, True])
+    assert rep.mismatches and rep.exempt == 0
+
+
 def test_fallback_pick_between_near_equal_candidates_is_exempt():
     # nothing reaches tau: the oracle picks position 2 (0.4003), the GPU position 0 (0.4)
     ref = _ref([0.4, 0.1, 0.4003], [False, False, True])
