@@ -411,6 +411,12 @@ def run_fdllm(args, wl):
     e2e_value = job_tokens_per_s(world, args.steps, G,
                                  max_over_ranks(e2.elapsed_time(e3), world, f"cuda:{local}"))
     steps_per_gen = e2e_steps / args.steps
+    # the device-resident call and the host-buffer call run the same decode:
+    # their tokens must be identical
+    same_tokens = bool(np.array_equal(np.asarray(tokens), np.asarray(out_host.numpy())))
+    if not same_tokens:
+        print("bench: device-resident and host-buffer generates returned different tokens",
+              file=sys.stderr)
     h2d = P * 4
     d2h = G * 4 + int(round(steps_per_gen)) * 20   # tokens + per-step state / error words
 
@@ -452,7 +458,8 @@ def run_fdllm(args, wl):
                            "steps_per_block": timing.steps_per_block,
                            "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
                            "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3),
-                           "tokens_checksum": int(np.asarray(tokens, dtype=np.int64).sum())},
+                           "tokens_checksum": int(np.asarray(tokens, dtype=np.int64).sum()),
+                           "tokens_match_host_call": same_tokens},
                 "block_step_roofline": (block_step_roofline(
                     wl, timing.cached_ms / timing.cached_steps, hbm)
                     if timing.cached_steps else None),   # cache off: every step is a refresh

@@ -48,6 +48,22 @@ def test_small_generate_path_matches_oracle(small, mode):
     assert not rep.mismatches, rep.mismatches[:5]
 
 
+@pytest.mark.parametrize("mode", ["dual", "prefix", "none"])
+def test_device_resident_generate_equals_the_host_call(small, mode):
+    # fdllm_generate_device (prompt and tokens in device memory; the call the
+    # benchmark times) runs the same decode as the host-buffer call
+    shape, dec, model = small
+    prompt = synth.make_prompt(shape, 40, salt=9).numpy()
+    host, steps, _ = dec.generate(prompt, 64, 32, 0.9, mode)
+    p_dev = torch.as_tensor(prompt, dtype=torch.int32).cuda()
+    out_dev = torch.full((64,), -1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    dev_steps = dec.generate_device(p_dev, 64, 32, 0.9, out_dev, mode)
+    torch.cuda.synchronize()
+    assert dev_steps == steps
+    np.testing.assert_array_equal(out_dev.cpu().numpy(), host)
+
+
 @pytest.mark.parametrize("shape", [LLADA_2L, DREAM_2L], ids=["llada8b-2layer", "dream7b-2layer"])
 def test_full_width_generate_path_matches_oracle(shape):
     # the LLaDA-8B / Dream-7B layer widths, vocabularies and head layouts
