@@ -69,3 +69,24 @@ def test_traffic_records_follow_their_kernel_sources():
             assert got == float(rec["bytes_per_launch"])
         else:                       # kernel changed since the counters were taken
             assert got is None
+
+
+def test_reference_arm_line_on_a_small_model():
+    # the float64 oracle's whole generate of the tiny workload, timed on the
+    # host cores: one JSON line with the contract's keys, not an estimate
+    import json
+    import subprocess
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["estimated"] is False
+    assert line["unit"] == "tokens/s" and line["value"] > 0 and line["higher_is_better"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"] == "tiny"
