@@ -231,6 +231,7 @@ def oracle_sample(wl, weights_host, step_counts, sample_layers=4):
     from kv_cache_decode_dualcache_b200 import synth
     from oracle.model import Model
 
+    sample_layers = min(sample_layers, wl.shape.n_layers)
     shape = synth.with_layers(wl.shape, sample_layers)
     w = {k: v for k, v in weights_host.items()
          if not k.startswith("layers.") or int(k.split(".")[1]) < sample_layers}
@@ -251,7 +252,8 @@ def oracle_sample(wl, weights_host, step_counts, sample_layers=4):
     n_ref, n_cached = step_counts
     total = scale * (n_ref * t_refresh + n_cached * t_step)
     return {"tok_s": G / total, "t_refresh_s": t_refresh * scale, "t_step_s": t_step * scale,
-            "sample_s": t_refresh + t_step, "threads": torch.get_num_threads()}
+            "sample_s": t_refresh + t_step, "threads": torch.get_num_threads(),
+            "layers": sample_layers}
 
 
 def oracle_full_generate(wl, weights_host, reps=1):
@@ -320,7 +322,7 @@ def run_reference(args, wl):
                              "sample": f"per step: one block-start full forward and one DualCache "
                                        f"block step of the first {sample_layers} of "
                                        f"{wl.shape.n_layers} layers, scaled x"
-                                       f"{wl.shape.n_layers // sample_layers}; "
+                                       f"{wl.shape.n_layers / sample_layers:g}; "
                                        f"{counts[0]} refresh + {counts[1]} cached steps"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -472,7 +474,8 @@ def run_fdllm(args, wl):
         r = oracle_sample(wl, w_host, (timing.refresh_steps, timing.cached_steps))
         cpu = {"value": r["tok_s"], "unit": "tokens/s", "cores": r["threads"], "kind": "oracle",
                "sample": "one block-start full forward and one DualCache block step of the "
-                         "first 4 of 32 layers (float64 oracle), scaled x8 and weighted by "
+                         f"first {r['layers']} of {wl.shape.n_layers} layers (float64 oracle), "
+                         f"scaled x{wl.shape.n_layers / r['layers']:g} and weighted by "
                          f"this run's {timing.refresh_steps} refresh + {timing.cached_steps} "
                          f"cached steps ({r['sample_s']:.1f} s of CPU work)",
                "t_refresh_s": round(r["t_refresh_s"], 3), "t_step_s": round(r["t_step_s"], 3)}

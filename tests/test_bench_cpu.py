@@ -90,3 +90,14 @@ def test_reference_arm_line_on_a_small_model():
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == "tiny"
+
+
+def test_oracle_sample_clamps_its_depth_to_the_model():
+    # a model with fewer layers than the 4-layer sample runs all of them,
+    # unscaled
+    wl = synth.WORKLOADS["tiny"]
+    w = {k: v.cpu() for k, v in synth.make_weights(wl.shape, device="cpu").items()}
+    r = bench.oracle_sample(wl, w, (4, 10))
+    assert r["layers"] == wl.shape.n_layers == 2
+    assert abs(r["t_refresh_s"] + r["t_step_s"] - r["sample_s"]) < 1e-12
+    assert r["tok_s"] > 0
