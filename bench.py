@@ -168,6 +168,59 @@ def block_step_roofline(wl, cached_ms, hbm):
             "note": "weights (bf16) + K,V of all L positions read once per block step"}
 
 
+def generate_roofline(wl, steps_per_block, value, hbm, tf):
+    """Whole-generate roofline: every executed step at the slower of its
+    algorithmic bytes / HBM bandwidth and its FLOPs / tensor peak; gen_len
+    over the sum is the roofline tokens/s, and the measured tokens/s is a
+    fraction of it.  A block's first step (every step without a cache) is a
+    full forward over all L rows; a DualCache step runs the block rows, a
+    prefix-cache step rows [s, L), both over the K/V of all L positions.
+    Bytes: the weights once and the K/V of all positions once per step;
+    FLOPs: 2 x weights x rows (the LM head on the block rows only) plus
+    4 x rows x L x H x hd per layer of attention.  Single-sequence bf16
+    workloads only (None for batches and for the fp32 model)."""
+    from kv_cache_decode_dualcache_b200 import synth
+    if wl.batch != 1 or not steps_per_block or wl.shape.dtype == "fp32":
+        return None   # the fp32 model lives in L2 and runs no tensor-core path
+    sh = wl.shape
+    P, G, B = wl.prompt_len, wl.gen_len, wl.block_size
+    L = P + G
+    es = sh.elem_bytes
+    head = sh.vocab * sh.d_model
+    layers = synth.step_weight_params(sh) - head
+    bytes_step = es * (layers + head) + es * 2 * sh.n_layers * L * sh.n_kv_heads * sh.head_dim
+
+    def flops(rows):
+        return (2.0 * layers * rows + 2.0 * head * B
+                + 4.0 * rows * L * sh.n_heads * sh.head_dim * sh.n_layers)
+
+    def step_s(rows, bw, pk):
+        return max(bytes_step / bw, flops(rows) / pk)
+
+    peaks = {"nominal": (8e12, 2.25e15), "measured": (hbm * 1e9, tf * 1e12)}
+    out = {"steps": {"full": 0, "cached": 0}, "tokens_per_s": {}, "frac": {},
+           "full_step_ms": {}, "block_step_ms": {}}
+    for b, n in enumerate(steps_per_block):
+        out["steps"]["full"] += 1 if wl.cache_mode != "none" else n
+        out["steps"]["cached"] += n - 1 if wl.cache_mode != "none" else 0
+    for name, (bw, pk) in peaks.items():
+        total = 0.0
+        for b, n in enumerate(steps_per_block):
+            s = P + b * B
+            cached_rows = {"dual": B, "prefix": L - s}.get(wl.cache_mode)
+            if cached_rows is None:
+                total += n * step_s(L, bw, pk)
+            else:
+                total += step_s(L, bw, pk) + (n - 1) * step_s(cached_rows, bw, pk)
+        out["tokens_per_s"][name] = round(G / total, 2)
+        out["frac"][name] = round(value / (G / total), 4)
+        out["full_step_ms"][name] = round(1e3 * step_s(L, bw, pk), 3)
+        out["block_step_ms"][name] = round(1e3 * step_s(B, bw, pk), 3)
+    out["peaks"] = {"nominal": "8 TB/s, 2.25 PFLOP/s dense bf16",
+                    "measured": f"{hbm:g} GB/s copy, {tf:g} TFLOP/s sustained bf16 GEMM"}
+    return out
+
+
 def _traffic_record(record, source):
     """ncu DRAM bytes per launch recorded in profiles/<record> for the current
     source of the kernel (csrc/<source>), if any: null once the kernel has
@@ -492,6 +545,8 @@ def run_fdllm(args, wl):
                            "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3),
                            "tokens_checksum": int(np.asarray(tokens, dtype=np.int64).sum()),
                            "tokens_match_host_call": same_tokens},
+                "generate_roofline": generate_roofline(wl, timing.steps_per_block, value, hbm,
+                                                       tf_sust),
                 "block_step_roofline": (block_step_roofline(
                     wl, timing.cached_ms / timing.cached_steps, hbm)
                     if timing.cached_steps else None),   # cache off: every step is a refresh

@@ -101,3 +101,43 @@ def test_oracle_sample_clamps_its_depth_to_the_model():
     assert r["layers"] == wl.shape.n_layers == 2
     assert abs(r["t_refresh_s"] + r["t_step_s"] - r["sample_s"]) < 1e-12
     assert r["tok_s"] > 0
+
+
+def test_generate_roofline_of_the_headline_workload():
+    wl = synth.WORKLOADS["llada8b-p256-g256"]
+    spb = [1, 3, 3, 3, 4, 4, 4, 4]                      # 8 refresh + 18 block steps
+    r = bench.generate_roofline(wl, spb, 1000.0, 6549.0, 1381.7)
+    assert r["steps"] == {"full": 8, "cached": 18}
+    # a block step is HBM-bound: the same bytes as block_step_roofline
+    b = bench.block_step_roofline(wl, 1.0, 6549.0)["bytes_per_step"]
+    assert abs(r["block_step_ms"]["nominal"] - 1e3 * b / 8e12) < 1e-3
+    assert abs(r["block_step_ms"]["measured"] - 1e3 * b / 6549e9) < 1e-3
+    # a full forward over L = 512 rows is tensor-bound: 2 x layer weights x L
+    # + 2 x LM head x B + 4 L^2 H hd per layer
+    sh = wl.shape
+    head = sh.vocab * sh.d_model
+    layers = synth.step_weight_params(sh) - head
+    fl = 2 * layers * 512 + 2 * head * 32 + 4 * 512 * 512 * 32 * 128 * 32
+    assert abs(r["full_step_ms"]["nominal"] - 1e3 * fl / 2.25e15) < 1e-3
+    total = 8 * fl / 2.25e15 + 18 * b / 8e12
+    assert abs(r["tokens_per_s"]["nominal"] - 256 / total) < 0.01
+    assert abs(r["frac"]["nominal"] - 1000.0 / (256 / total)) < 1e-4
+
+
+def test_generate_roofline_cache_modes():
+    wl = synth.WORKLOADS["llada8b-p256-g256"]
+    none = bench.generate_roofline(type(wl)(**{**wl.__dict__, "cache_mode": "none"}),
+                                   [3] * 8, 100.0, 6549.0, 1381.7)
+    assert none["steps"] == {"full": 24, "cached": 0}
+    pre = bench.generate_roofline(type(wl)(**{**wl.__dict__, "cache_mode": "prefix"}),
+                                  [3] * 8, 100.0, 6549.0, 1381.7)
+    dual = bench.generate_roofline(wl, [3] * 8, 100.0, 6549.0, 1381.7)
+    # the same step counts cost most without a cache, least with DualCache;
+    # a prefix step over at most 256 rows costs a DualCache step's bytes, and
+    # is HBM-bound at the nominal peaks (ridge 281 FLOP/B) but tensor-bound at
+    # the measured ones (ridge 211 FLOP/B)
+    assert none["tokens_per_s"]["nominal"] < pre["tokens_per_s"]["nominal"]
+    assert pre["tokens_per_s"]["nominal"] == dual["tokens_per_s"]["nominal"]
+    assert pre["tokens_per_s"]["measured"] < dual["tokens_per_s"]["measured"]
+    assert bench.generate_roofline(synth.WORKLOADS["llada8b-batch16"], [3] * 8, 1.0, 1.0,
+                                   1.0) is None
