@@ -83,9 +83,12 @@ typedef enum {
 } fdllm_dtype;
 
 /* Model shape and numerics.  Requirements (FDLLM_ERR_ARG otherwise):
- * n_layers >= 1; d_model, ffn_dim and n_heads*head_dim multiples of 64;
- * head_dim in {32, 64, 128}; n_heads a multiple of n_kv_heads;
- * 0 <= mask_id < vocab; vocab >= 2; max_seq >= 1; 1 <= max_batch <= 64. */
+ * n_layers >= 1; d_model a multiple of 64 in [64, 8192]; ffn_dim and
+ * n_heads*head_dim multiples of 64; head_dim in {32, 64, 128} (bf16: 64 or
+ * 128, and n_kv_heads*head_dim a multiple of 64); n_heads a multiple of
+ * n_kv_heads; 0 <= mask_id < vocab; vocab >= 2; 1 <= max_seq <= 2^20;
+ * 1 <= max_batch <= 64; rope_theta finite and > 0, rms_eps >= 0,
+ * logit_scale finite. */
 typedef struct {
   int32_t n_layers;
   int32_t d_model;
