@@ -60,6 +60,22 @@ def test_create_rejects_bad_configs_without_a_device(lib):
     cfg.n_heads = 16
     assert lib.fdllm_create(ctypes.byref(cfg), 0, None, None, ctypes.byref(ctx)) == \
         fdllm.FDLLM_ERR_ARG
+    # the remaining limits the header states for fdllm_config
+    more = {"d_model": 8256, "max_seq": 0, "max_batch": 65, "rope_theta": 0.0,
+            "rms_eps": -1.0, "logit_scale": float("nan")}
+    for field, value in more.items():
+        cfg = fdllm.make_config(good, 96)
+        setattr(cfg, field, value)
+        assert lib.fdllm_create(ctypes.byref(cfg), 0, None, None, ctypes.byref(ctx)) == \
+            fdllm.FDLLM_ERR_ARG, field
+        assert b"device" not in lib.fdllm_last_error(None), field
+    cfg = fdllm.make_config(good, (1 << 20) + 1)
+    assert lib.fdllm_create(ctypes.byref(cfg), 0, None, None, ctypes.byref(ctx)) == \
+        fdllm.FDLLM_ERR_ARG
+    cfg = fdllm.make_config(good, 96)
+    cfg.n_heads, cfg.n_kv_heads = 3, 3                  # 3 x 32 is not a multiple of 64
+    assert lib.fdllm_create(ctypes.byref(cfg), 0, None, None, ctypes.byref(ctx)) == \
+        fdllm.FDLLM_ERR_ARG
 
 
 def test_null_ctx_calls_are_rejected(lib):
