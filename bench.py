@@ -463,14 +463,16 @@ def run_fdllm(args, wl):
     steps_total = 0
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    # one event between generations (the call returns once its work is done)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
         steps_total += dec.generate_device(prompt_dev, G, B, tau, out_dev, wl.cache_mode)
-    e1.record(stream)
+        evs[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
+    ms = evs[0].elapsed_time(evs[-1])
+    per_gen = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps))
     launches = dec.launch_count(reset=True)
     clocks = sampler.stop() if sampler else None
     ms_max = max_over_ranks(ms, world, f"cuda:{local}")
@@ -540,6 +542,9 @@ def run_fdllm(args, wl):
                 "scaling": "weak", "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
                 "config": _config(wl, world),
                 "decode": {"denoising_steps_per_generation": steps_total / args.steps,
+                           "ms_per_generation": {"median": round(per_gen[len(per_gen) // 2], 3),
+                                                 "min": round(per_gen[0], 3),
+                                                 "max": round(per_gen[-1], 3)},
                            "steps_per_block": timing.steps_per_block,
                            "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
                            "cached_ms_per_step": round(timing.cached_ms / max(1, timing.cached_steps), 3),
