@@ -64,6 +64,15 @@ def _dtype(wl):
     return "f32" if wl.shape.dtype == "fp32" else "bf16"
 
 
+def _arithmetic(wl):
+    """What the kernels compute in, beside the model dtype of `dtype`."""
+    if wl.shape.dtype == "fp32":
+        return "f32 on CUDA cores (f32 weights and activations)"
+    return ("bf16 weights held as f16 (exact for |w| >= 2^-17); tensor-core products on f16 "
+            "operands with f32 accumulation; activations, q, K/V and softmax weights stored "
+            "as two f16 terms (hi + lo); f32 residual stream, norms and softmax")
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
 
@@ -539,7 +548,8 @@ def run_fdllm(args, wl):
         line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": _dtype(wl), "arithmetic": _arithmetic(wl),
+                "data": "synthetic",
                 "config": _config(wl, world),
                 "decode": {"denoising_steps_per_generation": steps_total / args.steps,
                            "ms_per_generation": {"median": round(per_gen[len(per_gen) // 2], 3),
@@ -636,7 +646,8 @@ def run_fdllm_batch(args, wl):
         line = {"metric": metric_name(wl), "value": round(value, 2), "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "arithmetic": _arithmetic(wl), "data": "synthetic",
                 "config": cfg,
                 "decode": {"denoising_steps_per_generation": int(np.asarray(steps).sum()),
                            "refresh_ms_per_step": round(timing.refresh_ms / max(1, timing.refresh_steps), 3),
