@@ -340,12 +340,16 @@ FDLLM_API int fdllm_gemm_f16(fdllm_ctx* ctx, const void* w_dev, const void* x_de
 
 /* Kernel-level check of the decoder's attention over the ctx's KV cache:
  * o = softmax(q K^T / sqrt(head_dim)) V with keys [0, L) of layer `layer`
- * (as left by the last forward), no mask.  fp32 model: q_dev [M, n_heads,
+ * (as left by the last forward), no mask: the bidirectional attention of
+ * the block queries over cached prefix, block and cached suffix K/V
+ * (techwalker.com Fast-dLLM article, section "核心创新：适合扩散模型的KV缓存";
+ * ccyt168.com overview, section 一, item 1).  fp32 model: q_dev [M, n_heads,
  * head_dim] and o_dev [M, n_heads * head_dim] float.  bf16 model: q_dev is
  * two planes of fp16 [M, n_heads, head_dim] (hi terms, then lo terms) and
  * o_dev receives two-term fp16 rows of n_heads * head_dim in the 32-token
- * grouping described for fdllm_gemm (the decoder's storage format).  The same kernel choice (and key split
- * for M <= 64) as a decode step.  Errors: ARG, STATE, CUDA. */
+ * grouping described for fdllm_gemm (the decoder's storage format).  The
+ * same kernel choice (and key split for M <= 64) as a decode step.
+ * Errors: ARG, STATE, CUDA. */
 FDLLM_API int fdllm_attention(fdllm_ctx* ctx, const void* q_dev, void* o_dev, int layer, int M,
                               int L);
 
