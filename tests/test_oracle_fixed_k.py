@@ -19,6 +19,7 @@ def test_select_top_k_order_and_ties():
     assert list(np.flatnonzero(select_top_k(masked, conf, 1))) == [1]
     assert select_top_k(masked, conf, 9).tolist() == masked.tolist()
     assert not select_top_k(np.zeros(4, bool), conf[:4], 2).any()
+    assert not select_top_k(masked, conf, 0).any() and not select_top_k(masked, conf, -2).any()
     # k = 1 is the threshold rule's fallback pick
     assert np.array_equal(select_top_k(masked, conf, 1), select_unmask(masked, conf, 2.0))
 

@@ -84,3 +84,20 @@ def test_attention_equal_keys_average_all_values_bidirectionally():
     out = attention(q, k, v)
     for m in range(3):
         np.testing.assert_allclose(out[m, 0], v[:, 0, :].mean(axis=0), rtol=1e-13)
+
+
+def test_attention_is_stable_for_large_scores():
+    # scores of several thousand (far beyond exp's range) must give the same
+    # softmax as torch's float64 attention: the max shift is per query row
+    rng = np.random.default_rng(6)
+    M, L, H, hd = 5, 13, 2, 8
+    q = rng.standard_normal((M, H, hd)) * 300.0
+    k = rng.standard_normal((L, H, hd)) * 30.0
+    v = rng.standard_normal((L, H, hd))
+    qt = torch.from_numpy(q).permute(1, 0, 2)
+    kt = torch.from_numpy(k).permute(1, 0, 2)
+    vt = torch.from_numpy(v).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=False)
+    out = attention(q, k, v)
+    assert np.isfinite(out).all()
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=1e-9, atol=1e-9)

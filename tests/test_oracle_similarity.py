@@ -23,6 +23,18 @@ def test_closed_forms():
     np.testing.assert_allclose(c[0, 1], [1.0, 1.0, 1.0, 1.0], atol=1e-15)
 
 
+def test_invariant_to_positive_scale_at_any_norm():
+    # cos(s a, t b) = cos(a, b) for s, t > 0, also when the norms' product is
+    # below 1 (K/V of N(0, 0.02) weights have small norms)
+    rng = np.random.default_rng(7)
+    a = rng.standard_normal((6, 2, 4))
+    b = rng.standard_normal((6, 2, 4))
+    ref = kv_cosine(_kv(a, b), _kv(b, a))
+    for s, t in ((1e-3, 1.0), (1e-3, 2e-4), (50.0, 1e-2)):
+        np.testing.assert_allclose(kv_cosine(_kv(s * a, t * b), _kv(t * b, s * a)), ref,
+                                   rtol=1e-12, atol=1e-14)
+
+
 def test_zero_vectors():
     z = np.zeros((2, 1, 3))
     nz = np.ones((2, 1, 3))
