@@ -52,6 +52,32 @@ def test_replay_of_the_oracles_own_decisions_passes(tiny, prompt, mode):
     rep = replay_gpu_trace(tiny, prompt, G, B, TAU, mode, res.tokens, st)
     assert rep.steps == res.steps
     assert not rep.mismatches and rep.exempt == 0
+    assert rep.max_dconf < 1e-6                       # float32 rounding of the trace only
+
+
+def test_replay_limits_the_compared_steps(tiny, prompt):
+    res, st = _run(tiny, prompt, "dual")
+    one = replay_gpu_trace(tiny, prompt, G, B, TAU, "dual", res.tokens, st, max_steps_per_block=1)
+    assert one.steps == G // B and not one.mismatches
+    two = replay_gpu_trace(tiny, prompt, G, B, TAU, "dual", res.tokens, st, max_steps_per_block=2)
+    assert two.steps == sum(min(2, n) for n in res.steps_per_block) and not two.mismatches
+    only = replay_gpu_trace(tiny, prompt, G, B, TAU, "dual", res.tokens, st, blocks={1})
+    assert only.steps == res.steps_per_block[1] and not only.mismatches
+
+
+def test_replay_catches_a_block_left_with_masked_positions(tiny, prompt):
+    # block 1's last step is dropped from the trace: block 2 starts while
+    # block 1 still holds the mask id
+    res, st = _run(tiny, prompt, "dual")
+    last0 = int(np.flatnonzero(st.trace_block == 1)[-1])
+    keep = np.ones(len(st.trace_block), bool)
+    keep[last0] = False
+    cut = SimpleNamespace(trace_block=st.trace_block[keep], trace_conf=st.trace_conf[keep],
+                          trace_tok=st.trace_tok[keep], trace_unmask=st.trace_unmask[keep])
+    tokens = res.tokens.copy()
+    tokens[B + np.flatnonzero(res.trace[last0].unmask)] = MASK
+    rep = replay_gpu_trace(tiny, prompt, G, B, TAU, "dual", tokens, cut)
+    assert any("block 1 left masked positions" in m for m in rep.mismatches)
 
 
 def _first_cached_step(res):
@@ -164,3 +190,9 @@ def test_teacher_forced_driver(tiny, prompt, mode):
     bad_c = teacher_forced(_OracleStandIn(tiny, dconf=2e-3), tiny, ref.trace, prompt, G, B, TAU,
                            mode, MASK, z_tol=1e-4)
     assert any("conf" in m for m in bad_c.mismatches)
+    some = teacher_forced(_OracleStandIn(tiny), tiny, ref.trace, prompt, G, B, TAU, mode, MASK,
+                          z_tol=1e-4, max_steps=2)
+    assert some.steps == 2 and not some.mismatches
+    every3 = teacher_forced(_OracleStandIn(tiny), tiny, ref.trace, prompt, G, B, TAU, mode, MASK,
+                            z_tol=1e-4, stride=3)
+    assert every3.steps == -(-ref.steps // 3) and not every3.mismatches

@@ -8,7 +8,7 @@ oracle had no position reaching tau.
 """
 import numpy as np
 
-from tests.parity import StepReport, compare_step
+from tests.parity import StepReport, compare_step, top2_margin
 
 MASK = 7
 TAU = 0.9
@@ -103,3 +103,31 @@ def test_confidence_tolerance():
     ref = _ref([0.5, 0.6], [False, True])
     assert _run(_gpu(ref, conf=[0.5, 0.6011]), ref, [True, True]).mismatches
     assert not _run(_gpu(ref, conf=[0.5, 0.6009]), ref, [True, True]).mismatches
+
+
+def test_exemptions_stop_at_1e3():
+    # 1.5e-3 from tau is not a near-tau difference
+    ref = _ref([0.9015, 0.95, 0.2], [True, True, False])
+    gpu = _gpu(ref, unmask=[False, True, False])
+    rep = _run(gpu, ref, [True, True, True])
+    assert rep.mismatches and rep.exempt == 0
+
+
+def test_top2_margin_is_the_gap_between_the_two_largest_non_mask_logits():
+    rng = np.random.default_rng(8)
+    for width in (8, 1000):                  # a vocabulary-sized row as well
+        z = rng.standard_normal((40, width))
+        srt = np.sort(np.delete(z, MASK, axis=1), axis=1)
+        np.testing.assert_array_equal(top2_margin(z, MASK), srt[:, -1] - srt[:, -2])
+        z[:, MASK] = 100.0                   # the mask id's logit never counts
+        np.testing.assert_array_equal(top2_margin(z, MASK), srt[:, -1] - srt[:, -2])
+
+
+def test_report_summary_and_maxima():
+    ref = _ref([0.9004, 0.95, 0.2], [True, True, False])
+    gpu = _gpu(ref, unmask=[False, True, False], conf=[0.9004, 0.9502, 0.2])
+    rep = _run(gpu, ref, [True, True, True])
+    assert abs(rep.max_dconf - 2e-4) < 1e-12 and rep.max_dz == 0.0
+    text = rep.summary()
+    assert text.startswith("1 steps, ") and "exemptions 1 (" in text
+    assert StepReport().summary() == "0 steps, max|dz| 0, max|dconf| 0, exemptions 0"
