@@ -49,3 +49,27 @@ def test_bf16_weights_are_the_rounded_float32_draw():
     gen = torch.Generator().manual_seed(shape.seed)
     first = torch.empty(synth.weight_shapes(shape)["embed"]).normal_(0.0, 0.02, generator=gen)
     assert torch.equal(w["embed"], first.to(torch.bfloat16))
+
+
+def test_prompt_and_length_draws_are_the_stated_generators():
+    # prompts: ids uniform in [0, vocab - 2] from a CPU generator seeded with
+    # 1000 + model seed + salt; batch lengths: uniform in [128, 1024] from one
+    # seeded with 3
+    for shape, salt in ((synth.TINY, 0), (synth.LLADA_8B, 0), (synth.LLADA_8B, 5)):
+        gen = torch.Generator().manual_seed(1000 + shape.seed + salt)
+        want = torch.randint(0, shape.vocab - 1, (64,), generator=gen, dtype=torch.int64)
+        assert torch.equal(synth.make_prompt(shape, 64, salt=salt), want.to(torch.int32))
+    gen = torch.Generator().manual_seed(3)
+    assert synth.make_batch_prompt_lengths(16) == \
+        [int(v) for v in torch.randint(128, 1025, (16,), generator=gen)]
+
+
+def test_batched_workload_lengths_are_the_recorded_ones():
+    # the 16 prompt lengths this generator gave the batched workload when its
+    # measurements were taken (listed beside them in the design notes)
+    assert synth.make_batch_prompt_lengths(16) == [1014, 199, 510, 989, 570, 1022, 419, 988, 789,
+                                                   615, 588, 323, 913, 952, 341, 552]
+
+
+def test_element_sizes():
+    assert synth.TINY.elem_bytes == 4 and synth.LLADA_8B.elem_bytes == 2
