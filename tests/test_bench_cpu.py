@@ -30,6 +30,13 @@ def test_hbm_bound_class_dominates():
     assert abs(r["frac"] - 0.5) < 1e-9
     assert r["traffic"] == 123.0 and r["launches"] == 33
     assert abs(r["share_of_kernel_time"] - 100.0 / 150.0) < 1e-3
+    assert r["algorithmic_bytes_per_launch"] == round(300e9 / 33)
+    assert r["kernel"].startswith("chain_kernel") and r["peak_source"] == "measured"
+    # per class: bytes and FLOPs over its own time
+    assert r["classes"]["chain.step"] == {"launches": 33, "ms": 100.0, "GBps": 3000.0,
+                                          "TFps": 0.0}
+    assert r["classes"]["gemm.qkv.full"]["TFps"] == 500.0
+    assert r["classes"]["attn.step"]["GBps"] == 50.0
 
 
 def test_tensor_bound_class_dominates():
@@ -39,6 +46,7 @@ def test_tensor_bound_class_dominates():
     r = bench.roofline_from_profile(stats, 6000.0, 1400.0, "measured",
                                     {"step": 123.0, "full": None})
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["kernel"].startswith("gemm_tc2_kernel") and r["launches"] == 64
     assert abs(r["achieved"] - 60.0 / 0.1) < 1e-6       # 60 TFLOP in 100 ms
     assert abs(r["frac"] - 600.0 / 1400.0) < 1e-4
     assert r["traffic"] is None                          # no capture of this class
@@ -53,6 +61,7 @@ def test_block_step_roofline_of_the_headline_workload():
     # weights of one block step (bf16) + K and V of all 512 positions
     want = 2 * synth.step_weight_params(wl.shape) + 32 * 512 * 32 * 128 * 2 * 2
     assert r["bytes_per_step"] == want
+    assert r["ms_per_step"] == 4.0 and r["achieved_GBps"] == round(want / 4e-3 / 1e9, 1)
     assert abs(r["frac_of_8TBps"] - want / 4e-3 / 8e12) < 1e-4
     assert abs(r["frac_of_measured"] - want / 4e-3 / 6e12) < 1e-4
 
@@ -100,7 +109,16 @@ def test_oracle_sample_clamps_its_depth_to_the_model():
     r = bench.oracle_sample(wl, w, (4, 10))
     assert r["layers"] == wl.shape.n_layers == 2
     assert abs(r["t_refresh_s"] + r["t_step_s"] - r["sample_s"]) < 1e-12
-    assert r["tok_s"] > 0
+    assert 0 < r["t_refresh_s"] < 60 and 0 < r["t_step_s"] < 60
+    # generated tokens over the weighted, depth-scaled step times
+    assert abs(r["tok_s"] - 64 / (4 * r["t_refresh_s"] + 10 * r["t_step_s"])) < 1e-9 * r["tok_s"]
+    # a deeper model: the first 4 layers, scaled to its depth
+    deep = synth.with_layers(synth.TINY, 6)
+    wl6 = type(wl)(**{**wl.__dict__, "shape": deep})
+    w6 = {k: v.cpu() for k, v in synth.make_weights(deep, device="cpu").items()}
+    r6 = bench.oracle_sample(wl6, w6, (4, 10))
+    assert r6["layers"] == 4
+    assert abs(r6["t_refresh_s"] + r6["t_step_s"] - 1.5 * r6["sample_s"]) < 1e-12
 
 
 def test_generate_roofline_of_the_headline_workload():
@@ -141,3 +159,18 @@ def test_generate_roofline_cache_modes():
     assert pre["tokens_per_s"]["measured"] < dual["tokens_per_s"]["measured"]
     assert bench.generate_roofline(synth.WORKLOADS["llada8b-batch16"], [3] * 8, 1.0, 1.0,
                                    1.0) is None
+    # exact totals: cache off = 24 full forwards; prefix = per block one full
+    # forward and two steps over rows [s, L) (tensor-bound at the measured
+    # peaks once the rows pass the ridge)
+    full = [none["full_step_ms"][k] for k in ("nominal", "measured")]
+    assert abs(none["tokens_per_s"]["nominal"] - 256 / (24 * full[0] * 1e-3)) < 1.0
+    sh = wl.shape
+    head = sh.vocab * sh.d_model
+    layers = synth.step_weight_params(sh) - head
+    step_bytes = 2 * (layers + head) + 2 * 2 * sh.n_layers * 512 * sh.n_kv_heads * sh.head_dim
+
+    def t(rows):
+        fl = 2.0 * layers * rows + 2.0 * head * 32 + 4.0 * rows * 512 * 32 * 128 * 32
+        return max(step_bytes / 6549e9, fl / 1381.7e12)
+    want = sum(t(512) + 2 * t(512 - (256 + 32 * b)) for b in range(8))
+    assert abs(pre["tokens_per_s"]["measured"] - 256 / want) < 0.01
